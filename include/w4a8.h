@@ -1,0 +1,161 @@
+/*
+ * libw4a8 -- block-quantized W4A8 matmul y = x . W^T on one NVIDIA B200 (sm_100a).
+ *
+ * Weights are stored as Q4_0 (4-bit codes in blocks of 32 along K with one fp16 scale
+ * per block); activations are quantised on the fly to Q8_0 (int8 codes in blocks of 32
+ * with one f32 scale per block). Each 32-wide block dot product is computed exactly in
+ * integer arithmetic and then rescaled by the two block scales and accumulated in f32.
+ * Sources: tract PR #2432 "W4A8 (Q4_0 int8-dot) path for block_quant", sections
+ * "Pipeline" (4-bit N x K weight, activation to int8 per block) and "The kernel"
+ * (per-32-block weight scales, per-block f32 rescale, no per-op allocation wanted);
+ * and for the affine variant, MLX PR #4802 "mx.qqmm ... mode=affine" (int8 MMA on the
+ * original 4-bit codes, per-group scales and biases applied in the kernel).
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer argument is DEVICE memory owned by the caller; the library never
+ *    allocates, frees or keeps a pointer after the call returns. Pointers must be
+ *    16-byte aligned (W4A8_ERR_MISALIGNED otherwise).
+ *  - All work is enqueued asynchronously on `stream` (0 = the legacy default stream).
+ *    The returned status covers argument checks and launch errors only; a fault inside
+ *    a kernel surfaces at the caller's next synchronisation.
+ *  - Matrices are dense row-major with no padding: x is M x K, W is N x K ("N x K" as
+ *    on the tract page), y is M x N (f32).
+ *  - The kernels never trap, assert or wait without bound. Every internal wait has a
+ *    time limit; when one runs out the kernel records W4A8_ERR_DEVICE_TIMEOUT in a
+ *    device status word (read it with w4a8_last_device_error) and exits cleanly.
+ */
+#ifndef W4A8_H_
+#define W4A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A8_OK = 0,
+    W4A8_ERR_INVALID_ARG = 1,    /* null pointer, non-positive or too large size, K % 32 != 0 */
+    W4A8_ERR_UNSUPPORTED = 2,    /* a mode the kernels do not implement (dtype, group size, path) */
+    W4A8_ERR_WORKSPACE = 3,      /* workspace pointer null or smaller than w4a8_workspace_bytes() */
+    W4A8_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed */
+    W4A8_ERR_DEVICE_TIMEOUT = 5, /* a bounded wait inside a kernel ran out (see w4a8_last_device_error) */
+    W4A8_ERR_MISALIGNED = 6      /* a pointer is not 16-byte aligned */
+} w4a8_status;
+
+/* Element type of the unquantised input (x or W). bf16 is widened exactly to f32. */
+typedef enum { W4A8_F32 = 0, W4A8_BF16 = 1 } w4a8_dtype;
+
+/* Which kernel path a matmul takes. AUTO chooses by M (small M streams the weights
+ * once with a dp4a GEMV; larger M runs the tcgen05 tensor-core GEMM). */
+typedef enum { W4A8_PATH_AUTO = 0, W4A8_PATH_GEMV = 1, W4A8_PATH_GEMM = 2 } w4a8_path;
+
+/* Largest M, N or K any entry point accepts (keeps every byte offset inside int64 and
+ * every per-row count inside int32). */
+#define W4A8_MAX_DIM (1 << 20)
+
+/*
+ * Q4_0 weight pack (once per weight; not part of the per-call matmul).
+ * w      : N x K row-major, f32 or bf16 (`dtype`).
+ * qs     : out, N x K/2 bytes. Row n, block b occupies bytes [n*K/2 + 16b, +16); byte j of
+ *          a block holds the code of element 32b+j in its low nibble and of element
+ *          32b+j+16 in its high nibble.
+ * d_fp16 : out, N x K/32 fp16 bit patterns, the scale of each block.
+ * Per block: mx = the element of largest magnitude (first on ties), d = mx / -8 (f32),
+ * q = min(15, trunc(x * (1/d) + 8.5)) (0 when d == 0), stored scale fp16(d) (round to
+ * nearest even). Dequantised weight: fp16(d) * (q - 8).
+ * Errors: INVALID_ARG (null, N or K <= 0 or > W4A8_MAX_DIM, K % 32 != 0), MISALIGNED,
+ * UNSUPPORTED (dtype), CUDA.
+ */
+w4a8_status w4a8_pack_q4_0(const void* w, w4a8_dtype dtype, int N, int K,
+                           uint8_t* qs, uint16_t* d_fp16, cudaStream_t stream);
+
+/*
+ * Q8_0 activation quantisation (the per-call step that w4a8_gemm runs internally).
+ * x  : M x K row-major, f32 or bf16.
+ * qx : out, M x K int8 codes (row-major, same element order as x).
+ * dx : out, M x K/32 f32 block scales, d = amax/127 over the block.
+ * sx : out (may be NULL), M x K/32 int32 block sums of the codes.
+ * q = clamp(round_half_away_from_zero(x * (1/d)), -127, 127); all codes 0 when d == 0.
+ * Errors: as w4a8_pack_q4_0.
+ */
+w4a8_status w4a8_quant_act_q8_0(const void* x, w4a8_dtype dtype, int M, int K,
+                                int8_t* qx, float* dx, int32_t* sx, cudaStream_t stream);
+
+/*
+ * Size in bytes of the workspace w4a8_gemm / w4a8_gemm_affine need for this shape
+ * (group = 0 for Q4_0, else the affine group size). Covers every path, so one
+ * allocation serves AUTO and both forced paths. Returns 0 for invalid sizes.
+ */
+size_t w4a8_workspace_bytes(int M, int N, int K, int group);
+
+/*
+ * y = x . W^T with W in Q4_0 (from w4a8_pack_q4_0) and x quantised to Q8_0 inside the
+ * call: y[m][n] = sum_b f32(d_w[n][b]) * d_x[m][b] * D[m][n][b], with
+ * D = sum_{j<32} (q_w - 8) * q_x computed exactly. The sum over blocks is taken in f32;
+ * each output is within 1e-5 * sum_b |term_b| of the exact value.
+ * x        : M x K, f32 or bf16.       qs, d_fp16 : as produced by w4a8_pack_q4_0.
+ * y        : out, M x N f32.           ws, ws_bytes : scratch of at least
+ *            w4a8_workspace_bytes(M, N, K, 0) bytes, owned by the caller; contents on
+ *            entry are ignored and are garbage afterwards. Calls that share a workspace
+ *            must be ordered on one stream.
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype,
+                      const uint8_t* qs, const uint16_t* d_fp16, float* y,
+                      void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* w4a8_gemm with the kernel path forced (for tests and measurements). */
+w4a8_status w4a8_gemm_ex(int M, int N, int K, const void* x, w4a8_dtype dtype,
+                         const uint8_t* qs, const uint16_t* d_fp16, float* y,
+                         void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream);
+
+/*
+ * Affine 4-bit weight pack. Per row n and group g of `group` (64 or 128) elements:
+ * s = bf16((max - min) / 15), b = bf16(min), q = clamp(round_half_away((w - b) / s), 0, 15)
+ * (q = 0 when s == 0), using the stored bf16 s and b. Dequantised weight: s * q + b.
+ * w          : N x K row-major, f32 or bf16.
+ * q          : out, N x K/8 uint32 words; element k of row n sits at bits 4*(k%8) of
+ *              word n*K/8 + k/8.
+ * scale_bf16 : out, N x K/group bf16 bit patterns.   bias_bf16 : out, same shape.
+ * Errors: INVALID_ARG (also K % group != 0), UNSUPPORTED (group not 64 or 128), MISALIGNED, CUDA.
+ */
+w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int group,
+                             uint32_t* q, uint16_t* scale_bf16, uint16_t* bias_bf16,
+                             cudaStream_t stream);
+
+/*
+ * y = x . W^T with W affine 4-bit (from w4a8_pack_affine) and x quantised to Q8_0 in the
+ * call. The contraction runs on the original codes: per activation block b inside
+ * group g, y += d_x * (s_g * sum q*q_x + b_g * sum q_x). Tolerance as w4a8_gemm.
+ * Arguments and errors as w4a8_gemm, plus `group` (64 or 128).
+ */
+w4a8_status w4a8_gemm_affine(int M, int N, int K, int group, const void* x, w4a8_dtype dtype,
+                             const uint32_t* q, const uint16_t* scale_bf16,
+                             const uint16_t* bias_bf16, float* y, void* ws, size_t ws_bytes,
+                             cudaStream_t stream);
+
+/* w4a8_gemm_affine with the kernel path forced. */
+w4a8_status w4a8_gemm_affine_ex(int M, int N, int K, int group, const void* x, w4a8_dtype dtype,
+                                const uint32_t* q, const uint16_t* scale_bf16,
+                                const uint16_t* bias_bf16, float* y, void* ws, size_t ws_bytes,
+                                w4a8_path path, cudaStream_t stream);
+
+/*
+ * Reads and clears the device status word that kernels set when a bounded wait runs
+ * out. Synchronises the current device. Returns W4A8_OK when no kernel has reported a
+ * problem since the last call, W4A8_ERR_DEVICE_TIMEOUT otherwise, W4A8_ERR_CUDA if the
+ * read itself failed.
+ */
+w4a8_status w4a8_last_device_error(void);
+
+/* Static, human-readable name of a status code. */
+const char* w4a8_status_string(w4a8_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_H_ */

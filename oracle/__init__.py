@@ -1,0 +1,261 @@
+"""Scalar CPU oracle for the block-quantized W4A8 matmul (Q4_0 x Q8_0) and its affine
+4-bit variant.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline / reference leg are the only callers. The CUDA library never imports,
+links or runs anything here, and nothing here touches the CUDA library.
+
+The arithmetic lives in ``oracle.cpp`` (plain scalar C++, built with
+``-O2 -ffp-contract=off``); this module only marshals numpy arrays to it.
+
+Functions and the definitions they follow (see the header of ``oracle.cpp``):
+
+* ``f32_to_f16`` / ``f32_to_bf16`` / ``f16_to_f32`` / ``bf16_to_f32`` -- IEEE 754
+  round-to-nearest-even narrowing and exact widening.
+* ``pack_q4_0`` -- Q4_0 weights (tract PR #2432, "The kernel": 4-bit N x K weight,
+  per-32-block scale), d = mx/-8, q = min(15, trunc(x/d + 8.5)).
+* ``quant_act_q8_0`` -- Q8_0 activations (tract PR #2432, "Pipeline": activation to int8
+  per block), d = amax/127 in f32, q = round-half-away(x * (1/d)).
+* ``gemm_q4_0`` -- y = x . W^T as sum over blocks of d_w * d_x * (exact int block dot),
+  in f64 (each term exact), plus T = sum of |terms| (the tolerance scale).
+* ``pack_affine`` / ``gemm_affine`` -- MLX PR #4802 "mx.qqmm ... mode=affine": codes
+  q in [0,15], per-group bf16 scale (max-min)/15 and bias min; the contraction runs on
+  the original codes and applies d_x * (s * sum q q_x + b * sum q_x) per block.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.cpp`` into ``liboracle.so`` (g++, -O2, no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+               "-pthread", _SRC, "-o", _LIB_PATH + ".tmp"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    I64 = ctypes.c_int64
+    sigs = {
+        "orc_f32_to_f16": (ctypes.c_uint16, [ctypes.c_float]),
+        "orc_f32_to_bf16": (ctypes.c_uint16, [ctypes.c_float]),
+        "orc_f16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
+        "orc_bf16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
+        "orc_f32_to_f16_array": (None, [P, P, I64]),
+        "orc_f32_to_bf16_array": (None, [P, P, I64]),
+        "orc_f16_to_f32_array": (None, [P, P, I64]),
+        "orc_bf16_to_f32_array": (None, [P, P, I64]),
+        "orc_pack_q4_0": (None, [P, I, I, P, P]),
+        "orc_dequant_q4_0": (None, [P, P, I, I, P]),
+        "orc_quant_act_q8_0": (None, [P, I, I, P, P, P]),
+        "orc_dequant_q8_0": (None, [P, P, I, I, P]),
+        "orc_gemm_q4_0": (None, [I, I, I, P, P, P, P, P, P, I]),
+        "orc_gemm_q4_0_sampled": (None, [I, I, P, P, P, P, P, P, P, P]),
+        "orc_gemm_q4_0_f32": (None, [I, I, I, P, P, P, P, P]),
+        "orc_pack_affine": (None, [P, I, I, I, P, P, P]),
+        "orc_dequant_affine": (None, [P, P, P, I, I, I, P]),
+        "orc_gemm_affine": (None, [I, I, I, I, P, P, P, P, P, P, P, P, I]),
+        "orc_gemm_affine_sampled": (None, [I, I, I, P, P, P, P, P, P, P, P, P, P]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+# ----------------------------------------------------------------------------- O1
+def f32_to_f16(a) -> np.ndarray:
+    a = _f32(a)
+    out = np.empty(a.shape, dtype=np.uint16)
+    _load().orc_f32_to_f16_array(_p(a), _p(out), a.size)
+    return out
+
+
+def f32_to_bf16(a) -> np.ndarray:
+    a = _f32(a)
+    out = np.empty(a.shape, dtype=np.uint16)
+    _load().orc_f32_to_bf16_array(_p(a), _p(out), a.size)
+    return out
+
+
+def f16_to_f32(h) -> np.ndarray:
+    h = np.ascontiguousarray(np.asarray(h, dtype=np.uint16))
+    out = np.empty(h.shape, dtype=np.float32)
+    _load().orc_f16_to_f32_array(_p(h), _p(out), h.size)
+    return out
+
+
+def bf16_to_f32(h) -> np.ndarray:
+    h = np.ascontiguousarray(np.asarray(h, dtype=np.uint16))
+    out = np.empty(h.shape, dtype=np.float32)
+    _load().orc_bf16_to_f32_array(_p(h), _p(out), h.size)
+    return out
+
+
+# ----------------------------------------------------------------------------- O2
+def pack_q4_0(w) -> tuple[np.ndarray, np.ndarray]:
+    """W (N, K) f32 -> (qs uint8 (N, K/2), d fp16 bits uint16 (N, K/32))."""
+    w = _f32(w)
+    N, K = w.shape
+    assert K % 32 == 0
+    qs = np.empty((N, K // 2), dtype=np.uint8)
+    d = np.empty((N, K // 32), dtype=np.uint16)
+    _load().orc_pack_q4_0(_p(w), N, K, _p(qs), _p(d))
+    return qs, d
+
+
+def dequant_q4_0(qs: np.ndarray, d: np.ndarray) -> np.ndarray:
+    N, K2 = qs.shape
+    K = 2 * K2
+    out = np.empty((N, K), dtype=np.float64)
+    _load().orc_dequant_q4_0(_p(np.ascontiguousarray(qs)), _p(np.ascontiguousarray(d)), N, K, _p(out))
+    return out
+
+
+# ----------------------------------------------------------------------------- O3
+def quant_act_q8_0(x) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """x (M, K) f32 -> (qx int8 (M, K), dx f32 (M, K/32), sx int32 (M, K/32))."""
+    x = _f32(x)
+    M, K = x.shape
+    assert K % 32 == 0
+    qx = np.empty((M, K), dtype=np.int8)
+    dx = np.empty((M, K // 32), dtype=np.float32)
+    sx = np.empty((M, K // 32), dtype=np.int32)
+    _load().orc_quant_act_q8_0(_p(x), M, K, _p(qx), _p(dx), _p(sx))
+    return qx, dx, sx
+
+
+def dequant_q8_0(qx: np.ndarray, dx: np.ndarray) -> np.ndarray:
+    M, K = qx.shape
+    out = np.empty((M, K), dtype=np.float64)
+    _load().orc_dequant_q8_0(_p(np.ascontiguousarray(qx)), _p(np.ascontiguousarray(dx)), M, K, _p(out))
+    return out
+
+
+# ----------------------------------------------------------------------------- O4
+def gemm_q4_0(qx, dx, qs, d, nthreads: int = 1) -> tuple[np.ndarray, np.ndarray]:
+    """-> (y f64 (M, N), T f64 (M, N)) with T = sum over blocks of |term|."""
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    dx = np.ascontiguousarray(dx, dtype=np.float32)
+    qs = np.ascontiguousarray(qs, dtype=np.uint8)
+    d = np.ascontiguousarray(d, dtype=np.uint16)
+    M, K = qx.shape
+    N = qs.shape[0]
+    assert qs.shape[1] * 2 == K and d.shape == (N, K // 32) and dx.shape == (M, K // 32)
+    y = np.empty((M, N), dtype=np.float64)
+    T = np.empty((M, N), dtype=np.float64)
+    _load().orc_gemm_q4_0(M, N, K, _p(qx), _p(dx), _p(qs), _p(d), _p(y), _p(T), int(nthreads))
+    return y, T
+
+
+def gemm_q4_0_sampled(qx, dx, qs, d, ms, ns) -> tuple[np.ndarray, np.ndarray]:
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    dx = np.ascontiguousarray(dx, dtype=np.float32)
+    qs = np.ascontiguousarray(qs, dtype=np.uint8)
+    d = np.ascontiguousarray(d, dtype=np.uint16)
+    ms = np.ascontiguousarray(ms, dtype=np.int32)
+    ns = np.ascontiguousarray(ns, dtype=np.int32)
+    K = qx.shape[1]
+    y = np.empty(ms.shape, dtype=np.float64)
+    T = np.empty(ms.shape, dtype=np.float64)
+    _load().orc_gemm_q4_0_sampled(K, ms.size, _p(ms), _p(ns), _p(qx), _p(dx), _p(qs), _p(d), _p(y), _p(T))
+    return y, T
+
+
+def gemm_q4_0_f32(qx, dx, qs, d) -> np.ndarray:
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    dx = np.ascontiguousarray(dx, dtype=np.float32)
+    qs = np.ascontiguousarray(qs, dtype=np.uint8)
+    d = np.ascontiguousarray(d, dtype=np.uint16)
+    M, K = qx.shape
+    N = qs.shape[0]
+    y = np.empty((M, N), dtype=np.float32)
+    _load().orc_gemm_q4_0_f32(M, N, K, _p(qx), _p(dx), _p(qs), _p(d), _p(y))
+    return y
+
+
+# ----------------------------------------------------------------------------- O5
+def pack_affine(w, group: int) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """W (N, K) f32 -> (q uint32 (N, K/8), scale bf16 bits (N, K/g), bias bf16 bits (N, K/g))."""
+    w = _f32(w)
+    N, K = w.shape
+    assert K % group == 0 and group % 32 == 0
+    q = np.empty((N, K // 8), dtype=np.uint32)
+    s = np.empty((N, K // group), dtype=np.uint16)
+    b = np.empty((N, K // group), dtype=np.uint16)
+    _load().orc_pack_affine(_p(w), N, K, int(group), _p(q), _p(s), _p(b))
+    return q, s, b
+
+
+def dequant_affine(q, scale, bias, group: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint32)
+    N = q.shape[0]
+    K = q.shape[1] * 8
+    out = np.empty((N, K), dtype=np.float64)
+    _load().orc_dequant_affine(_p(q), _p(np.ascontiguousarray(scale, dtype=np.uint16)),
+                               _p(np.ascontiguousarray(bias, dtype=np.uint16)), N, K, int(group), _p(out))
+    return out
+
+
+# ----------------------------------------------------------------------------- O6
+def gemm_affine(qx, dx, sx, q, scale, bias, group: int, nthreads: int = 1) -> tuple[np.ndarray, np.ndarray]:
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    dx = np.ascontiguousarray(dx, dtype=np.float32)
+    sx = np.ascontiguousarray(sx, dtype=np.int32)
+    q = np.ascontiguousarray(q, dtype=np.uint32)
+    scale = np.ascontiguousarray(scale, dtype=np.uint16)
+    bias = np.ascontiguousarray(bias, dtype=np.uint16)
+    M, K = qx.shape
+    N = q.shape[0]
+    assert q.shape[1] * 8 == K and scale.shape == (N, K // group) and bias.shape == scale.shape
+    y = np.empty((M, N), dtype=np.float64)
+    T = np.empty((M, N), dtype=np.float64)
+    _load().orc_gemm_affine(M, N, K, int(group), _p(qx), _p(dx), _p(sx), _p(q), _p(scale), _p(bias),
+                            _p(y), _p(T), int(nthreads))
+    return y, T
+
+
+def gemm_affine_sampled(qx, dx, sx, q, scale, bias, group: int, ms, ns) -> tuple[np.ndarray, np.ndarray]:
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    dx = np.ascontiguousarray(dx, dtype=np.float32)
+    sx = np.ascontiguousarray(sx, dtype=np.int32)
+    q = np.ascontiguousarray(q, dtype=np.uint32)
+    ms = np.ascontiguousarray(ms, dtype=np.int32)
+    ns = np.ascontiguousarray(ns, dtype=np.int32)
+    K = qx.shape[1]
+    y = np.empty(ms.shape, dtype=np.float64)
+    T = np.empty(ms.shape, dtype=np.float64)
+    _load().orc_gemm_affine_sampled(K, int(group), ms.size, _p(ms), _p(ns), _p(qx), _p(dx), _p(sx), _p(q),
+                                    _p(np.ascontiguousarray(scale, dtype=np.uint16)),
+                                    _p(np.ascontiguousarray(bias, dtype=np.uint16)), _p(y), _p(T))
+    return y, T

@@ -1,0 +1,71 @@
+"""Independent numpy decoders of the packed formats, used only to pin the oracle.
+
+They restate the storage layouts from the format definitions (not from the oracle's
+code) so that a layout or indexing mistake in the oracle shows up as a mismatch:
+
+* Q4_0: row n, block b = 16 bytes at n*K/2 + 16b; byte j low nibble = element 32b+j,
+  high nibble = element 32b+j+16; w = fp16(d) * (q - 8).
+* Q8_0: x = d * q with one f32 d per 32-block.
+* affine: element k of row n at bits 4*(k%8) of uint32 word k/8; w = s*q + b with bf16
+  s and b per group.
+"""
+import numpy as np
+import torch
+
+
+def q4_0_codes(qs: np.ndarray) -> np.ndarray:
+    N, K2 = qs.shape
+    blocks = qs.reshape(N, K2 // 16, 16)
+    lo = blocks & 0x0F
+    hi = blocks >> 4
+    return np.concatenate([lo, hi], axis=2).reshape(N, K2 * 2).astype(np.int64)
+
+
+def fp16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).astype(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def q4_0_weights(qs: np.ndarray, d: np.ndarray) -> np.ndarray:
+    codes = q4_0_codes(qs)
+    scales = np.repeat(fp16_bits_to_f64(d), 32, axis=1)
+    return scales * (codes - 8)
+
+
+def q8_0_values(qx: np.ndarray, dx: np.ndarray) -> np.ndarray:
+    return np.repeat(dx.astype(np.float64), 32, axis=1) * qx.astype(np.float64)
+
+
+def affine_codes(q: np.ndarray) -> np.ndarray:
+    N, W = q.shape
+    shifts = (4 * np.arange(8, dtype=np.uint32))[None, None, :]
+    return ((q[:, :, None] >> shifts) & 0xF).reshape(N, W * 8).astype(np.int64)
+
+
+def affine_weights(q: np.ndarray, scale: np.ndarray, bias: np.ndarray, group: int) -> np.ndarray:
+    codes = affine_codes(q)
+    s = np.repeat(bf16_bits_to_f64(scale), group, axis=1)
+    b = np.repeat(bf16_bits_to_f64(bias), group, axis=1)
+    return s * codes + b
+
+
+def read_golden(path):
+    out = {}
+    rows = []
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if ":" in line:
+                k, v = line.split(":", 1)
+                out[k.strip()] = v.split()
+            else:
+                rows.append(line.split())
+    if rows:
+        out["rows"] = rows
+    return out
