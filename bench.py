@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the block-quantized W4A8 matmul (Q4_0 weights x Q8_0 activations) on B200.
+
+Headline (one JSON line on rank 0): the decode GEMV, M=1, K=N=4096, x f32 ~N(0,1),
+W ~N(0,0.02) packed to Q4_0; metric = weight GB/s (packed weight + scale bytes per call /
+call time). One step = one w4a8_gemm call through the C ABI: Q8_0 activation
+quantisation + the M-dispatched contraction (the GEMV at M=1). Weights are packed once,
+outside the timed region. Packed weight copies are rotated so that the set read by the
+timed loop (28 x 9.44 MB) is larger than twice the 126 MB L2.
+
+The same line carries: the dominant kernel's roofline (the contraction kernel alone, timed
+with CUDA events through w4a8_gemm_prepared), an end-to-end figure through the C ABI with
+host buffers (pinned H2D of x and D2H of y inside the timed region), the CPU oracle timed
+on the host cores, SM clocks sampled during the timed region, and -- unless --no-extra --
+the other workloads (MiniLM 64x384x1536, prefill 1024x4096x4096, the MLP-shape sweep, the
+affine gs64/gs128 workloads) with µs, TOP/s and roofline fractions. Every timed workload
+is first checked against the oracle; a workload that fails parity is reported as failed
+and not timed.
+
+--impl reference times the CPU oracle (the only reference this method has) on the same
+workload and metric. Under torchrun every rank runs the same workload (independent
+replicas: the path has no exchange step); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="headline workload only")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sweep", choices=["some", "all", "none"], default="some")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def traffic_table():
+    """Per-launch DRAM bytes (read + write) from the committed ncu summaries, keyed by
+    kernel and workload; lines of the form `traffic_bytes_per_launch <key> <bytes>`."""
+    out = {}
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
+        return out
+    for f in sorted(os.listdir(d)):
+        if not f.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(d, f)) as fh:
+            for line in fh:
+                parts = line.strip().strip("`").split()
+                if len(parts) == 3 and parts[0] == "traffic_bytes_per_launch":
+                    try:
+                        out[parts[1]] = float(parts[2])
+                    except ValueError:
+                        pass
+    return out
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms in the background; keeps host-timestamped rows."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = (bus_id or "").lower()
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 10:
+                self.rows.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [p for (t, p) in self.rows if self.bus_id == "" or self.bus_id.endswith(p[1].lower()[-12:])
+                or p[1].lower().endswith(self.bus_id[-12:])]
+        if not rows:
+            rows = [p for (_, p) in self.rows]
+        inwin = [p for (t, p) in self.rows if t0 - 0.25 <= t <= t1 + 0.25 and p in rows]
+        use = inwin if inwin else rows[-5:]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = sorted(float(p[2]) for p in use if p[2].replace(".", "").isdigit())
+        smx = max((float(p[3]) for p in use if p[3].replace(".", "").isdigit()), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in use for i in range(4) if p[6 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smx, "reasons": reasons,
+                "samples": len(use), "in_window": bool(inwin)}
+
+
+# ------------------------------------------------------------------ helpers
+def rank_info():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def check_parity_sampled(y_dev, ref_fn, M, N, count=400, seed=7):
+    import numpy as np
+    from block_quantized_w4a8_b200 import inputs
+    ms, ns = inputs.sample_indices(M, N, count, seed)
+    yref, T = ref_fn(ms, ns)
+    y = y_dev.cpu().numpy()[ms, ns].astype(np.float64)
+    return bool(np.all(np.abs(y - yref) <= 1e-5 * T))
+
+
+def timed(step, steps, torch, dist=None):
+    """Time exactly `steps` calls of step(i) with CUDA events on the current stream,
+    bracketed by a barrier and a device synchronize on both sides. Returns ms (max over ranks)."""
+    stream = torch.cuda.current_stream()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def copies_for(bytes_per_copy: int) -> int:
+    return max(2, math.ceil(2 * L2_BYTES / max(1, bytes_per_copy)))
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_decode_seconds(budget_s: float, nthreads: int):
+    """Time the oracle on the decode workload (quantise x, contract over all 4096 rows)."""
+    import oracle
+    from block_quantized_w4a8_b200 import inputs
+    x, w = inputs.make(inputs.DECODE)
+    qs, d = oracle.pack_q4_0(w.numpy())
+    xn = x.numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        qx, dx, _ = oracle.quant_act_q8_0(xn)
+        oracle.gemm_q4_0(qx, dx, qs, d, nthreads=nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s and reps >= 1:
+            return el / reps, reps
+
+
+def weight_bytes(N, K):
+    return N * K // 2 + N * (K // 32) * 2
+
+
+def gemv_algorithmic_bytes(M, N, K):
+    B = K // 32
+    return weight_bytes(N, K) + M * K + M * B * 8 + M * N * 4
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank, world, _ = rank_info()
+    if rank != 0:
+        return 0
+    nthreads = os.cpu_count() or 1
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        s, _ = oracle_decode_seconds(0.0, nthreads)
+        if i >= args.warmup:
+            per_step.append(s)
+    sec = sum(per_step) / len(per_step)
+    M, N, K = 1, 4096, 4096
+    gbs = weight_bytes(N, K) / sec / 1e9
+    line = {
+        "impl": "reference", "metric": "W4A8 decode GEMV weight GB/s (M=1, K=N=4096)", "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode_gemv_m1_4096x4096", "M": M, "N": N, "K": K},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                         "sample": "each step: the oracle's Q8_0 quantisation of x and the full 1x4096x4096 "
+                                   "contraction (all 4096 outputs), threads over output elements"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist_mod
+
+    import block_quantized_w4a8_b200 as w4a8
+    import oracle
+    from block_quantized_w4a8_b200 import inputs
+
+    rank, world, local_rank = rank_info()
+    dist = None
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist_mod.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist = dist_mod
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w4a8.load_library()
+    peaks = load_peaks()
+    traffic = traffic_table()
+    props = torch.cuda.get_device_properties(dev)
+    bus = None
+    try:
+        bus = f"{props.pci_domain_id:04x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}"
+    except Exception:
+        pass
+    launches = 0
+
+    # ---------------- headline: decode GEMV
+    wl = inputs.DECODE
+    M, N, K = wl.M, wl.N, wl.K
+    x, w = inputs.make(wl)
+    xd, wd = x.to(dev), w.to(dev)
+    qs0, d0 = w4a8.pack_q4_0(wd)
+    R = copies_for(weight_bytes(N, K))
+    qsl = [qs0.clone() for _ in range(R)]
+    dl = [d0.clone() for _ in range(R)]
+    ws = w4a8.workspace(M, N, K, 0, dev)
+    y = torch.empty(M, N, device=dev)
+    w4a8.w4a8_gemm(xd, qs0, d0, y, ws)
+    torch.cuda.synchronize()
+    rqx, rdx, _ = oracle.quant_act_q8_0(x.numpy())
+    rqs, rd = oracle.pack_q4_0(w.numpy())
+    yref, T = oracle.gemm_q4_0(rqx, rdx, rqs, rd, nthreads=os.cpu_count() or 1)
+    parity = bool(np.array_equal(qs0.cpu().numpy(), rqs)) and bool(
+        np.all(np.abs(y.cpu().numpy().astype(np.float64) - yref) <= 1e-5 * T))
+    if not parity:
+        if rank == 0:
+            print(json.dumps({"metric": "W4A8 decode GEMV weight GB/s (M=1, K=N=4096)", "value": None,
+                              "error": "parity check against the oracle failed; not timed"}), flush=True)
+        return 1
+
+    def step(i):
+        w4a8.w4a8_gemm(xd, qsl[i % R], dl[i % R], y, ws)
+
+    sampler = ClockSampler(bus)
+    sampler.start()
+    t_ramp = time.time()
+    while time.time() - t_ramp < 1.0:  # bring clocks up before warm-up
+        for i in range(200):
+            step(i)
+        torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.time()
+    ms = timed(step, args.steps, torch, dist)
+    t1 = time.time()
+    launches += 2 * args.steps  # act-quant + GEMV per step
+    ms_step = ms / args.steps
+    value = weight_bytes(N, K) * args.steps * world / (ms * 1e-3) / 1e9
+
+    # dominant kernel alone: the contraction from a prepared workspace
+    w4a8.w4a8_prepare_act(xd, ws)
+    for i in range(args.warmup):
+        w4a8.w4a8_gemm_prepared(M, K, qsl[i % R], dl[i % R], y, ws)
+    kms = timed(lambda i: w4a8.w4a8_gemm_prepared(M, K, qsl[i % R], dl[i % R], y, ws), args.steps, torch, dist)
+    k_us = kms / args.steps * 1e3
+    alg = gemv_algorithmic_bytes(M, N, K)
+    achieved = alg / (k_us * 1e-6) / 1e9
+    tkey = "gemv_kernel_m1_q4_0:decode_m1_4096x4096"
+
+    # end to end through the C ABI with host buffers
+    xh = x.pin_memory()
+    yh = torch.empty(M, N, pin_memory=True)
+
+    def step_e2e(i):
+        xd.copy_(xh, non_blocking=True)
+        w4a8.w4a8_gemm(xd, qsl[i % R], dl[i % R], y, ws)
+        yh.copy_(y, non_blocking=True)
+
+    for i in range(args.warmup):
+        step_e2e(i)
+    ems = timed(step_e2e, args.steps, torch, dist)
+    e2e_value = weight_bytes(N, K) * args.steps * world / (ems * 1e-3) / 1e9
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    line = {
+        "metric": "W4A8 decode GEMV weight GB/s (M=1, K=N=4096)", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": "decode_gemv_m1_4096x4096", "M": M, "N": N, "K": K,
+                   "weights": "Q4_0 (32-blocks, fp16 scale)", "activations": "f32 -> Q8_0 in the call",
+                   "l2": f"inputs larger than L2: {R} rotating packed weight copies "
+                         f"({R * weight_bytes(N, K) / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "parity": "pass",
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic.get(tkey),
+                     "kernel": "gemv_kernel<1,0> (Q4_0, M=1)", "kernel_us": k_us,
+                     "algorithmic_bytes_per_launch": alg, "peak_source": peaks.get("source", "measured") +
+                     " (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": M * K * 4, "d2h_bytes_per_step": M * N * 4,
+                "ms_per_step": ems / args.steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+
+    # ---------------- CPU baseline (rank 0, N=1)
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        nth = os.cpu_count() or 1
+        sec, reps = oracle_decode_seconds(args.cpu_seconds, nth)
+        line["cpu_baseline"] = {"value": weight_bytes(N, K) / sec / 1e9, "unit": "GB/s", "cores": nth,
+                                "kind": "oracle", "ms_per_step": sec * 1e3,
+                                "sample": f"{reps} full decode steps (Q8_0 quantisation of x + all 4096 outputs "
+                                          f"of the 1x4096x4096 contraction), ~{args.cpu_seconds:.0f} s, "
+                                          f"threads over output elements"}
+
+    # ---------------- other workloads (rank 0 only, after the collective steps)
+    if rank == 0 and not args.no_extra:
+        line["configs"] = run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev)
+
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
+    import numpy as np
+    int8_peak = 2.0 * peaks["bf16_tflops"]      # dense INT8 = 2 x the measured dense bf16 rate
+    f16_peak = peaks["bf16_tflops"]             # the MMA here runs kind::f16 (fp16 = bf16 rate)
+    results = []
+    wls = [inputs.MINILM, inputs.PREFILL]
+    if args.sweep != "none":
+        sweep = inputs.sweep_workloads()
+        if args.sweep == "some":
+            keep = {(1, 4096, 14336), (16, 4096, 14336), (64, 4096, 14336), (256, 14336, 4096),
+                    (1024, 4096, 14336), (4096, 8192, 2048), (8, 8192, 2048)}
+            sweep = [s for s in sweep if (s.M, s.K, s.N) in keep]
+        wls += sweep
+    wls += [inputs.AFFINE_GS64, inputs.AFFINE_GS128]
+    steps = max(5, min(args.steps, 50))
+    for wl in wls:
+        M, N, K = wl.M, wl.N, wl.K
+        x, w = inputs.make(wl)
+        xd = x.to(dev)
+        affine = wl.kind == "affine"
+        if affine:
+            q, s, b = w4a8.pack_affine(w.to(dev), wl.group)
+            wbytes = N * K // 2 + 2 * N * (K // wl.group) * 2
+        else:
+            qs, d = w4a8.pack_q4_0(w.to(dev))
+            wbytes = weight_bytes(N, K)
+        R = copies_for(wbytes)
+        ws = w4a8.workspace(M, N, K, wl.group if affine else 0, dev)
+        y = torch.empty(M, N, device=dev)
+        rqx, rdx, rsx = oracle.quant_act_q8_0(x.float().numpy())
+        if affine:
+            sets = [(q.clone(), s.clone(), b.clone()) for _ in range(R)]
+            rq, rs, rb = oracle.pack_affine(w.numpy(), wl.group)
+            w4a8.w4a8_gemm_affine(xd, q, s, b, y, ws, wl.group)
+            ok = check_parity_sampled(y, lambda ms, ns: oracle.gemm_affine_sampled(rqx, rdx, rsx, rq, rs, rb, wl.group,
+                                                                                   ms, ns), M, N)
+
+            def step(i):
+                qq, ss, bb = sets[i % R]
+                w4a8.w4a8_gemm_affine(xd, qq, ss, bb, y, ws, wl.group)
+
+            def kstep(i):
+                qq, ss, bb = sets[i % R]
+                w4a8.w4a8_gemm_affine_prepared(M, K, wl.group, qq, ss, bb, y, ws)
+        else:
+            sets = [(qs.clone(), d.clone()) for _ in range(R)]
+            rqs, rd = oracle.pack_q4_0(w.numpy())
+            w4a8.w4a8_gemm(xd, qs, d, y, ws)
+            ok = check_parity_sampled(y, lambda ms, ns: oracle.gemm_q4_0_sampled(rqx, rdx, rqs, rd, ms, ns), M, N)
+
+            def step(i):
+                qq, dd = sets[i % R]
+                w4a8.w4a8_gemm(xd, qq, dd, y, ws)
+
+            def kstep(i):
+                qq, dd = sets[i % R]
+                w4a8.w4a8_gemm_prepared(M, K, qq, dd, y, ws)
+        gemv = M <= 8
+        entry = {"workload": wl.name, "M": M, "N": N, "K": K, "path": "gemv" if gemv else "gemm_tc",
+                 "parity": "pass" if ok else "FAIL"}
+        if ok:
+            for i in range(3):
+                step(i)
+            ms = timed(step, steps, torch)
+            if affine:
+                w4a8.w4a8_prepare_act(xd, ws, wl.group)
+            else:
+                w4a8.w4a8_prepare_act(xd, ws)
+            for i in range(3):
+                kstep(i)
+            kms = timed(kstep, steps, torch)
+            us, kus = ms / steps * 1e3, kms / steps * 1e3
+            ops = 2.0 * M * N * K
+            entry.update({"us_per_call": us, "kernel_us": kus, "tops_call": ops / (us * 1e-6) / 1e12,
+                          "tops_kernel": ops / (kus * 1e-6) / 1e12,
+                          "weight_gbs_call": wbytes / (us * 1e-6) / 1e9})
+            if gemv:
+                alg = wbytes + M * K + M * (K // 32) * 8 + M * N * 4
+                entry["roofline"] = {"bound": "hbm", "achieved": alg / (kus * 1e-6) / 1e9, "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s"}
+                entry["roofline"]["frac"] = entry["roofline"]["achieved"] / peaks["hbm_gbs"]
+            else:
+                tk = entry["tops_kernel"]
+                entry["roofline"] = {"bound": "tensor", "achieved": tk, "unit": "TOP/s",
+                                     "peak_int8": int8_peak, "frac_int8": tk / int8_peak,
+                                     "peak_f16_mma": f16_peak, "frac_f16_mma": tk / f16_peak}
+            entry["l2"] = f"{R} rotating weight copies"
+        results.append(entry)
+        del sets
+        torch.cuda.empty_cache()
+    return results
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

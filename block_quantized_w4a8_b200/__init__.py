@@ -1,1 +1,237 @@
-"""Block-quantized W4A8 matmul for NVIDIA B200 (placeholder; the binding lands next)."""
+"""Python binding of libw4a8, the block-quantized W4A8 matmul for NVIDIA B200 (sm_100a).
+
+Argument marshalling only: every function here forwards torch CUDA tensors (their
+device pointers and sizes) and the current CUDA stream to the C ABI declared in
+``include/w4a8.h`` under the same name; all computation runs in the library's CUDA
+kernels. PyTorch provides device memory and streams, nothing else. The library is
+built in-tree (``block_quantized_w4a8_b200/libw4a8.so``); if it is missing or cannot be
+loaded, every call raises -- there is no fallback.
+
+The ``pack_q4_0`` / ``pack_affine`` / ``gemm`` / ``gemm_affine`` helpers at the bottom
+allocate the outputs and the workspace with torch and then call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a8.so")
+
+W4A8_OK = 0
+STATUS_NAMES = {0: "W4A8_OK", 1: "W4A8_ERR_INVALID_ARG", 2: "W4A8_ERR_UNSUPPORTED", 3: "W4A8_ERR_WORKSPACE",
+                4: "W4A8_ERR_CUDA", 5: "W4A8_ERR_DEVICE_TIMEOUT", 6: "W4A8_ERR_MISALIGNED"}
+W4A8_F32, W4A8_BF16 = 0, 1
+PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
+
+EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a8_gemm", "w4a8_gemm_ex",
+           "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_prepare_act",
+           "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_last_device_error", "w4a8_status_string"]
+
+
+class W4A8Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libw4a8.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libw4a8 is not built ({path} missing); run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sigs = {
+        "w4a8_pack_q4_0": (I, [P, I, I, I, P, P, P]),
+        "w4a8_quant_act_q8_0": (I, [P, I, I, I, P, P, P, P]),
+        "w4a8_workspace_bytes": (Z, [I, I, I, I]),
+        "w4a8_gemm": (I, [I, I, I, P, I, P, P, P, P, Z, P]),
+        "w4a8_gemm_ex": (I, [I, I, I, P, I, P, P, P, P, Z, I, P]),
+        "w4a8_pack_affine": (I, [P, I, I, I, I, P, P, P, P]),
+        "w4a8_gemm_affine": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, P]),
+        "w4a8_gemm_affine_ex": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, I, P]),
+        "w4a8_prepare_act": (I, [I, I, I, P, I, P, Z, I, P]),
+        "w4a8_gemm_prepared": (I, [I, I, I, P, P, P, P, Z, I, P]),
+        "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
+        "w4a8_last_device_error": (I, []),
+        "w4a8_status_string": (ctypes.c_char_p, [I]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libw4a8 takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libw4a8 takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return W4A8_F32
+    if t.dtype == torch.bfloat16:
+        return W4A8_BF16
+    return 99  # rejected by the library as W4A8_ERR_UNSUPPORTED
+
+
+def _check(fn: str, status: int) -> None:
+    if status != W4A8_OK:
+        raise W4A8Error(fn, status)
+
+
+# ------------------------------------------------------------------ C ABI, one to one
+def w4a8_pack_q4_0(w: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, stream=None) -> None:
+    N, K = w.shape
+    _check("w4a8_pack_q4_0", load_library().w4a8_pack_q4_0(_ptr(w), _dtype(w), N, K, _ptr(qs), _ptr(d), _stream(stream)))
+
+
+def w4a8_quant_act_q8_0(x: torch.Tensor, qx: torch.Tensor, dx: torch.Tensor, sx: torch.Tensor | None = None,
+                        stream=None) -> None:
+    M, K = x.shape
+    _check("w4a8_quant_act_q8_0",
+           load_library().w4a8_quant_act_q8_0(_ptr(x), _dtype(x), M, K, _ptr(qx), _ptr(dx), _ptr(sx), _stream(stream)))
+
+
+def w4a8_workspace_bytes(M: int, N: int, K: int, group: int = 0) -> int:
+    return int(load_library().w4a8_workspace_bytes(M, N, K, group))
+
+
+def w4a8_gemm_ex(x, qs, d, y, ws, path: int = PATH_AUTO, stream=None) -> None:
+    M, K = x.shape
+    N = qs.shape[0]
+    _check("w4a8_gemm_ex", load_library().w4a8_gemm_ex(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d), _ptr(y),
+                                                       _ptr(ws), ws.numel() * ws.element_size(), path,
+                                                       _stream(stream)))
+
+
+def w4a8_gemm(x, qs, d, y, ws, stream=None) -> None:
+    M, K = x.shape
+    N = qs.shape[0]
+    _check("w4a8_gemm", load_library().w4a8_gemm(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d), _ptr(y), _ptr(ws),
+                                                 ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def w4a8_pack_affine(w, group: int, q, scale, bias, stream=None) -> None:
+    N, K = w.shape
+    _check("w4a8_pack_affine", load_library().w4a8_pack_affine(_ptr(w), _dtype(w), N, K, group, _ptr(q), _ptr(scale),
+                                                               _ptr(bias), _stream(stream)))
+
+
+def w4a8_gemm_affine_ex(x, q, scale, bias, y, ws, group: int, path: int = PATH_AUTO, stream=None) -> None:
+    M, K = x.shape
+    N = q.shape[0]
+    _check("w4a8_gemm_affine_ex",
+           load_library().w4a8_gemm_affine_ex(M, N, K, group, _ptr(x), _dtype(x), _ptr(q), _ptr(scale), _ptr(bias),
+                                              _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), path,
+                                              _stream(stream)))
+
+
+def w4a8_gemm_affine(x, q, scale, bias, y, ws, group: int, stream=None) -> None:
+    M, K = x.shape
+    N = q.shape[0]
+    _check("w4a8_gemm_affine",
+           load_library().w4a8_gemm_affine(M, N, K, group, _ptr(x), _dtype(x), _ptr(q), _ptr(scale), _ptr(bias),
+                                           _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def w4a8_prepare_act(x, ws, group: int = 0, path: int = PATH_AUTO, stream=None) -> None:
+    M, K = x.shape
+    _check("w4a8_prepare_act", load_library().w4a8_prepare_act(M, K, group, _ptr(x), _dtype(x), _ptr(ws),
+                                                               ws.numel() * ws.element_size(), path, _stream(stream)))
+
+
+def w4a8_gemm_prepared(M: int, K: int, qs, d, y, ws, path: int = PATH_AUTO, stream=None) -> None:
+    N = qs.shape[0]
+    _check("w4a8_gemm_prepared", load_library().w4a8_gemm_prepared(M, N, K, _ptr(qs), _ptr(d), _ptr(y), _ptr(ws),
+                                                                   ws.numel() * ws.element_size(), path,
+                                                                   _stream(stream)))
+
+
+def w4a8_gemm_affine_prepared(M: int, K: int, group: int, q, scale, bias, y, ws, path: int = PATH_AUTO,
+                              stream=None) -> None:
+    N = q.shape[0]
+    _check("w4a8_gemm_affine_prepared",
+           load_library().w4a8_gemm_affine_prepared(M, N, K, group, _ptr(q), _ptr(scale), _ptr(bias), _ptr(y),
+                                                    _ptr(ws), ws.numel() * ws.element_size(), path,
+                                                    _stream(stream)))
+
+
+def w4a8_last_device_error() -> int:
+    return int(load_library().w4a8_last_device_error())
+
+
+def w4a8_status_string(status: int) -> str:
+    return load_library().w4a8_status_string(status).decode()
+
+
+# ------------------------------------------------------------------ allocating helpers
+def pack_q4_0(w: torch.Tensor, stream=None):
+    N, K = w.shape
+    qs = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device)
+    d = torch.empty(N, K // 32, dtype=torch.int16, device=w.device)
+    w4a8_pack_q4_0(w, qs, d, stream)
+    return qs, d
+
+
+def quant_act_q8_0(x: torch.Tensor, stream=None):
+    M, K = x.shape
+    qx = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    dx = torch.empty(M, K // 32, dtype=torch.float32, device=x.device)
+    sx = torch.empty(M, K // 32, dtype=torch.int32, device=x.device)
+    w4a8_quant_act_q8_0(x, qx, dx, sx, stream)
+    return qx, dx, sx
+
+
+def pack_affine(w: torch.Tensor, group: int, stream=None):
+    N, K = w.shape
+    q = torch.empty(N, K // 8, dtype=torch.int32, device=w.device)
+    s = torch.empty(N, K // group, dtype=torch.int16, device=w.device)
+    b = torch.empty(N, K // group, dtype=torch.int16, device=w.device)
+    w4a8_pack_affine(w, group, q, s, b, stream)
+    return q, s, b
+
+
+def workspace(M: int, N: int, K: int, group: int = 0, device="cuda") -> torch.Tensor:
+    nbytes = w4a8_workspace_bytes(M, N, K, group)
+    if nbytes == 0:
+        raise W4A8Error("w4a8_workspace_bytes", 1)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def gemm(x, qs, d, path: int = PATH_AUTO, ws=None, stream=None):
+    M, K = x.shape
+    N = qs.shape[0]
+    y = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    ws = workspace(M, N, K, 0, x.device) if ws is None else ws
+    w4a8_gemm_ex(x, qs, d, y, ws, path, stream)
+    return y
+
+
+def gemm_affine(x, q, s, b, group: int, path: int = PATH_AUTO, ws=None, stream=None):
+    M, K = x.shape
+    N = q.shape[0]
+    y = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    ws = workspace(M, N, K, group, x.device) if ws is None else ws
+    w4a8_gemm_affine_ex(x, q, s, b, y, ws, group, path, stream)
+    return y

@@ -1,0 +1,47 @@
+"""Builds libw4a8.so in-tree with nvcc for sm_100a (no JIT, no torch extension)."""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+SRC_DIR = os.path.join(PKG, "csrc")
+LIB = os.path.join(PKG, "libw4a8.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+
+def sources() -> list[str]:
+    out = [os.path.join(ROOT, "include", "w4a8.h")]
+    for f in sorted(os.listdir(SRC_DIR)):
+        if f.endswith((".cu", ".cuh")):
+            out.append(os.path.join(SRC_DIR, f))
+    return out
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(s) <= t for s in sources())
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return LIB
+    cmd = [
+        NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+        "-shared", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"),
+        os.path.join(SRC_DIR, "w4a8.cu"), "-o", LIB + ".tmp", "-lcudart",
+    ]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.check_call(cmd)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose="-v" in sys.argv)
+    print(LIB)

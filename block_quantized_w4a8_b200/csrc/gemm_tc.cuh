@@ -1,0 +1,318 @@
+// Large-M path: tcgen05 tensor-core GEMM with per-block rescaling.
+//
+// y[m][n] = sum_b  s_w[n][b] * d_x[m][b] * D[m][n][b],  D = exact 32-wide block dot.
+// The block dot must stay exact and each block must be rescaled separately (tract PR
+// #2432, "The kernel": Q4_0's per-32-block scales force a per-block rescale; there it
+// is one vector multiply per block over accumulator lanes that each hold one output).
+// Here every block gets its own tensor-memory accumulator: TMEM lane = weight row,
+// TMEM column = token, so each epilogue thread owns one output row and rescales its
+// columns with per-thread (weight) and per-column (activation) scales, with no
+// cross-lane reduction.
+//
+// Operands are fp16 holding small integers, so the MMA (kind::f16, f32 accumulate) is
+// exact: weight codes (q-8 or 16(q-8); affine q or 16q) times activation codes (16q_x or
+// q_x, see quant_act_tc_kernel), every product an integer below 2^15 and every block
+// sum below 2^20. The block dot comes out of TMEM as 16*D in f32 with no conversion.
+//
+// CTA tile: 128 weight rows x 128 tokens; one pipeline stage = 4 quant blocks (K=128).
+// Warp roles (448 threads):
+//   warps 0-7   epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane quarter)
+//               and token columns 64(w/4)..+63 of each block's accumulator, scales
+//               them and accumulates in f32 registers
+//   warps 8-11  producer: load packed 4-bit codes (16 B per row-block), expand to fp16
+//               in the MMA's K-major core-matrix layout, store scales
+//   warp 12     TMEM allocation + single-thread MMA issue
+//   warp 13     one thread issuing the bulk copies of the token operand and its scales
+// Every wait is bounded (bounded_wait); on a timeout all roles stop, outstanding copies
+// and MMAs are drained, TMEM is freed and the kernel returns.
+#pragma once
+
+#include "device_common.cuh"
+#include "quant.cuh"
+
+namespace w4a8 {
+namespace tc {
+
+constexpr int BN = 128;                   // weight rows per CTA (MMA M, TMEM lanes)
+constexpr int TT = tcgeo::kTokTile;       // tokens per CTA (MMA N)
+constexpr int S = 4;                      // quant blocks per stage
+constexpr int NS = 3;                     // stages in the ring
+constexpr int A_BLK = BN * 64;            // fp16 weight operand bytes per block
+constexpr int B_BLK = tcgeo::kTokBlockBytes;
+constexpr int OFF_B = S * A_BLK;
+constexpr int OFF_DX = OFF_B + S * B_BLK;
+constexpr int OFF_WS = OFF_DX + S * TT * 4;
+constexpr int OFF_WB = OFF_WS + S * BN * 4;
+constexpr int OFF_Z = OFF_WB + S * BN * 4;
+constexpr int STAGE_BYTES = OFF_Z + S * TT * 4;
+constexpr int CTRL_BYTES = 256;
+constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;  // + alignment slack
+constexpr int TMEM_COLS = 2 * TT;         // two accumulator buffers
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_COLS = TT / (EPI_WARPS / 4);   // token columns per epilogue warp
+constexpr int PROD_WARP0 = EPI_WARPS;            // first producer warp
+constexpr int MMA_WARP = PROD_WARP0 + 4;
+constexpr int COPY_WARP = MMA_WARP + 1;
+constexpr int NUM_THREADS = (COPY_WARP + 1) * 32;
+constexpr uint32_t IDESC = idesc_f16_f32(BN, TT);
+constexpr uint32_t LBO = 128, SBO = 512;  // core-matrix strides (K, M/N)
+
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(TMEM_COLS == 256, "tmem allocation must be a power of two >= 32");
+
+struct Ctrl {
+    unsigned long long full_a[NS];  // producer threads (128 arrivals)
+    unsigned long long full_b[NS];  // bulk copies (1 arrival + bytes)
+    unsigned long long empty[NS];   // MMA commit + one arrival per epilogue warp
+    unsigned long long tfull[2];    // MMA commit
+    unsigned long long tempty[2];   // one arrival per epilogue warp
+    unsigned long long drain;       // MMA drain on abort
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
+
+// Expand one 32-bit word of packed codes into four fp16x2 words (8 K-slots).
+// Q4_0 word = bytes 4i..4i+3 of a block: low nibbles elements 4i..4i+3, high nibbles
+// 16+4i..; affine word = elements 8t..8t+7 at bits 4e. Output slot order (both
+// operands use it): low nibbles of bytes 0,2 | of bytes 1,3 | high nibbles of bytes
+// 0,2 | of bytes 1,3. Low-nibble slots hold the code, high-nibble slots 16*code; the
+// Q4_0 codes are shifted by -8 (-128 for the x16 slots). 0x6400 is fp16 1024, so
+// (0x6400 | v) is 1024 + v exactly and one packed subtract removes the offset.
+template <int FMT>
+__device__ __forceinline__ uint4 expand_word(uint32_t w) {
+    const uint32_t ea = (w & 0x000F000Fu) | 0x64006400u;
+    const uint32_t eb = ((w >> 8) & 0x000F000Fu) | 0x64006400u;
+    const uint32_t ec = (w & 0x00F000F0u) | 0x64006400u;
+    const uint32_t ed = ((w >> 8) & 0x00F000F0u) | 0x64006400u;
+    const uint32_t off_lo = (FMT == 0) ? 0x64086408u : 0x64006400u;  // 1032 : 1024
+    const uint32_t off_hi = (FMT == 0) ? 0x64806480u : 0x64006400u;  // 1152 : 1024
+    auto sub = [](uint32_t a, uint32_t b) {
+        __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+        return *reinterpret_cast<uint32_t*>(&r);
+    };
+    return make_uint4(sub(ea, off_lo), sub(eb, off_lo), sub(ec, off_hi), sub(ed, off_hi));
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dx16,
+                   const float* __restrict__ zb, const uint8_t* __restrict__ wq,
+                   const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
+                   float* __restrict__ y) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + NS * STAGE_BYTES);
+    volatile uint32_t* abort = &ctrl->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = K >> 5;
+    const int nstages = (B + S - 1) / S;
+    const int n0 = blockIdx.x * BN;
+    const int t = blockIdx.y;
+    const int bpg = (FMT == 1) ? (group >> 5) : 1;  // blocks per affine group
+    const int G = (FMT == 1) ? K / group : 0;
+
+    auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
+    auto bar = [](unsigned long long* p) { return smem_addr(p); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(&ctrl->full_a[s]), 128);
+            mbar_init(bar(&ctrl->full_b[s]), 1);
+            mbar_init(bar(&ctrl->empty[s]), 1 + EPI_WARPS);
+        }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(bar(&ctrl->tfull[j]), 1);
+            mbar_init(bar(&ctrl->tempty[j]), EPI_WARPS);
+        }
+        mbar_init(bar(&ctrl->drain), 1);
+        ctrl->abort = 0;
+        mbar_init_fence();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(smem_addr(&ctrl->tmem_base), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctrl->tmem_base;
+
+    if (warp >= PROD_WARP0 && warp < PROD_WARP0 + 4) {
+        // ------------------------------------------------------------ producer
+        const int p = threadIdx.x - PROD_WARP0 * 32;
+        const int n = n0 + p;
+        const bool row_ok = n < N;
+        const uint4* wrow = reinterpret_cast<const uint4*>(wq + int64_t(row_ok ? n : 0) * (K >> 1));
+        uint4 cur[S], nxt[S];
+        float cs[S], cb[S], ns_[S], nb_[S];
+        auto load = [&](int st, uint4 (&wv)[S], float (&sc)[S], float (&bi)[S]) {
+#pragma unroll
+            for (int k = 0; k < S; ++k) {
+                const int b = st * S + k;
+                wv[k] = make_uint4(0u, 0u, 0u, 0u);
+                sc[k] = 0.0f;
+                bi[k] = 0.0f;
+                if (row_ok && b < B) {
+                    wv[k] = __ldg(wrow + b);
+                    if (FMT == 0) {
+                        sc[k] = __half2float(__ushort_as_half(wscale[int64_t(n) * B + b]));
+                    } else {
+                        sc[k] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + b / bpg]));
+                        bi[k] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + b / bpg]));
+                    }
+                }
+            }
+        };
+        load(0, cur, cs, cb);
+        for (int st = 0; st < nstages; ++st) {
+            const int slot = st % NS;
+            const uint32_t par = (st / NS) & 1;
+            if (st + 1 < nstages) load(st + 1, nxt, ns_, nb_);
+            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), par ^ 1, abort)) break;
+            uint8_t* sp = stage_ptr(slot);
+#pragma unroll
+            for (int k = 0; k < S; ++k) {
+                const uint32_t w[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+                uint8_t* arow = sp + k * A_BLK + (p >> 3) * 512 + (p & 7) * 16;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(arow + c * 128) = expand_word<FMT>(w[c]);
+                reinterpret_cast<float*>(sp + OFF_WS)[k * BN + p] = cs[k];
+                if (FMT == 1) reinterpret_cast<float*>(sp + OFF_WB)[k * BN + p] = cb[k];
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(&ctrl->full_a[slot]));
+#pragma unroll
+            for (int k = 0; k < S; ++k) { cur[k] = nxt[k]; cs[k] = ns_[k]; cb[k] = nb_[k]; }
+        }
+    } else if (warp == COPY_WARP) {
+        // ------------------------------------------------------------ bulk copies
+        if (lane == 0) {
+            pdl_wait_primary();  // the token operand is written by the preceding kernel
+            int issued = 0;
+            for (int st = 0; st < nstages; ++st) {
+                const int slot = st % NS;
+                const uint32_t par = (st / NS) & 1;
+                if (!bounded_wait(bar(&ctrl->empty[slot]), par ^ 1, abort)) break;
+                const int b0 = st * S;
+                const int nb = min(S, B - b0);
+                const uint32_t bytes_tok = nb * B_BLK, bytes_dx = nb * TT * 4;
+                const uint32_t bytes_z = (FMT == 1) ? (nb / bpg) * TT * 4 : 0;
+                const uint32_t fb = bar(&ctrl->full_b[slot]);
+                uint8_t* sp = stage_ptr(slot);
+                mbar_arrive_expect_tx(fb, bytes_tok + bytes_dx + bytes_z);
+                bulk_g2s(smem_addr(sp + OFF_B), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * B_BLK,
+                         bytes_tok, fb);
+                bulk_g2s(smem_addr(sp + OFF_DX), dx16 + (int64_t(t) * B + b0) * TT, bytes_dx, fb);
+                if (FMT == 1) bulk_g2s(smem_addr(sp + OFF_Z), zb + (int64_t(t) * G + b0 / bpg) * TT, bytes_z, fb);
+                issued = st + 1;
+            }
+            // Let every copy this thread issued land before the CTA can exit (on the
+            // normal path they have, or soon will; after an abort some may not be consumed).
+            uint32_t local_abort = 0;
+            for (int st = max(0, issued - NS); st < issued; ++st)
+                bounded_wait(bar(&ctrl->full_b[st % NS]), (st / NS) & 1, &local_abort);
+        }
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            bool ok = true;
+            for (int i = 0; i < B && ok; ++i) {
+                const int st = i / S, k = i - st * S, slot = st % NS;
+                const uint32_t par = (st / NS) & 1;
+                if (k == 0) {
+                    ok = bounded_wait(bar(&ctrl->full_a[slot]), par, abort) &&
+                         bounded_wait(bar(&ctrl->full_b[slot]), par, abort);
+                    if (!ok) break;
+                }
+                const int buf = i & 1;
+                if (!bounded_wait(bar(&ctrl->tempty[buf]), ((i >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_addr = smem_addr(stage_ptr(slot) + k * A_BLK);
+                const uint32_t b_addr = smem_addr(stage_ptr(slot) + OFF_B + k * B_BLK);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    tc_mma_f16(tmem_base + uint32_t(buf * TT), smem_desc_kmajor(a_addr + h * 256, LBO, SBO),
+                               smem_desc_kmajor(b_addr + h * 256, LBO, SBO), IDESC, h);
+                }
+                tc_commit(bar(&ctrl->tfull[buf]));
+                if (k == S - 1 || i == B - 1) tc_commit(bar(&ctrl->empty[slot]));
+            }
+            // Wait until every MMA (and the barrier arrivals their commits trigger) is done
+            // before TMEM and shared memory are released.
+            uint32_t local_abort = 0;
+            tc_commit(bar(&ctrl->drain));
+            bounded_wait(bar(&ctrl->drain), 0, &local_abort);
+            (void)ok;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int p = (warp & 3) * 32 + lane;   // TMEM lane == weight row within the tile
+        const int col0 = (warp >> 2) * EPI_COLS; // first token column of this warp
+        float acc[EPI_COLS];
+#pragma unroll
+        for (int j = 0; j < EPI_COLS; ++j) acc[j] = 0.0f;
+        const uint32_t lane_base = tmem_base + (uint32_t((warp & 3) * 32) << 16);
+        for (int i = 0; i < B; ++i) {
+            const int st = i / S, k = i - st * S, slot = st % NS;
+            const int buf = i & 1;
+            if (!bounded_wait_warp(bar(&ctrl->tfull[buf]), (i >> 1) & 1, abort)) break;
+            tc_fence_after();
+            const uint8_t* sp = stage_ptr(slot);
+            const float* dxs = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT + col0;
+            const float wsc = reinterpret_cast<const float*>(sp + OFF_WS)[k * BN + p];
+            uint32_t r[32];
+#pragma unroll
+            for (int c = 0; c < EPI_COLS / 32; ++c) {
+                tmem_ld_32x32(lane_base + uint32_t(buf * TT + col0 + c * 32), r);
+                tmem_wait_ld(r);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 dv = *reinterpret_cast<const float4*>(dxs + c * 32 + j);
+                    acc[c * 32 + j + 0] = fmaf(__uint_as_float(r[j + 0]), __fmul_rn(wsc, dv.x), acc[c * 32 + j + 0]);
+                    acc[c * 32 + j + 1] = fmaf(__uint_as_float(r[j + 1]), __fmul_rn(wsc, dv.y), acc[c * 32 + j + 1]);
+                    acc[c * 32 + j + 2] = fmaf(__uint_as_float(r[j + 2]), __fmul_rn(wsc, dv.z), acc[c * 32 + j + 2]);
+                    acc[c * 32 + j + 3] = fmaf(__uint_as_float(r[j + 3]), __fmul_rn(wsc, dv.w), acc[c * 32 + j + 3]);
+                }
+            }
+            if (FMT == 1 && ((i + 1) % bpg) == 0) {  // last block of a group: add bias * Z
+                const float bsc = reinterpret_cast<const float*>(sp + OFF_WB)[k * BN + p];
+                const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + (k / bpg) * TT + col0;
+#pragma unroll
+                for (int j = 0; j < EPI_COLS; j += 4) {
+                    const float4 zv = *reinterpret_cast<const float4*>(zs + j);
+                    acc[j + 0] = fmaf(bsc, zv.x, acc[j + 0]);
+                    acc[j + 1] = fmaf(bsc, zv.y, acc[j + 1]);
+                    acc[j + 2] = fmaf(bsc, zv.z, acc[j + 2]);
+                    acc[j + 3] = fmaf(bsc, zv.w, acc[j + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(&ctrl->tempty[buf]));
+                if (k == S - 1 || i == B - 1) mbar_arrive(bar(&ctrl->empty[slot]));
+            }
+        }
+        const int n = n0 + p;
+        if (n < N && !*abort) {
+#pragma unroll
+            for (int j = 0; j < EPI_COLS; ++j) {
+                const int m = t * TT + col0 + j;
+                if (m < M) y[int64_t(m) * N + n] = acc[j];
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace tc
+}  // namespace w4a8

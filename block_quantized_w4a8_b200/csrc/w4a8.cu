@@ -1,0 +1,339 @@
+// libw4a8: C-ABI entry points (argument checks, workspace layout, M-dispatch, launches).
+// Declarations and the contract of each call: include/w4a8.h.
+#include "w4a8.h"
+
+#include <cuda_runtime.h>
+
+#include "device_common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace w4a8;
+
+// Largest M served by the dp4a GEMV when the path is AUTO.
+constexpr int kGemvMaxM = 8;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline bool dims_ok(int a, int b) { return a > 0 && b > 0 && a <= W4A8_MAX_DIM && b <= W4A8_MAX_DIM; }
+
+w4a8_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ workspace layouts
+struct GemvWs {  // row-major Q8_0 activations
+    int8_t* qx;
+    float* dx;
+    int32_t* sx;
+    size_t bytes;
+};
+GemvWs gemv_ws(void* ws, int M, int K) {
+    const int64_t B = K / 32;
+    GemvWs w{};
+    size_t off = 0;
+    char* base = static_cast<char*>(ws);
+    w.qx = reinterpret_cast<int8_t*>(base + off); off = align256(off + size_t(M) * K);
+    w.dx = reinterpret_cast<float*>(base + off); off = align256(off + size_t(M) * B * 4);
+    w.sx = reinterpret_cast<int32_t*>(base + off); off = align256(off + size_t(M) * B * 4);
+    w.bytes = off;
+    return w;
+}
+
+struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
+    __half* tok;
+    float* dx16;
+    float* z;
+    int tiles;
+    size_t bytes;
+};
+TcWs tc_ws(void* ws, int M, int K, int group) {
+    const int64_t B = K / 32;
+    TcWs w{};
+    w.tiles = int(cdiv(M, tcgeo::kTokTile));
+    const int64_t rows = int64_t(w.tiles) * tcgeo::kTokTile;
+    size_t off = 0;
+    char* base = static_cast<char*>(ws);
+    w.tok = reinterpret_cast<__half*>(base + off); off = align256(off + size_t(rows) * B * 64);
+    w.dx16 = reinterpret_cast<float*>(base + off); off = align256(off + size_t(rows) * B * 4);
+    w.z = reinterpret_cast<float*>(base + off);
+    if (group > 0) off = align256(off + size_t(rows) * (K / group) * 4);
+    w.bytes = off;
+    return w;
+}
+
+// ------------------------------------------------------------------ launch helpers
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+w4a8_status run_quant_rowmajor(const void* x, w4a8_dtype dt, int M, int K, int8_t* qx, float* dx, int32_t* sx,
+                               cudaStream_t stream) {
+    const int64_t nblocks = int64_t(M) * (K / 32);
+    const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
+    if (dt == W4A8_BF16)
+        quant_act_rowmajor_kernel<true><<<grid, 256, 0, stream>>>(x, nblocks, qx, dx, sx);
+    else
+        quant_act_rowmajor_kernel<false><<<grid, 256, 0, stream>>>(x, nblocks, qx, dx, sx);
+    return launch_status();
+}
+
+w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, const TcWs& w, cudaStream_t stream) {
+    const int64_t nblocks = int64_t(w.tiles) * tcgeo::kTokTile * (K / 32);
+    const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
+    if (group == 0) {
+        if (dt == W4A8_BF16)
+            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, 0);
+        else
+            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, 0);
+    } else {
+        if (dt == W4A8_BF16)
+            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, group);
+        else
+            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, group);
+    }
+    return launch_status();
+}
+
+template <int FMT>
+w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint8_t* wq, const uint16_t* ws,
+                     const uint16_t* wb, float* y, cudaStream_t stream) {
+    const dim3 grid(unsigned(cdiv(N, kGemvWarps)));
+    const dim3 block(kGemvWarps * 32);
+    const int B = K / 32;
+    for (int m0 = 0; m0 < M; m0 += 8) {
+        const int mc = (M - m0 < 8) ? (M - m0) : 8;
+        const int8_t* qx = a.qx + int64_t(m0) * K;
+        const float* dx = a.dx + int64_t(m0) * B;
+        const int32_t* sx = a.sx + int64_t(m0) * B;
+        float* yy = y + int64_t(m0) * N;
+        cudaError_t e;
+        if (mc == 1)
+            e = launch_pdl(gemv_kernel<1, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+        else if (mc == 2)
+            e = launch_pdl(gemv_kernel<2, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+        else if (mc <= 4)
+            e = launch_pdl(gemv_kernel<4, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+        else
+            e = launch_pdl(gemv_kernel<8, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+        if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    }
+    return W4A8_OK;
+}
+
+template <int FMT>
+w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
+                        const uint16_t* wb, float* y, cudaStream_t stream) {
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        if (cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::SMEM_BYTES) != cudaSuccess)
+            return W4A8_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const dim3 grid(unsigned(cdiv(N, tc::BN)), unsigned(w.tiles));
+    cudaError_t e = launch_pdl(tc::gemm_tc_kernel<FMT>, grid, dim3(tc::NUM_THREADS), size_t(tc::SMEM_BYTES), stream,
+                               M, N, K, group, (const __half*)w.tok, (const float*)w.dx16, (const float*)w.z, wq, ws,
+                               wb, y);
+    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
+                            const void* wb, bool affine, int group, const float* y, const void* work,
+                            size_t work_bytes, w4a8_path path) {
+    if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 32) != 0) return W4A8_ERR_INVALID_ARG;
+    if (!x || !wq || !ws || !y || (affine && !wb)) return W4A8_ERR_INVALID_ARG;
+    if (dt != W4A8_F32 && dt != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
+    if (path != W4A8_PATH_AUTO && path != W4A8_PATH_GEMV && path != W4A8_PATH_GEMM) return W4A8_ERR_UNSUPPORTED;
+    if (affine) {
+        if (group != 64 && group != 128) return W4A8_ERR_UNSUPPORTED;
+        if (K % group != 0) return W4A8_ERR_INVALID_ARG;
+    }
+    if (!aligned16(x) || !aligned16(wq) || !aligned16(ws) || !aligned16(y) || (affine && !aligned16(wb)))
+        return W4A8_ERR_MISALIGNED;
+    if (!work) return W4A8_ERR_WORKSPACE;
+    if (!aligned16(work)) return W4A8_ERR_MISALIGNED;
+    if (work_bytes < w4a8_workspace_bytes(M, N, K, affine ? group : 0)) return W4A8_ERR_WORKSPACE;
+    return W4A8_OK;
+}
+
+inline bool use_gemv(int M, w4a8_path path) {
+    return (path == W4A8_PATH_GEMV) || (path == W4A8_PATH_AUTO && M <= kGemvMaxM);
+}
+
+// Quantise x into the workspace layout of the chosen path.
+w4a8_status prepare_impl(int M, int K, int group, const void* x, w4a8_dtype dt, void* work, bool gemv,
+                         cudaStream_t stream) {
+    if (gemv) {
+        GemvWs a = gemv_ws(work, M, K);
+        return run_quant_rowmajor(x, dt, M, K, a.qx, a.dx, a.sx, stream);
+    }
+    return run_quant_tc(x, dt, M, K, group, tc_ws(work, M, K, group), stream);
+}
+
+// Contraction from a prepared workspace.
+template <int FMT>
+w4a8_status contract_impl(int M, int N, int K, int group, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb,
+                          float* y, void* work, bool gemv, cudaStream_t stream) {
+    if (gemv) return run_gemv<FMT>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, stream);
+    return run_gemm_tc<FMT>(M, N, K, group, tc_ws(work, M, K, FMT == 1 ? group : 0), wq, ws, wb, y, stream);
+}
+
+template <int FMT>
+w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
+                      const uint16_t* ws, const uint16_t* wb, float* y, void* work, size_t work_bytes,
+                      w4a8_path path, cudaStream_t stream) {
+    w4a8_status st = check_gemm_args(M, N, K, x, dt, wq, ws, wb, FMT == 1, group, y, work, work_bytes, path);
+    if (st != W4A8_OK) return st;
+    const bool gemv = use_gemv(M, path);
+    st = prepare_impl(M, K, FMT == 1 ? group : 0, x, dt, work, gemv, stream);
+    if (st != W4A8_OK) return st;
+    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, gemv, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+w4a8_status w4a8_pack_q4_0(const void* w, w4a8_dtype dtype, int N, int K, uint8_t* qs, uint16_t* d_fp16,
+                           cudaStream_t stream) {
+    if (!dims_ok(N, K) || (K % 32) != 0 || !w || !qs || !d_fp16) return W4A8_ERR_INVALID_ARG;
+    if (dtype != W4A8_F32 && dtype != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
+    if (!aligned16(w) || !aligned16(qs) || !aligned16(d_fp16)) return W4A8_ERR_MISALIGNED;
+    const int64_t nblocks = int64_t(N) * (K / 32);
+    const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
+    if (dtype == W4A8_BF16)
+        pack_q4_0_kernel<true><<<grid, 256, 0, stream>>>(w, nblocks, qs, d_fp16);
+    else
+        pack_q4_0_kernel<false><<<grid, 256, 0, stream>>>(w, nblocks, qs, d_fp16);
+    return launch_status();
+}
+
+w4a8_status w4a8_quant_act_q8_0(const void* x, w4a8_dtype dtype, int M, int K, int8_t* qx, float* dx, int32_t* sx,
+                                cudaStream_t stream) {
+    if (!dims_ok(M, K) || (K % 32) != 0 || !x || !qx || !dx) return W4A8_ERR_INVALID_ARG;
+    if (dtype != W4A8_F32 && dtype != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(qx) || !aligned16(dx) || (sx && !aligned16(sx))) return W4A8_ERR_MISALIGNED;
+    return run_quant_rowmajor(x, dtype, M, K, qx, dx, sx, stream);
+}
+
+size_t w4a8_workspace_bytes(int M, int N, int K, int group) {
+    if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 32) != 0) return 0;
+    if (group != 0 && (group != 64 && group != 128)) return 0;
+    if (group != 0 && (K % group) != 0) return 0;
+    const size_t a = gemv_ws(nullptr, M, K).bytes;
+    const size_t b = tc_ws(nullptr, M, K, group).bytes;
+    return a > b ? a : b;
+}
+
+w4a8_status w4a8_gemm_ex(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
+                         const uint16_t* d_fp16, float* y, void* ws, size_t ws_bytes, w4a8_path path,
+                         cudaStream_t stream) {
+    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, ws, ws_bytes, path, stream);
+}
+
+w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
+                      const uint16_t* d_fp16, float* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    return w4a8_gemm_ex(M, N, K, x, dtype, qs, d_fp16, y, ws, ws_bytes, W4A8_PATH_AUTO, stream);
+}
+
+w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int group, uint32_t* q,
+                             uint16_t* scale_bf16, uint16_t* bias_bf16, cudaStream_t stream) {
+    if (!dims_ok(N, K) || (K % 32) != 0 || !w || !q || !scale_bf16 || !bias_bf16) return W4A8_ERR_INVALID_ARG;
+    if (group != 64 && group != 128) return W4A8_ERR_UNSUPPORTED;
+    if (K % group != 0) return W4A8_ERR_INVALID_ARG;
+    if (dtype != W4A8_F32 && dtype != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
+    if (!aligned16(w) || !aligned16(q) || !aligned16(scale_bf16) || !aligned16(bias_bf16)) return W4A8_ERR_MISALIGNED;
+    const int64_t ngroups = int64_t(N) * (K / group);
+    const int64_t threads = ngroups * (group / 4);
+    const dim3 grid(unsigned(cdiv(threads, 256)));
+    if (dtype == W4A8_BF16)
+        pack_affine_kernel<true><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale_bf16, bias_bf16);
+    else
+        pack_affine_kernel<false><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale_bf16, bias_bf16);
+    return launch_status();
+}
+
+w4a8_status w4a8_gemm_affine_ex(int M, int N, int K, int group, const void* x, w4a8_dtype dtype, const uint32_t* q,
+                                const uint16_t* scale_bf16, const uint16_t* bias_bf16, float* y, void* ws,
+                                size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
+    return gemm_impl<1>(M, N, K, group, x, dtype, reinterpret_cast<const uint8_t*>(q), scale_bf16, bias_bf16, y, ws,
+                        ws_bytes, path, stream);
+}
+
+w4a8_status w4a8_gemm_affine(int M, int N, int K, int group, const void* x, w4a8_dtype dtype, const uint32_t* q,
+                             const uint16_t* scale_bf16, const uint16_t* bias_bf16, float* y, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    return w4a8_gemm_affine_ex(M, N, K, group, x, dtype, q, scale_bf16, bias_bf16, y, ws, ws_bytes, W4A8_PATH_AUTO,
+                               stream);
+}
+
+w4a8_status w4a8_prepare_act(int M, int K, int group, const void* x, w4a8_dtype dtype, void* ws, size_t ws_bytes,
+                             w4a8_path path, cudaStream_t stream) {
+    const bool affine = group != 0;
+    // the weight pointers are not used here; pass x so their null / alignment checks pass
+    w4a8_status st = check_gemm_args(M, 1, K, x, dtype, x, x, x, affine, group, static_cast<const float*>(x), ws,
+                                     ws_bytes, path);
+    if (st != W4A8_OK) return st;
+    return prepare_impl(M, K, group, x, dtype, ws, use_gemv(M, path), stream);
+}
+
+w4a8_status w4a8_gemm_prepared(int M, int N, int K, const uint8_t* qs, const uint16_t* d_fp16, float* y,
+                               const void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
+    w4a8_status st = check_gemm_args(M, N, K, qs, W4A8_F32, qs, d_fp16, nullptr, false, 0, y, ws, ws_bytes, path);
+    if (st != W4A8_OK) return st;
+    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, const_cast<void*>(ws), use_gemv(M, path), stream);
+}
+
+w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint32_t* q, const uint16_t* scale_bf16,
+                                      const uint16_t* bias_bf16, float* y, const void* ws, size_t ws_bytes,
+                                      w4a8_path path, cudaStream_t stream) {
+    const uint8_t* wq = reinterpret_cast<const uint8_t*>(q);
+    w4a8_status st =
+        check_gemm_args(M, N, K, wq, W4A8_F32, wq, scale_bf16, bias_bf16, true, group, y, ws, ws_bytes, path);
+    if (st != W4A8_OK) return st;
+    return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, const_cast<void*>(ws), use_gemv(M, path),
+                            stream);
+}
+
+w4a8_status w4a8_last_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return W4A8_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, w4a8::g_device_status, sizeof(v)) != cudaSuccess) return W4A8_ERR_CUDA;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(w4a8::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return W4A8_ERR_CUDA;
+    return v ? W4A8_ERR_DEVICE_TIMEOUT : W4A8_OK;
+}
+
+const char* w4a8_status_string(w4a8_status s) {
+    switch (s) {
+        case W4A8_OK: return "W4A8_OK";
+        case W4A8_ERR_INVALID_ARG: return "W4A8_ERR_INVALID_ARG";
+        case W4A8_ERR_UNSUPPORTED: return "W4A8_ERR_UNSUPPORTED";
+        case W4A8_ERR_WORKSPACE: return "W4A8_ERR_WORKSPACE";
+        case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
+        case W4A8_ERR_DEVICE_TIMEOUT: return "W4A8_ERR_DEVICE_TIMEOUT";
+        case W4A8_ERR_MISALIGNED: return "W4A8_ERR_MISALIGNED";
+    }
+    return "W4A8_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

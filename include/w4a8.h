@@ -144,6 +144,30 @@ w4a8_status w4a8_gemm_affine_ex(int M, int N, int K, int group, const void* x, w
                                 w4a8_path path, cudaStream_t stream);
 
 /*
+ * Split form of w4a8_gemm / w4a8_gemm_affine for an activation that feeds several
+ * weight matrices (e.g. projections sharing one input): the activation is quantised
+ * once and the per-call re-quantisation the tract page identifies as per-op overhead
+ * ("W4A8MatMul op" measurements) is paid once.
+ *  w4a8_prepare_act   quantises x (M x K) into `ws` in the layout of the path that a
+ *                     matmul of this M takes (`path` AUTO resolves by M exactly as
+ *                     w4a8_gemm does; group = 0 for Q4_0 weights, else 64 or 128).
+ *  w4a8_gemm_prepared / w4a8_gemm_affine_prepared
+ *                     run only the contraction, reading the quantised activation from
+ *                     `ws`. They must be given the same M, K, group and path as the
+ *                     w4a8_prepare_act call that filled `ws`, on the same stream (or
+ *                     after it completed); `ws` is only read.
+ * Errors: as w4a8_gemm.
+ */
+w4a8_status w4a8_prepare_act(int M, int K, int group, const void* x, w4a8_dtype dtype, void* ws,
+                             size_t ws_bytes, w4a8_path path, cudaStream_t stream);
+w4a8_status w4a8_gemm_prepared(int M, int N, int K, const uint8_t* qs, const uint16_t* d_fp16, float* y,
+                               const void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream);
+w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint32_t* q,
+                                      const uint16_t* scale_bf16, const uint16_t* bias_bf16, float* y,
+                                      const void* ws, size_t ws_bytes, w4a8_path path,
+                                      cudaStream_t stream);
+
+/*
  * Reads and clears the device status word that kernels set when a bounded wait runs
  * out. Synchronises the current device. Returns W4A8_OK when no kernel has reported a
  * problem since the last call, W4A8_ERR_DEVICE_TIMEOUT otherwise, W4A8_ERR_CUDA if the

@@ -29,6 +29,24 @@
 #include <thread>
 #include <vector>
 
+// Runs f(e) for every e in [0, count), the range split into contiguous chunks over
+// `nthreads` host threads. Each output element is computed by exactly one call, so the
+// result does not depend on the thread count.
+template <class F>
+static void parallel_over(int64_t count, int nthreads, F f) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads == 1 || count < 2) {
+        for (int64_t e = 0; e < count; ++e) f(e);
+        return;
+    }
+    std::vector<std::thread> pool;
+    for (int t = 0; t < nthreads; ++t) {
+        const int64_t e0 = count * t / nthreads, e1 = count * (t + 1) / nthreads;
+        if (e1 > e0) pool.emplace_back([=]() { for (int64_t e = e0; e < e1; ++e) f(e); });
+    }
+    for (auto& th : pool) th.join();
+}
+
 extern "C" {
 
 // ---------------------------------------------------------------------------------
@@ -244,24 +262,14 @@ static void gemm_q4_0_one(int K, int m, int n, const int8_t* qx, const float* dx
     if (T) *T = tabs;
 }
 
-// Full output; rows of y are split over `nthreads` host threads (the arithmetic of
-// each output element is the same whatever the thread count).
+// Full output; output elements are split over `nthreads` host threads.
 void orc_gemm_q4_0(int M, int N, int K, const int8_t* qx, const float* dx, const uint8_t* qs,
                    const uint16_t* d, double* y, double* T, int nthreads) {
-    if (nthreads < 1) nthreads = 1;
-    auto work = [&](int m0, int m1) {
-        for (int m = m0; m < m1; ++m)
-            for (int n = 0; n < N; ++n)
-                gemm_q4_0_one(K, m, n, qx, dx, qs, d, y + int64_t(m) * N + n,
-                              T ? T + int64_t(m) * N + n : nullptr);
+    auto one = [&](int64_t e) {
+        const int m = int(e / N), n = int(e % N);
+        gemm_q4_0_one(K, m, n, qx, dx, qs, d, y + e, T ? T + e : nullptr);
     };
-    if (nthreads == 1 || M == 1) { work(0, M); return; }
-    std::vector<std::thread> pool;
-    for (int t = 0; t < nthreads; ++t) {
-        int m0 = int(int64_t(M) * t / nthreads), m1 = int(int64_t(M) * (t + 1) / nthreads);
-        if (m1 > m0) pool.emplace_back(work, m0, m1);
-    }
-    for (auto& th : pool) th.join();
+    parallel_over(int64_t(M) * N, nthreads, one);
 }
 
 // Selected output elements only: (ms[i], ns[i]) for i < count.
@@ -394,20 +402,11 @@ static void gemm_affine_one(int K, int group, int m, int n, const int8_t* qx, co
 void orc_gemm_affine(int M, int N, int K, int group, const int8_t* qx, const float* dx, const int32_t* sx,
                      const uint32_t* q, const uint16_t* scale, const uint16_t* bias, double* y, double* T,
                      int nthreads) {
-    if (nthreads < 1) nthreads = 1;
-    auto work = [&](int m0, int m1) {
-        for (int m = m0; m < m1; ++m)
-            for (int n = 0; n < N; ++n)
-                gemm_affine_one(K, group, m, n, qx, dx, sx, q, scale, bias, y + int64_t(m) * N + n,
-                                T ? T + int64_t(m) * N + n : nullptr);
+    auto one = [&](int64_t e) {
+        const int m = int(e / N), n = int(e % N);
+        gemm_affine_one(K, group, m, n, qx, dx, sx, q, scale, bias, y + e, T ? T + e : nullptr);
     };
-    if (nthreads == 1 || M == 1) { work(0, M); return; }
-    std::vector<std::thread> pool;
-    for (int t = 0; t < nthreads; ++t) {
-        int m0 = int(int64_t(M) * t / nthreads), m1 = int(int64_t(M) * (t + 1) / nthreads);
-        if (m1 > m0) pool.emplace_back(work, m0, m1);
-    }
-    for (auto& th : pool) th.join();
+    parallel_over(int64_t(M) * N, nthreads, one);
 }
 
 void orc_gemm_affine_sampled(int K, int group, int count, const int32_t* ms, const int32_t* ns,

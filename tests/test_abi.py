@@ -1,0 +1,108 @@
+"""Host-side checks of the C-ABI library (no GPU): it loads, exports every entry point
+include/w4a8.h declares, sizes workspaces, and rejects bad arguments with the status
+codes the header documents before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_quantized_w4a8_b200 as w4a8
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_quantized_w4a8_b200 import build
+    build.build()
+    return w4a8.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a8_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_gemm", "w4a8_gemm_affine",
+                     "w4a8_pack_affine", "w4a8_workspace_bytes"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(w4a8.EXPORTS) >= set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code, name in w4a8.STATUS_NAMES.items():
+        assert w4a8.w4a8_status_string(code) == name
+
+
+def _align(v):
+    return (v + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("M,N,K,group", [(1, 4096, 4096, 0), (64, 1536, 384, 0), (1024, 4096, 4096, 0),
+                                         (1024, 4096, 4096, 64), (1024, 4096, 4096, 128), (300, 333, 800, 0)])
+def test_workspace_bytes(lib, M, N, K, group):
+    B = K // 32
+    gemv = _align(M * K) + _align(M * B * 4) + _align(M * B * 4)
+    rows = -(-M // 128) * 128
+    tc = _align(rows * B * 64) + _align(rows * B * 4) + (_align(rows * (K // group) * 4) if group else 0)
+    assert w4a8.w4a8_workspace_bytes(M, N, K, group) == max(gemv, tc)
+
+
+@pytest.mark.parametrize("args", [(0, 16, 32, 0), (16, 16, 33, 0), (16, 16, 64, 32), (16, 16, 96, 64),
+                                  (-1, 16, 32, 0), (16, (1 << 20) + 1, 32, 0)])
+def test_workspace_bytes_rejects(lib, args):
+    assert w4a8.w4a8_workspace_bytes(*args) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails its checks first
+
+
+def _gemm(lib, M, N, K, x=FAKE, dt=0, qs=FAKE, d=FAKE, y=FAKE, ws=FAKE, wsb=1 << 40, path=0):
+    P = ctypes.c_void_p
+    return lib.w4a8_gemm_ex(M, N, K, P(x), dt, P(qs), P(d), P(y), P(ws), wsb, path, P(0))
+
+
+def test_gemm_argument_errors(lib):
+    assert _gemm(lib, 0, 8, 32) == 1            # INVALID_ARG
+    assert _gemm(lib, 8, 8, 48) == 1            # K % 32
+    assert _gemm(lib, 8, 8, 32, x=0) == 1       # null
+    assert _gemm(lib, 8, 8, 32, dt=7) == 2      # UNSUPPORTED dtype
+    assert _gemm(lib, 8, 8, 32, path=9) == 2    # UNSUPPORTED path
+    assert _gemm(lib, 8, 8, 32, y=FAKE + 4) == 6   # MISALIGNED
+    assert _gemm(lib, 8, 8, 32, ws=0) == 3      # WORKSPACE missing
+    assert _gemm(lib, 8, 8, 32, wsb=16) == 3    # WORKSPACE too small
+
+
+def test_affine_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib.w4a8_gemm_affine_ex
+    base = dict(x=P(FAKE), q=P(FAKE), s=P(FAKE), b=P(FAKE), y=P(FAKE), ws=P(FAKE))
+
+    def call(M=8, N=8, K=128, group=64, b=base["b"], dt=0):
+        return f(M, N, K, group, base["x"], dt, base["q"], base["s"], b, base["y"], base["ws"], 1 << 40, 0, P(0))
+
+    assert call(group=32) == 2      # only 64 and 128 (the guard of meTile PR #29: bit width / group checked)
+    assert call(group=256) == 2
+    assert call(K=192, group=128) == 1
+    assert call(b=P(0)) == 1
+    assert lib.w4a8_pack_affine(P(FAKE), 0, 8, 128, 96, P(FAKE), P(FAKE), P(FAKE), P(0)) == 2
+
+
+def test_pack_and_quant_argument_errors(lib):
+    P = ctypes.c_void_p
+    assert lib.w4a8_pack_q4_0(P(FAKE), 0, 8, 40, P(FAKE), P(FAKE), P(0)) == 1
+    assert lib.w4a8_pack_q4_0(P(FAKE), 3, 8, 32, P(FAKE), P(FAKE), P(0)) == 2
+    assert lib.w4a8_pack_q4_0(P(FAKE + 8), 0, 8, 32, P(FAKE), P(FAKE), P(0)) == 6
+    assert lib.w4a8_quant_act_q8_0(P(FAKE), 0, 0, 32, P(FAKE), P(FAKE), P(0), P(0)) == 1
+    assert lib.w4a8_quant_act_q8_0(P(FAKE), 0, 4, 32, P(FAKE), P(0), P(0), P(0)) == 1
+    assert lib.w4a8_quant_act_q8_0(P(FAKE), 0, 4, 32, P(FAKE), P(FAKE), P(FAKE + 4), P(0)) == 6

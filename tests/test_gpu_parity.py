@@ -1,0 +1,259 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Codes, scales and block sums must be bit-exact; matmul outputs must satisfy
+|y - y_ref| <= 1e-5 * T elementwise, T = sum over blocks of |d_w * d_x * D| (the oracle's
+exact f64 terms), and y must be exactly 0 where T is 0. Small shapes are compared in
+full (several tiles in every dimension plus ragged tails); the full-size workloads are
+compared on sampled outputs that the oracle computes one by one, in the launch
+configuration the benchmark times.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_w4a8_b200 as w4a8
+import oracle
+from block_quantized_w4a8_b200 import inputs
+from tests import refdecode as ref
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-5
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+PATHS = {"auto": w4a8.PATH_AUTO, "gemv": w4a8.PATH_GEMV, "gemm": w4a8.PATH_GEMM}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    w4a8.load_library()
+    yield
+    assert w4a8.w4a8_last_device_error() == 0, "a kernel reported a bounded-wait timeout"
+
+
+def dev(t):
+    return t.contiguous().cuda()
+
+
+def as_np(t):
+    return t.cpu().numpy()
+
+
+def check_tol(y, yref, T, what=""):
+    y = np.asarray(y, dtype=np.float64)
+    err = np.abs(y - yref)
+    bad = err > TOL * T
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; first at {tuple(i)}: "
+                             f"y={y[tuple(i)]!r} ref={yref[tuple(i)]!r} T={T[tuple(i)]!r}")
+    nz = T > 0
+    return float((err[nz] / T[nz]).max()) if nz.any() else 0.0
+
+
+# ------------------------------------------------------------------ act quant
+@pytest.mark.parametrize("M,K,dtype", [(64, 384, "f32"), (1, 4096, "f32"), (37, 160, "bf16"), (300, 800, "f32"),
+                                       (5, 14336, "bf16")])
+def test_quant_act_bit_exact(M, K, dtype):
+    x = inputs.randn((M, K), seed=M * 7 + K)
+    x[0, :32] = 0.0
+    if M > 2:
+        x[2, 32:64] = torch.arange(32, dtype=torch.float32) - 15.5  # exact half-way products
+    xt = x.to(torch.bfloat16) if dtype == "bf16" else x
+    qx, dx, sx = w4a8.quant_act_q8_0(dev(xt))
+    rq, rd, rs = oracle.quant_act_q8_0(xt.float().numpy())
+    assert np.array_equal(as_np(qx), rq)
+    assert np.array_equal(as_np(dx).view(np.uint32), rd.view(np.uint32))
+    assert np.array_equal(as_np(sx), rs)
+
+
+def test_quant_act_golden_rounding():
+    g = ref.read_golden(os.path.join(GOLDEN, "q8_0_rounding.txt"))
+    x = torch.tensor([[float(v) for v in g["x"]]], dtype=torch.float32)
+    qx, dx, sx = w4a8.quant_act_q8_0(dev(x))
+    assert [int(v) for v in as_np(qx)[0]] == [int(v) for v in g["q"]]
+    assert int(as_np(sx)[0, 0]) == int(g["sum"][0])
+
+
+# ------------------------------------------------------------------ weight packs
+@pytest.mark.parametrize("N,K,dtype,std", [(1536, 384, "f32", 0.02), (4096, 4096, "f32", 0.02), (333, 800, "bf16", 1.0),
+                                           (64, 14336, "f32", 1.0)])
+def test_pack_q4_0_bit_exact(N, K, dtype, std):
+    w = inputs.randn((N, K), seed=N + K, std=std)
+    w[1, :32] = 0.0
+    w[2, 32] = 0.5
+    w[2, 33] = -0.5
+    wt = w.to(torch.bfloat16) if dtype == "bf16" else w
+    qs, d = w4a8.pack_q4_0(dev(wt))
+    rqs, rd = oracle.pack_q4_0(wt.float().numpy())
+    assert np.array_equal(as_np(qs), rqs)
+    assert np.array_equal(as_np(d).view(np.uint16), rd)
+
+
+def test_pack_q4_0_golden_block():
+    g = ref.read_golden(os.path.join(GOLDEN, "q4_0_block_layout.txt"))
+    w = torch.tensor([[float(v) for v in g["x"]]], dtype=torch.float32)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    assert [int(b) for b in as_np(qs)[0]] == [int(v, 16) for v in g["bytes"]]
+    assert int(as_np(d).view(np.uint16)[0, 0]) == int(g["scale_fp16_bits"][0], 16)
+
+
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("N,K,dtype", [(512, 1024, "f32"), (4096, 4096, "bf16"), (33, 384, "f32")])
+def test_pack_affine_bit_exact(group, N, K, dtype):
+    w = inputs.randn((N, K), seed=N * 3 + group)
+    w[1, :group] = 0.25
+    wt = w.to(torch.bfloat16) if dtype == "bf16" else w
+    q, s, b = w4a8.pack_affine(dev(wt), group)
+    rq, rs, rb = oracle.pack_affine(wt.float().numpy(), group)
+    assert np.array_equal(as_np(q).view(np.uint32), rq)
+    assert np.array_equal(as_np(s).view(np.uint16), rs)
+    assert np.array_equal(as_np(b).view(np.uint16), rb)
+
+
+# ------------------------------------------------------------------ Q4_0 matmul, full compare
+SHAPES = [(1, 1, 32), (1, 4096, 4096), (2, 333, 800), (5, 1536, 384), (8, 200, 256), (64, 1536, 384),
+          (300, 333, 800), (129, 128, 128), (130, 257, 4128), (3, 64, 32768)]
+
+
+def _q4_0_case(M, N, K, x_dtype="f32", w_std=0.02, seed=0):
+    wl = inputs.Workload("case", M=M, K=K, N=N, x_dtype=x_dtype, w_std=w_std, seed=seed)
+    x, w = inputs.make(wl)
+    rqx, rdx, _ = oracle.quant_act_q8_0(x.float().numpy())
+    rqs, rd = oracle.pack_q4_0(w.numpy())
+    return x, w, rqx, rdx, rqs, rd
+
+
+@pytest.mark.parametrize("path", ["gemv", "gemm", "auto"])
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_gemm_q4_0_vs_oracle(M, N, K, path):
+    x, w, rqx, rdx, rqs, rd = _q4_0_case(M, N, K, seed=M + N)
+    yref, T = oracle.gemm_q4_0(rqx, rdx, rqs, rd, nthreads=8)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    y = w4a8.gemm(dev(x), qs, d, path=PATHS[path])
+    torch.cuda.synchronize()
+    check_tol(as_np(y), yref, T, f"M={M} N={N} K={K} {path}")
+
+
+def test_gemm_bf16_input_and_paths_agree():
+    x, w, rqx, rdx, rqs, rd = _q4_0_case(48, 640, 1024, x_dtype="bf16", w_std=1.0, seed=5)
+    yref, T = oracle.gemm_q4_0(rqx, rdx, rqs, rd, nthreads=8)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    ya = as_np(w4a8.gemm(dev(x), qs, d, path=w4a8.PATH_GEMV))
+    yb = as_np(w4a8.gemm(dev(x), qs, d, path=w4a8.PATH_GEMM))
+    check_tol(ya, yref, T, "gemv bf16")
+    check_tol(yb, yref, T, "gemm bf16")
+    assert np.all(np.abs(ya.astype(np.float64) - yb) <= 2 * TOL * T)
+
+
+def test_gemm_degenerate_inputs_give_exact_zero():
+    M, N, K = 130, 160, 256
+    x = torch.zeros(M, K)
+    w = inputs.randn((N, K), seed=1, std=0.02)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    for path in (w4a8.PATH_GEMV, w4a8.PATH_GEMM):
+        assert torch.count_nonzero(w4a8.gemm(dev(x), qs, d, path=path)).item() == 0
+    qs0, d0 = w4a8.pack_q4_0(dev(torch.zeros(N, K)))
+    x1 = inputs.randn((M, K), seed=2)
+    for path in (w4a8.PATH_GEMV, w4a8.PATH_GEMM):
+        assert torch.count_nonzero(w4a8.gemm(dev(x1), qs0, d0, path=path)).item() == 0
+
+
+def test_gemm_is_deterministic_and_ignores_workspace_contents():
+    M, N, K = 200, 384, 1024
+    x, w, *_ = _q4_0_case(M, N, K, seed=3)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    for path in (w4a8.PATH_GEMV, w4a8.PATH_GEMM):
+        ws = w4a8.workspace(M, N, K)
+        ws.random_(0, 256)
+        y1 = w4a8.gemm(dev(x), qs, d, path=path, ws=ws)
+        ws.random_(0, 256)
+        y2 = w4a8.gemm(dev(x), qs, d, path=path, ws=ws)
+        assert torch.equal(y1, y2)
+
+
+def test_empty_input_is_rejected():
+    qs = torch.zeros(8, 16, dtype=torch.uint8, device="cuda")
+    d = torch.zeros(8, 1, dtype=torch.int16, device="cuda")
+    x = torch.zeros(0, 32, device="cuda")
+    y = torch.zeros(0, 8, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(w4a8.W4A8Error) as e:
+        w4a8.w4a8_gemm(x, qs, d, y, ws)
+    assert e.value.status == 1
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+FULL = [inputs.MINILM, inputs.DECODE, inputs.PREFILL,
+        inputs.Workload("mlp_m16_k4096_n14336", M=16, K=4096, N=14336),
+        inputs.Workload("mlp_m256_k14336_n4096", M=256, K=14336, N=4096),
+        inputs.Workload("mlp_m4096_k8192_n2048", M=4096, K=8192, N=2048)]
+
+
+@pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)
+def test_full_size_sampled(wl):
+    x, w = inputs.make(wl)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    y = as_np(w4a8.gemm(dev(x), qs, d))           # AUTO: the path the benchmark times
+    rqx, rdx, _ = oracle.quant_act_q8_0(x.float().numpy())
+    rqs, rd = oracle.pack_q4_0(w.numpy())
+    assert np.array_equal(as_np(qs), rqs) and np.array_equal(as_np(d).view(np.uint16), rd)
+    ms, ns = inputs.sample_indices(wl.M, wl.N, 3000)
+    yref, T = oracle.gemm_q4_0_sampled(rqx, rdx, rqs, rd, ms, ns)
+    check_tol(y[ms, ns], yref, T, wl.name)
+
+
+# ------------------------------------------------------------------ affine
+AFFINE_SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (64, 1536, 384), (200, 333, 1280), (130, 128, 4096)]
+
+
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("path", ["gemv", "gemm"])
+@pytest.mark.parametrize("M,N,K", AFFINE_SHAPES)
+def test_gemm_affine_vs_oracle(M, N, K, path, group):
+    if K % group:
+        pytest.skip("K not a multiple of the group")
+    wl = inputs.Workload("aff", M=M, K=K, N=N, x_dtype="bf16", w_std=1.0, seed=M * 5 + N)
+    x, w = inputs.make(wl)
+    rqx, rdx, rsx = oracle.quant_act_q8_0(x.float().numpy())
+    rq, rs, rb = oracle.pack_affine(w.numpy(), group)
+    yref, T = oracle.gemm_affine(rqx, rdx, rsx, rq, rs, rb, group, nthreads=8)
+    q, s, b = w4a8.pack_affine(dev(w), group)
+    y = as_np(w4a8.gemm_affine(dev(x), q, s, b, group, path=PATHS[path]))
+    check_tol(y, yref, T, f"affine gs{group} M={M} N={N} K={K} {path}")
+
+
+@pytest.mark.parametrize("wl", [inputs.AFFINE_GS64, inputs.AFFINE_GS128], ids=lambda w: w.name)
+def test_affine_full_size_sampled(wl):
+    x, w = inputs.make(wl)
+    q, s, b = w4a8.pack_affine(dev(w), wl.group)
+    y = as_np(w4a8.gemm_affine(dev(x), q, s, b, wl.group))
+    rqx, rdx, rsx = oracle.quant_act_q8_0(x.float().numpy())
+    rq, rs, rb = oracle.pack_affine(w.numpy(), wl.group)
+    assert np.array_equal(as_np(q).view(np.uint32), rq)
+    ms, ns = inputs.sample_indices(wl.M, wl.N, 3000)
+    yref, T = oracle.gemm_affine_sampled(rqx, rdx, rsx, rq, rs, rb, wl.group, ms, ns)
+    check_tol(y[ms, ns], yref, T, wl.name)
+
+
+def test_affine_bias_minus_8s_matches_q4_0_on_gpu():
+    """Cross-format invariant on the GPU: affine codes with bias = -8*scale reproduce the
+    Q4_0 matmul with d = scale and the same codes."""
+    rng = np.random.default_rng(12)
+    M, N, K, group = 160, 256, 512, 64
+    codes = rng.integers(0, 16, size=(N, K))
+    scale = (2.0 ** rng.integers(-8, -4, size=(N, K // group))).astype(np.float32)
+    words = (codes.reshape(N, K // 8, 8).astype(np.uint64) << (4 * np.arange(8, dtype=np.uint64))).sum(axis=2).astype(np.uint32)
+    s_bits = torch.from_numpy(scale).to(torch.bfloat16).view(torch.int16)
+    b_bits = torch.from_numpy(-8 * scale).to(torch.bfloat16).view(torch.int16)
+    blocks = codes.reshape(N, K // 32, 32)
+    qs = (blocks[:, :, :16] | (blocks[:, :, 16:] << 4)).reshape(N, K // 2).astype(np.uint8)
+    d_bits = np.repeat(scale, group // 32, axis=1).astype(np.float16).view(np.int16)
+    x = dev(inputs.randn((M, K), seed=13))
+    for path in (w4a8.PATH_GEMV, w4a8.PATH_GEMM):
+        ya = w4a8.gemm_affine(x, dev(torch.from_numpy(words.view(np.int32))), dev(s_bits), dev(b_bits), group,
+                              path=path)
+        yq = w4a8.gemm(x, dev(torch.from_numpy(qs)), dev(torch.from_numpy(d_bits)), path=path)
+        rqx, rdx, _ = oracle.quant_act_q8_0(as_np(x))
+        _, T = oracle.gemm_q4_0(rqx, rdx, qs, d_bits.view(np.uint16), nthreads=8)
+        assert np.all(np.abs(as_np(ya).astype(np.float64) - as_np(yq)) <= 2 * TOL * T)
