@@ -28,12 +28,14 @@ PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 
 EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a8_gemm", "w4a8_gemm_ex",
            "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_prepare_act",
-           "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_last_device_error", "w4a8_status_string"]
+           "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_last_device_error", "w4a8_last_cuda_error_string",
+           "w4a8_status_string"]
 
 
 class W4A8Error(RuntimeError):
-    def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        msg = f"{fn} failed: {STATUS_NAMES.get(status, status)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
         self.status = status
 
 
@@ -63,6 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
         "w4a8_last_device_error": (I, []),
         "w4a8_status_string": (ctypes.c_char_p, [I]),
+        "w4a8_last_cuda_error_string": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -97,7 +100,8 @@ def _dtype(t: torch.Tensor) -> int:
 
 def _check(fn: str, status: int) -> None:
     if status != W4A8_OK:
-        raise W4A8Error(fn, status)
+        detail = load_library().w4a8_last_cuda_error_string().decode() if status == 4 else ""
+        raise W4A8Error(fn, status, detail)
 
 
 # ------------------------------------------------------------------ C ABI, one to one
@@ -179,6 +183,10 @@ def w4a8_gemm_affine_prepared(M: int, K: int, group: int, q, scale, bias, y, ws,
 
 def w4a8_last_device_error() -> int:
     return int(load_library().w4a8_last_device_error())
+
+
+def w4a8_last_cuda_error_string() -> str:
+    return load_library().w4a8_last_cuda_error_string().decode()
 
 
 def w4a8_status_string(status: int) -> str:

@@ -37,7 +37,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     ]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
-    subprocess.check_call(cmd)
+    subprocess.check_call(cmd, timeout=900)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

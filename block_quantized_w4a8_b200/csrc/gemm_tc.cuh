@@ -6,7 +6,7 @@
 // is one vector multiply per block over accumulator lanes that each hold one output).
 // Here every block gets its own tensor-memory accumulator: TMEM lane = weight row,
 // TMEM column = token, so each epilogue thread owns one output row and rescales its
-// columns with per-thread (weight) and per-column (activation) scales, with no
+// columns with a per-thread (weight) and a per-column (activation) scale, with no
 // cross-lane reduction.
 //
 // Operands are fp16 holding small integers, so the MMA (kind::f16, f32 accumulate) is
@@ -14,15 +14,19 @@
 // q_x, see quant_act_tc_kernel), every product an integer below 2^15 and every block
 // sum below 2^20. The block dot comes out of TMEM as 16*D in f32 with no conversion.
 //
-// CTA tile: 128 weight rows x 128 tokens; one pipeline stage = 4 quant blocks (K=128).
+// CTA tile: 128 weight rows x 128 tokens; one pipeline stage = 4 quant blocks (K=128),
+// 3 stages; 4 TMEM accumulator buffers of 128 columns (the whole 512-column TMEM).
 // Warp roles (448 threads):
-//   warps 0-7   epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane quarter)
-//               and token columns 64(w/4)..+63 of each block's accumulator, scales
-//               them and accumulates in f32 registers
-//   warps 8-11  producer: load packed 4-bit codes (16 B per row-block), expand to fp16
-//               in the MMA's K-major core-matrix layout, store scales
-//   warp 12     TMEM allocation + single-thread MMA issue
-//   warp 13     one thread issuing the bulk copies of the token operand and its scales
+//   WG0, WG1 (warps 0-7)  epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane
+//                         quarter) and token columns 64(w/4)..+63 of each block's
+//                         accumulator, scales them and accumulates in f32 registers
+//   WG2 (warps 8-11)      producer: load packed 4-bit codes (16 B per row-block, two
+//                         stages ahead), expand to fp16 in the MMA's K-major core-matrix
+//                         layout, store the per-row scales
+//   warp 12               TMEM allocation + single-thread MMA issue
+//   warp 13               one thread issuing the bulk copies of the token operand and
+//                         its scales
+// The kernel runs one CTA per SM with 128 registers per thread.
 // Every wait is bounded (bounded_wait); on a timeout all roles stop, outstanding copies
 // and MMAs are drained, TMEM is freed and the kernel returns.
 #pragma once
@@ -37,6 +41,7 @@ constexpr int BN = 128;                   // weight rows per CTA (MMA M, TMEM la
 constexpr int TT = tcgeo::kTokTile;       // tokens per CTA (MMA N)
 constexpr int S = 4;                      // quant blocks per stage
 constexpr int NS = 3;                     // stages in the ring
+constexpr int NACC = 4;                   // TMEM accumulator buffers
 constexpr int A_BLK = BN * 64;            // fp16 weight operand bytes per block
 constexpr int B_BLK = tcgeo::kTokBlockBytes;
 constexpr int OFF_B = S * A_BLK;
@@ -47,27 +52,30 @@ constexpr int OFF_Z = OFF_WB + S * BN * 4;
 constexpr int STAGE_BYTES = OFF_Z + S * TT * 4;
 constexpr int CTRL_BYTES = 256;
 constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;  // + alignment slack
-constexpr int TMEM_COLS = 2 * TT;         // two accumulator buffers
+constexpr int TMEM_COLS = NACC * TT;
 constexpr int EPI_WARPS = 8;
-constexpr int EPI_COLS = TT / (EPI_WARPS / 4);   // token columns per epilogue warp
-constexpr int PROD_WARP0 = EPI_WARPS;            // first producer warp
-constexpr int MMA_WARP = PROD_WARP0 + 4;
-constexpr int COPY_WARP = MMA_WARP + 1;
-constexpr int NUM_THREADS = (COPY_WARP + 1) * 32;
+constexpr int EPI_COLS = TT / (EPI_WARPS / 4);   // token columns per epilogue warp (64)
+constexpr int PROD_WARP0 = 8;
+constexpr int MMA_WARP = 12;
+constexpr int COPY_WARP = 13;
+constexpr int NUM_THREADS = 448;
+constexpr int MAX_REGS = 128;
 constexpr uint32_t IDESC = idesc_f16_f32(BN, TT);
 constexpr uint32_t LBO = 128, SBO = 512;  // core-matrix strides (K, M/N)
 
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-static_assert(TMEM_COLS == 256, "tmem allocation must be a power of two >= 32");
+static_assert(TMEM_COLS == 512, "tmem allocation must be a power of two >= 32");
+static_assert(EPI_COLS == 64, "epilogue loads 64 columns per warp");
+static_assert(NUM_THREADS * MAX_REGS <= 65536, "register file");
 
 struct Ctrl {
-    unsigned long long full_a[NS];  // producer threads (128 arrivals)
-    unsigned long long full_b[NS];  // bulk copies (1 arrival + bytes)
-    unsigned long long empty[NS];   // MMA commit + one arrival per epilogue warp
-    unsigned long long tfull[2];    // MMA commit
-    unsigned long long tempty[2];   // one arrival per epilogue warp
-    unsigned long long drain;       // MMA drain on abort
+    unsigned long long full_a[NS];    // producer threads (128 arrivals)
+    unsigned long long full_b[NS];    // bulk copies (1 arrival + bytes)
+    unsigned long long empty[NS];     // MMA commit + one arrival per epilogue warp
+    unsigned long long tfull[NACC];   // MMA commit
+    unsigned long long tempty[NACC];  // one arrival per epilogue warp
+    unsigned long long drain;         // final MMA drain
     uint32_t tmem_base;
     uint32_t abort;
 };
@@ -94,6 +102,12 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
     };
     return make_uint4(sub(ea, off_lo), sub(eb, off_lo), sub(ec, off_hi), sub(ed, off_hi));
 }
+
+// Codes and scales of one stage of one weight row, held in registers until stored.
+struct RowStage {
+    uint4 w[S];
+    float s[S], b[S];
+};
 
 template <int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -123,7 +137,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(bar(&ctrl->full_b[s]), 1);
             mbar_init(bar(&ctrl->empty[s]), 1 + EPI_WARPS);
         }
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < NACC; ++j) {
             mbar_init(bar(&ctrl->tfull[j]), 1);
             mbar_init(bar(&ctrl->tempty[j]), EPI_WARPS);
         }
@@ -139,6 +153,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctrl->tmem_base;
+    // Dependent launches may begin their prologue; they wait for this grid's completion
+    // before reading its output.
+    pdl_launch_dependents();
 
     if (warp >= PROD_WARP0 && warp < PROD_WARP0 + 4) {
         // ------------------------------------------------------------ producer
@@ -146,56 +163,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int n = n0 + p;
         const bool row_ok = n < N;
         const uint4* wrow = reinterpret_cast<const uint4*>(wq + int64_t(row_ok ? n : 0) * (K >> 1));
-        uint4 cur[S], nxt[S];
-        float cs[S], cb[S], ns_[S], nb_[S];
-        auto load = [&](int st, uint4 (&wv)[S], float (&sc)[S], float (&bi)[S]) {
+        auto load = [&](int st, RowStage& rs) {
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 const int b = st * S + k;
-                wv[k] = make_uint4(0u, 0u, 0u, 0u);
-                sc[k] = 0.0f;
-                bi[k] = 0.0f;
+                rs.w[k] = make_uint4(0u, 0u, 0u, 0u);
+                rs.s[k] = 0.0f;
+                rs.b[k] = 0.0f;
                 if (row_ok && b < B) {
-                    wv[k] = __ldg(wrow + b);
+                    rs.w[k] = __ldg(wrow + b);
                     if (FMT == 0) {
-                        sc[k] = __half2float(__ushort_as_half(wscale[int64_t(n) * B + b]));
+                        rs.s[k] = __half2float(__ushort_as_half(wscale[int64_t(n) * B + b]));
                     } else {
-                        sc[k] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + b / bpg]));
-                        bi[k] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + b / bpg]));
+                        rs.s[k] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + b / bpg]));
+                        rs.b[k] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + b / bpg]));
                     }
                 }
             }
         };
-        load(0, cur, cs, cb);
-        for (int st = 0; st < nstages; ++st) {
+        // Store one stage into shared memory; false if the wait gave up.
+        auto produce = [&](int st, const RowStage& rs) {
             const int slot = st % NS;
-            const uint32_t par = (st / NS) & 1;
-            if (st + 1 < nstages) load(st + 1, nxt, ns_, nb_);
-            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), par ^ 1, abort)) break;
+            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) return false;
             uint8_t* sp = stage_ptr(slot);
 #pragma unroll
             for (int k = 0; k < S; ++k) {
-                const uint32_t w[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+                const uint32_t w[4] = {rs.w[k].x, rs.w[k].y, rs.w[k].z, rs.w[k].w};
                 uint8_t* arow = sp + k * A_BLK + (p >> 3) * 512 + (p & 7) * 16;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(arow + c * 128) = expand_word<FMT>(w[c]);
-                reinterpret_cast<float*>(sp + OFF_WS)[k * BN + p] = cs[k];
-                if (FMT == 1) reinterpret_cast<float*>(sp + OFF_WB)[k * BN + p] = cb[k];
+                reinterpret_cast<float*>(sp + OFF_WS)[k * BN + p] = rs.s[k];
+                if (FMT == 1) reinterpret_cast<float*>(sp + OFF_WB)[k * BN + p] = rs.b[k];
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(&ctrl->full_a[slot]));
-#pragma unroll
-            for (int k = 0; k < S; ++k) { cur[k] = nxt[k]; cs[k] = ns_[k]; cb[k] = nb_[k]; }
+            return true;
+        };
+        RowStage r0, r1, r2;  // stages st, st+1, st+2 in flight
+        load(0, r0);
+        if (1 < nstages) load(1, r1);
+        for (int st = 0; st < nstages; st += 3) {
+            if (st + 2 < nstages) load(st + 2, r2);
+            if (!produce(st, r0)) break;
+            if (st + 1 >= nstages) break;
+            if (st + 3 < nstages) load(st + 3, r0);
+            if (!produce(st + 1, r1)) break;
+            if (st + 2 >= nstages) break;
+            if (st + 4 < nstages) load(st + 4, r1);
+            if (!produce(st + 2, r2)) break;
         }
-    } else if (warp == COPY_WARP) {
-        // ------------------------------------------------------------ bulk copies
-        if (lane == 0) {
+    } else if (warp >= MMA_WARP) {
+        if (warp == COPY_WARP && lane == 0) {
+            // -------------------------------------------------------- bulk copies
             pdl_wait_primary();  // the token operand is written by the preceding kernel
             int issued = 0;
             for (int st = 0; st < nstages; ++st) {
                 const int slot = st % NS;
-                const uint32_t par = (st / NS) & 1;
-                if (!bounded_wait(bar(&ctrl->empty[slot]), par ^ 1, abort)) break;
+                if (!bounded_wait(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) break;
                 const int b0 = st * S;
                 const int nb = min(S, B - b0);
                 const uint32_t bytes_tok = nb * B_BLK, bytes_dx = nb * TT * 4;
@@ -214,21 +238,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t local_abort = 0;
             for (int st = max(0, issued - NS); st < issued; ++st)
                 bounded_wait(bar(&ctrl->full_b[st % NS]), (st / NS) & 1, &local_abort);
-        }
-    } else if (warp == MMA_WARP) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            bool ok = true;
-            for (int i = 0; i < B && ok; ++i) {
+        } else if (warp == MMA_WARP && lane == 0) {
+            // -------------------------------------------------------- MMA issue
+            for (int i = 0; i < B; ++i) {
                 const int st = i / S, k = i - st * S, slot = st % NS;
                 const uint32_t par = (st / NS) & 1;
                 if (k == 0) {
-                    ok = bounded_wait(bar(&ctrl->full_a[slot]), par, abort) &&
-                         bounded_wait(bar(&ctrl->full_b[slot]), par, abort);
-                    if (!ok) break;
+                    if (!bounded_wait(bar(&ctrl->full_a[slot]), par, abort)) break;
+                    if (!bounded_wait(bar(&ctrl->full_b[slot]), par, abort)) break;
                 }
-                const int buf = i & 1;
-                if (!bounded_wait(bar(&ctrl->tempty[buf]), ((i >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+                const int buf = i % NACC;
+                if (!bounded_wait(bar(&ctrl->tempty[buf]), ((i / NACC) & 1) ^ 1, abort)) break;
                 tc_fence_after();
                 const uint32_t a_addr = smem_addr(stage_ptr(slot) + k * A_BLK);
                 const uint32_t b_addr = smem_addr(stage_ptr(slot) + OFF_B + k * B_BLK);
@@ -245,63 +265,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t local_abort = 0;
             tc_commit(bar(&ctrl->drain));
             bounded_wait(bar(&ctrl->drain), 0, &local_abort);
-            (void)ok;
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int p = (warp & 3) * 32 + lane;   // TMEM lane == weight row within the tile
+        const int p = (warp & 3) * 32 + lane;    // TMEM lane == weight row within the tile
         const int col0 = (warp >> 2) * EPI_COLS; // first token column of this warp
-        float acc[EPI_COLS];
+        unsigned long long acc[EPI_COLS / 2];    // f32 pairs
 #pragma unroll
-        for (int j = 0; j < EPI_COLS; ++j) acc[j] = 0.0f;
+        for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = 0ull;
         const uint32_t lane_base = tmem_base + (uint32_t((warp & 3) * 32) << 16);
         for (int i = 0; i < B; ++i) {
             const int st = i / S, k = i - st * S, slot = st % NS;
-            const int buf = i & 1;
-            if (!bounded_wait_warp(bar(&ctrl->tfull[buf]), (i >> 1) & 1, abort)) break;
+            const int buf = i % NACC;
+            if (!bounded_wait_warp(bar(&ctrl->tfull[buf]), (i / NACC) & 1, abort)) break;
             tc_fence_after();
             const uint8_t* sp = stage_ptr(slot);
             const float* dxs = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT + col0;
             const float wsc = reinterpret_cast<const float*>(sp + OFF_WS)[k * BN + p];
-            uint32_t r[32];
+            const unsigned long long w2 = pack2(wsc, wsc);
 #pragma unroll
-            for (int c = 0; c < EPI_COLS / 32; ++c) {
-                tmem_ld_32x32(lane_base + uint32_t(buf * TT + col0 + c * 32), r);
+            for (int h = 0; h < EPI_COLS / 32; ++h) {  // two 32-column halves keep registers below the cap
+                uint32_t r[32];
+                tmem_ld_32x32(lane_base + uint32_t(buf * TT + col0 + h * 32), r);
                 tmem_wait_ld(r);
+                if (h == EPI_COLS / 32 - 1) {  // TMEM buffer free: every value is in registers
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(&ctrl->tempty[buf]));
+                }
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    const float4 dv = *reinterpret_cast<const float4*>(dxs + c * 32 + j);
-                    acc[c * 32 + j + 0] = fmaf(__uint_as_float(r[j + 0]), __fmul_rn(wsc, dv.x), acc[c * 32 + j + 0]);
-                    acc[c * 32 + j + 1] = fmaf(__uint_as_float(r[j + 1]), __fmul_rn(wsc, dv.y), acc[c * 32 + j + 1]);
-                    acc[c * 32 + j + 2] = fmaf(__uint_as_float(r[j + 2]), __fmul_rn(wsc, dv.z), acc[c * 32 + j + 2]);
-                    acc[c * 32 + j + 3] = fmaf(__uint_as_float(r[j + 3]), __fmul_rn(wsc, dv.w), acc[c * 32 + j + 3]);
+                    const float4 dv = *reinterpret_cast<const float4*>(dxs + h * 32 + j);
+                    fma2_scaled(acc[(h * 32 + j) / 2], r[j], r[j + 1], dv.x, dv.y, w2);
+                    fma2_scaled(acc[(h * 32 + j) / 2 + 1], r[j + 2], r[j + 3], dv.z, dv.w, w2);
                 }
             }
             if (FMT == 1 && ((i + 1) % bpg) == 0) {  // last block of a group: add bias * Z
                 const float bsc = reinterpret_cast<const float*>(sp + OFF_WB)[k * BN + p];
+                const unsigned long long b2 = pack2(bsc, bsc);
                 const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + (k / bpg) * TT + col0;
 #pragma unroll
                 for (int j = 0; j < EPI_COLS; j += 4) {
                     const float4 zv = *reinterpret_cast<const float4*>(zs + j);
-                    acc[j + 0] = fmaf(bsc, zv.x, acc[j + 0]);
-                    acc[j + 1] = fmaf(bsc, zv.y, acc[j + 1]);
-                    acc[j + 2] = fmaf(bsc, zv.z, acc[j + 2]);
-                    acc[j + 3] = fmaf(bsc, zv.w, acc[j + 3]);
+                    fma2_bias(acc[j / 2], zv.x, zv.y, b2);
+                    fma2_bias(acc[j / 2 + 1], zv.z, zv.w, b2);
                 }
             }
-            tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(&ctrl->tempty[buf]));
-                if (k == S - 1 || i == B - 1) mbar_arrive(bar(&ctrl->empty[slot]));
-            }
+            if (lane == 0 && (k == S - 1 || i == B - 1)) mbar_arrive(bar(&ctrl->empty[slot]));
         }
         const int n = n0 + p;
         if (n < N && !*abort) {
 #pragma unroll
-            for (int j = 0; j < EPI_COLS; ++j) {
+            for (int j = 0; j < EPI_COLS; j += 2) {
+                float a, b;
+                unpack2(acc[j / 2], a, b);
                 const int m = t * TT + col0 + j;
-                if (m < M) y[int64_t(m) * N + n] = acc[j];
+                if (m < M) y[int64_t(m) * N + n] = a;
+                if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
             }
         }
     }

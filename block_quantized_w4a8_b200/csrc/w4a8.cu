@@ -22,9 +22,16 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline bool dims_ok(int a, int b) { return a > 0 && b > 0 && a <= W4A8_MAX_DIM && b <= W4A8_MAX_DIM; }
 
-w4a8_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+// Last CUDA error a call of this thread turned into W4A8_ERR_CUDA.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+w4a8_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return W4A8_OK;
+    t_last_cuda_error = e;
+    return W4A8_ERR_CUDA;
 }
+
+w4a8_status launch_status() { return cuda_status(cudaGetLastError()); }
 
 // ------------------------------------------------------------------ workspace layouts
 struct GemvWs {  // row-major Q8_0 activations
@@ -111,30 +118,104 @@ w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, 
     return launch_status();
 }
 
+// Largest activation (shared-memory footprint) the persistent GEMV stages, and the
+// largest M*K for which each CTA quantises x itself instead of a separate kernel.
+constexpr size_t kGemv2MaxSmem = 160 * 1024;
+constexpr int64_t kFuseMaxElems = 16384;
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cached[dev] = v;
+    }
+    return cached[dev];
+}
+
+inline int gemv_mt(int mc) { return mc == 1 ? 1 : mc == 2 ? 2 : mc <= 4 ? 4 : 8; }
+
+// Launch one persistent-GEMV instantiation (sets its shared-memory limit once per device).
+template <int MT, int FMT, int XMODE>
+cudaError_t launch_gemv2(int M, int N, int K, int group, const void* x, const int8_t* qx, const float* dx,
+                         const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, float* y,
+                         cudaStream_t stream) {
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    const size_t smem = gemv2_smem_bytes(MT, K);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemv2_kernel<MT, FMT, XMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(kGemv2MaxSmem));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    const int64_t ctas = cdiv(N, kGemv2Warps);
+    const dim3 grid(unsigned(ctas < sm_count() ? ctas : sm_count()));
+    return launch_pdl(gemv2_kernel<MT, FMT, XMODE>, grid, dim3(kGemv2Threads), smem, stream, M, N, K, group, x, qx,
+                      dx, sx, wq, ws, wb, y);
+}
+
+template <int FMT, int XMODE>
+cudaError_t launch_gemv2_mt(int mt, int M, int N, int K, int group, const void* x, const int8_t* qx, const float* dx,
+                            const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, float* y,
+                            cudaStream_t stream) {
+    switch (mt) {
+        case 1: return launch_gemv2<1, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
+        case 2: return launch_gemv2<2, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
+        case 4: return launch_gemv2<4, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
+        default: return launch_gemv2<8, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
+    }
+}
+
+// True when one call can quantise x inside the GEMV (no separate act-quant launch).
+inline bool gemv_fused(int M, int K) {
+    return int64_t(M) * K <= kFuseMaxElems && gemv2_smem_bytes(gemv_mt(M < 8 ? M : 8), K) <= kGemv2MaxSmem && M <= 8;
+}
+
+// GEMV contraction from a prepared row-major Q8_0 workspace, in chunks of 8 rows of x.
 template <int FMT>
 w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint8_t* wq, const uint16_t* ws,
                      const uint16_t* wb, float* y, cudaStream_t stream) {
-    const dim3 grid(unsigned(cdiv(N, kGemvWarps)));
-    const dim3 block(kGemvWarps * 32);
     const int B = K / 32;
     for (int m0 = 0; m0 < M; m0 += 8) {
         const int mc = (M - m0 < 8) ? (M - m0) : 8;
+        const int mt = gemv_mt(mc);
         const int8_t* qx = a.qx + int64_t(m0) * K;
         const float* dx = a.dx + int64_t(m0) * B;
         const int32_t* sx = a.sx + int64_t(m0) * B;
         float* yy = y + int64_t(m0) * N;
         cudaError_t e;
-        if (mc == 1)
-            e = launch_pdl(gemv_kernel<1, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
-        else if (mc == 2)
-            e = launch_pdl(gemv_kernel<2, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
-        else if (mc <= 4)
-            e = launch_pdl(gemv_kernel<4, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
-        else
-            e = launch_pdl(gemv_kernel<8, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
-        if (e != cudaSuccess) return W4A8_ERR_CUDA;
+        if (gemv2_smem_bytes(mt, K) <= kGemv2MaxSmem) {
+            e = launch_gemv2_mt<FMT, 0>(mt, mc, N, K, group, nullptr, qx, dx, sx, wq, ws, wb, yy, stream);
+        } else {  // activation too large for shared memory: stream it from L1/L2
+            const dim3 grid(unsigned(cdiv(N, kGemvWarps)));
+            const dim3 block(kGemvWarps * 32);
+            if (mt == 1)
+                e = launch_pdl(gemv_kernel<1, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+            else if (mt == 2)
+                e = launch_pdl(gemv_kernel<2, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+            else if (mt == 4)
+                e = launch_pdl(gemv_kernel<4, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+            else
+                e = launch_pdl(gemv_kernel<8, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+        }
+        if (e != cudaSuccess) return cuda_status(e);
     }
     return W4A8_OK;
+}
+
+// One-launch GEMV that quantises x itself (requires gemv_fused(M, K)).
+template <int FMT>
+w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
+                           const uint16_t* ws, const uint16_t* wb, float* y, cudaStream_t stream) {
+    const int mt = gemv_mt(M);
+    cudaError_t e = (dt == W4A8_BF16)
+                        ? launch_gemv2_mt<FMT, 2>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, stream)
+                        : launch_gemv2_mt<FMT, 1>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, stream);
+    return cuda_status(e);
 }
 
 template <int FMT>
@@ -144,16 +225,16 @@ w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uin
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W4A8_ERR_CUDA;
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        if (cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::SMEM_BYTES) != cudaSuccess)
-            return W4A8_ERR_CUDA;
+        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+        if (ea != cudaSuccess) return cuda_status(ea);
         configured[dev] = true;
     }
     const dim3 grid(unsigned(cdiv(N, tc::BN)), unsigned(w.tiles));
     cudaError_t e = launch_pdl(tc::gemm_tc_kernel<FMT>, grid, dim3(tc::NUM_THREADS), size_t(tc::SMEM_BYTES), stream,
                                M, N, K, group, (const __half*)w.tok, (const float*)w.dx16, (const float*)w.z, wq, ws,
                                wb, y);
-    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+    return cuda_status(e);
 }
 
 w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
@@ -204,6 +285,7 @@ w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype 
     w4a8_status st = check_gemm_args(M, N, K, x, dt, wq, ws, wb, FMT == 1, group, y, work, work_bytes, path);
     if (st != W4A8_OK) return st;
     const bool gemv = use_gemv(M, path);
+    if (gemv && gemv_fused(M, K)) return run_gemv_fused<FMT>(M, N, K, group, x, dt, wq, ws, wb, y, stream);
     st = prepare_impl(M, K, FMT == 1 ? group : 0, x, dt, work, gemv, stream);
     if (st != W4A8_OK) return st;
     return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, gemv, stream);
@@ -322,6 +404,8 @@ w4a8_status w4a8_last_device_error(void) {
     if (cudaMemcpyToSymbol(w4a8::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return W4A8_ERR_CUDA;
     return v ? W4A8_ERR_DEVICE_TIMEOUT : W4A8_OK;
 }
+
+const char* w4a8_last_cuda_error_string(void) { return cudaGetErrorString(t_last_cuda_error); }
 
 const char* w4a8_status_string(w4a8_status s) {
     switch (s) {

@@ -175,6 +175,10 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
  */
 w4a8_status w4a8_last_device_error(void);
 
+/* Description of the CUDA error behind the last W4A8_ERR_CUDA returned to this thread
+ * ("no error" if there was none). Static string, never NULL. */
+const char* w4a8_last_cuda_error_string(void);
+
 /* Static, human-readable name of a status code. */
 const char* w4a8_status_string(w4a8_status status);
 
