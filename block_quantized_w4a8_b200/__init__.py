@@ -28,8 +28,8 @@ PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 
 EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a8_gemm", "w4a8_gemm_ex",
            "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_prepare_act",
-           "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_last_device_error", "w4a8_last_cuda_error_string",
-           "w4a8_status_string"]
+           "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_gemm_noalloc", "w4a8_last_device_error",
+           "w4a8_last_cuda_error_string", "w4a8_status_string"]
 
 
 class W4A8Error(RuntimeError):
@@ -63,6 +63,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_prepare_act": (I, [I, I, I, P, I, P, Z, I, P]),
         "w4a8_gemm_prepared": (I, [I, I, I, P, P, P, P, Z, I, P]),
         "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
+        "w4a8_gemm_noalloc": (I, [I, I, I, P, I, P, P, P, P]),
         "w4a8_last_device_error": (I, []),
         "w4a8_status_string": (ctypes.c_char_p, [I]),
         "w4a8_last_cuda_error_string": (ctypes.c_char_p, []),
@@ -179,6 +180,15 @@ def w4a8_gemm_affine_prepared(M: int, K: int, group: int, q, scale, bias, y, ws,
            load_library().w4a8_gemm_affine_prepared(M, N, K, group, _ptr(q), _ptr(scale), _ptr(bias), _ptr(y),
                                                     _ptr(ws), ws.numel() * ws.element_size(), path,
                                                     _stream(stream)))
+
+
+def w4a8_gemm_noalloc(x, qs, d, y, stream=None) -> None:
+    """w4a8_gemm with the library's built-in scratch array instead of a caller workspace
+    (for callers that may not allocate device memory). Calls must not overlap on the GPU."""
+    M, K = x.shape
+    N = qs.shape[0]
+    _check("w4a8_gemm_noalloc", load_library().w4a8_gemm_noalloc(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d),
+                                                                 _ptr(y), _stream(stream)))
 
 
 def w4a8_last_device_error() -> int:

@@ -210,6 +210,26 @@ __device__ __forceinline__ void tmem_wait_ld64(uint32_t (&r)[64]) {
                  : "memory");
 }
 
+// 16 lanes x (8 columns x 4) of 32-bit words (tcgen05.ld.16x256b.x4): thread t gets, for
+// column group j = 0..3, r[4j+0..1] = row (lane base + t/4), columns 8j + 2(t%4) + {0,1}
+// and r[4j+2..3] = row (lane base + t/4 + 8), the same columns.
+__device__ __forceinline__ void tmem_ld_16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 // Packed f32 pair arithmetic (sm_100): acc += d * (x * w), lane-wise on two floats, each
 // operation rounded to nearest (no contraction across the multiply and the FMA).
 __device__ __forceinline__ void fma2_scaled(unsigned long long& acc, uint32_t d0, uint32_t d1, float x0, float x1,
@@ -221,6 +241,19 @@ __device__ __forceinline__ void fma2_scaled(unsigned long long& acc, uint32_t d0
         "fma.rn.f32x2 %0, dd, ss, %0;\n\t}\n"
         : "+l"(acc)
         : "r"(d0), "r"(d1), "f"(x0), "f"(x1), "l"(w2));
+}
+// acc += (d0, d1) * s2, lane-wise, one rounding per lane.
+__device__ __forceinline__ void fma2(unsigned long long& acc, uint32_t d0, uint32_t d1, unsigned long long s2) {
+    asm("{\n\t.reg .b64 dd;\n\t"
+        "mov.b64 dd, {%1, %2};\n\t"
+        "fma.rn.f32x2 %0, dd, %3, %0;\n\t}\n"
+        : "+l"(acc)
+        : "r"(d0), "r"(d1), "l"(s2));
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
 }
 // acc += b * (z0, z1)
 __device__ __forceinline__ void fma2_bias(unsigned long long& acc, float z0, float z1, unsigned long long b2) {

@@ -19,7 +19,8 @@
 // Warp roles (448 threads):
 //   WG0, WG1 (warps 0-7)  epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane
 //                         quarter) and token columns 64(w/4)..+63 of each block's
-//                         accumulator, scales them and accumulates in f32 registers
+//                         accumulator (16x256b loads: each thread 4 rows x 16 columns),
+//                         scales them and accumulates in f32 registers
 //   WG2 (warps 8-11)      producer: load packed 4-bit codes (16 B per row-block, two
 //                         stages ahead), expand to fp16 in the MMA's K-major core-matrix
 //                         layout, store the per-row scales
@@ -268,61 +269,100 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int p = (warp & 3) * 32 + lane;    // TMEM lane == weight row within the tile
-        const int col0 = (warp >> 2) * EPI_COLS; // first token column of this warp
-        unsigned long long acc[EPI_COLS / 2];    // f32 pairs
+        // Warp w covers TMEM lanes 32q..32q+31 (q = w%4, its hardware lane quarter) and
+        // token columns c0..c0+63 (c0 = 64*(w/4)). It reads them as 2 row halves x 2
+        // column groups with tcgen05.ld.16x256b.x4, so thread t owns weight rows
+        // 32q + t/4 + {0, 8, 16, 24} and token columns c0 + 8j + 2(t%4) + {0, 1}
+        // (j = 0..7): 4 row scales and 8 column-scale pairs per block instead of one
+        // broadcast column scale per accumulator.
+        const int q = warp & 3;
+        const int c0 = (warp >> 2) * EPI_COLS;
+        const int tr = lane >> 2, tc = (lane & 3) * 2;
+        unsigned long long acc[4][8];  // [row 0..3][column pair j]
 #pragma unroll
-        for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = 0ull;
-        const uint32_t lane_base = tmem_base + (uint32_t((warp & 3) * 32) << 16);
+        for (int r_ = 0; r_ < 4; ++r_)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[r_][j] = 0ull;
+        const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
         for (int i = 0; i < B; ++i) {
             const int st = i / S, k = i - st * S, slot = st % NS;
             const int buf = i % NACC;
             if (!bounded_wait_warp(bar(&ctrl->tfull[buf]), (i / NACC) & 1, abort)) break;
             tc_fence_after();
             const uint8_t* sp = stage_ptr(slot);
-            const float* dxs = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT + col0;
-            const float wsc = reinterpret_cast<const float*>(sp + OFF_WS)[k * BN + p];
-            const unsigned long long w2 = pack2(wsc, wsc);
+            const float* dxs = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT + c0 + tc;
+            const float* wss = reinterpret_cast<const float*>(sp + OFF_WS) + k * BN + q * 32 + tr;
+            // Four chunks per block, chunk c = (column group g = c/2, row half h = c%2);
+            // the TMEM load of chunk c+1 is issued before chunk c is scaled, so only the
+            // first load of a block is exposed.
+            const uint32_t tbase = lane_base + uint32_t(buf * TT + c0);
+            auto chunk_addr = [&](int c) { return tbase + (uint32_t(16 * (c & 1)) << 16) + uint32_t(32 * (c >> 1)); };
+            unsigned long long dx2[4];
+            auto load_dx = [&](int g) {
 #pragma unroll
-            for (int h = 0; h < EPI_COLS / 32; ++h) {  // two 32-column halves keep registers below the cap
-                uint32_t r[32];
-                tmem_ld_32x32(lane_base + uint32_t(buf * TT + col0 + h * 32), r);
-                tmem_wait_ld(r);
-                if (h == EPI_COLS / 32 - 1) {  // TMEM buffer free: every value is in registers
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(&ctrl->tempty[buf]));
-                }
+                for (int jj = 0; jj < 4; ++jj)
+                    dx2[jj] = *reinterpret_cast<const unsigned long long*>(dxs + 8 * (4 * g + jj));
+            };
+            auto scale_chunk = [&](int c, const uint32_t (&r)[16]) {
+                const int g = c >> 1, h = c & 1;
+                const float wa = wss[16 * h], wb = wss[16 * h + 8];
+                const unsigned long long wa2 = pack2(wa, wa), wb2 = pack2(wb, wb);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 dv = *reinterpret_cast<const float4*>(dxs + h * 32 + j);
-                    fma2_scaled(acc[(h * 32 + j) / 2], r[j], r[j + 1], dv.x, dv.y, w2);
-                    fma2_scaled(acc[(h * 32 + j) / 2 + 1], r[j + 2], r[j + 3], dv.z, dv.w, w2);
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = 4 * g + jj;
+                    fma2(acc[2 * h][j], r[4 * jj], r[4 * jj + 1], mul2(dx2[jj], wa2));
+                    fma2(acc[2 * h + 1][j], r[4 * jj + 2], r[4 * jj + 3], mul2(dx2[jj], wb2));
                 }
-            }
+            };
+            uint32_t ra[16], rb[16];
+            load_dx(0);
+            tmem_ld_16x256_x4(chunk_addr(0), ra);
+            tmem_wait_ld16(ra);
+            tmem_ld_16x256_x4(chunk_addr(1), rb);
+            scale_chunk(0, ra);
+            tmem_wait_ld16(rb);
+            tmem_ld_16x256_x4(chunk_addr(2), ra);
+            scale_chunk(1, rb);
+            tmem_wait_ld16(ra);
+            tmem_ld_16x256_x4(chunk_addr(3), rb);
+            load_dx(1);
+            scale_chunk(2, ra);
+            tmem_wait_ld16(rb);
+            tc_fence_before();  // TMEM buffer free: every value of the block is in registers
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(&ctrl->tempty[buf]));
+            scale_chunk(3, rb);
             if (FMT == 1 && ((i + 1) % bpg) == 0) {  // last block of a group: add bias * Z
-                const float bsc = reinterpret_cast<const float*>(sp + OFF_WB)[k * BN + p];
-                const unsigned long long b2 = pack2(bsc, bsc);
-                const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + (k / bpg) * TT + col0;
+                const float* bss = reinterpret_cast<const float*>(sp + OFF_WB) + k * BN + q * 32 + tr;
+                const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + (k / bpg) * TT + c0 + tc;
 #pragma unroll
-                for (int j = 0; j < EPI_COLS; j += 4) {
-                    const float4 zv = *reinterpret_cast<const float4*>(zs + j);
-                    fma2_bias(acc[j / 2], zv.x, zv.y, b2);
-                    fma2_bias(acc[j / 2 + 1], zv.z, zv.w, b2);
+                for (int r_ = 0; r_ < 4; ++r_) {
+                    const float bv = bss[8 * r_];
+                    const unsigned long long b2 = pack2(bv, bv);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float2 z = *reinterpret_cast<const float2*>(zs + 8 * j);
+                        fma2_bias(acc[r_][j], z.x, z.y, b2);
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0 && (k == S - 1 || i == B - 1)) mbar_arrive(bar(&ctrl->empty[slot]));
         }
-        const int n = n0 + p;
-        if (n < N && !*abort) {
+        if (!*abort) {
 #pragma unroll
-            for (int j = 0; j < EPI_COLS; j += 2) {
-                float a, b;
-                unpack2(acc[j / 2], a, b);
-                const int m = t * TT + col0 + j;
-                if (m < M) y[int64_t(m) * N + n] = a;
-                if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
+            for (int r_ = 0; r_ < 4; ++r_) {
+                const int n = n0 + q * 32 + tr + 8 * r_;
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float a, b;
+                        unpack2(acc[r_][j], a, b);
+                        const int m = t * TT + c0 + 8 * j + tc;
+                        if (m < M) y[int64_t(m) * N + n] = a;
+                        if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
+                    }
+                }
             }
         }
     }

@@ -396,6 +396,30 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
                             stream);
 }
 
+// Scratch of w4a8_gemm_noalloc. In host code this name is only a stand-in for the
+// device array; its device address comes from cudaGetSymbolAddress (once per device).
+static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_BYTES];
+
+w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
+                              const uint16_t* d_fp16, float* y, cudaStream_t stream) {
+    static void* scratch_ptr[64] = {nullptr};
+    const size_t need = w4a8_workspace_bytes(M, N, K, 0);
+    if (need == 0) return W4A8_ERR_INVALID_ARG;
+    if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
+    int dev = 0;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return cuda_status(ed);
+    if (dev < 0 || dev >= 64) return W4A8_ERR_UNSUPPORTED;
+    if (scratch_ptr[dev] == nullptr) {  // set-up, once per device, with that device current
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_status(e);
+        scratch_ptr[dev] = p;
+    }
+    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, scratch_ptr[dev], W4A8_NOALLOC_SCRATCH_BYTES,
+                        W4A8_PATH_AUTO, stream);
+}
+
 w4a8_status w4a8_last_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return W4A8_ERR_CUDA;
     unsigned int v = 0;

@@ -168,6 +168,31 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
                                       cudaStream_t stream);
 
 /*
+ * w4a8_gemm for callers that cannot allocate device memory. Some callers are not allowed
+ * to call cudaMalloc at all: a host application that reserves every byte of device memory
+ * up front and owns its allocator, or a plug-in interface whose call signature carries
+ * only the inputs and the output, so there is nowhere to pass a workspace. This entry
+ * point computes exactly what w4a8_gemm computes (same kernels, same results) but takes
+ * its scratch from a buffer compiled into the library: a static device array of
+ * W4A8_NOALLOC_SCRATCH_BYTES (every GPU that loads the library holds it until the process
+ * exits). The library itself never calls cudaMalloc or cudaFree here.
+ *  - The first call on each device looks up that array's device address (with that device
+ *    current), so that first call should come before any stream capture.
+ *  - Shapes whose workspace (w4a8_workspace_bytes(M, N, K, 0)) exceeds the array are
+ *    rejected with W4A8_ERR_WORKSPACE; nothing is launched.
+ *  - Every call on a device shares the one array and the array keeps whatever the last call
+ *    left in it (the kernels overwrite what they read, nothing needs to start at zero).
+ *    Calls whose work overlaps on the GPU (different streams, or several host threads
+ *    without ordering) race on that array and corrupt each other's results: order them.
+ * Arguments and the other errors as w4a8_gemm. This entry point has no counterpart on the
+ * pages; it is a packaging of w4a8_gemm for allocation-free callers.
+ */
+#define W4A8_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dtype,
+                              const uint8_t* qs, const uint16_t* d_fp16, float* y,
+                              cudaStream_t stream);
+
+/*
  * Reads and clears the device status word that kernels set when a bounded wait runs
  * out. Synchronises the current device. Returns W4A8_OK when no kernel has reported a
  * problem since the last call, W4A8_ERR_DEVICE_TIMEOUT otherwise, W4A8_ERR_CUDA if the
