@@ -62,12 +62,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // when `*abort` is raised by another thread or after kWaitLimitNs; in the latter case
 // it records kDevErrTimeout in the device status word and raises `*abort` itself.
 // Returns false when it gave up. Called by one thread.
-__device__ __noinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool bounded_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
     const unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        {
+        if ((it & 15u) == 0u) {
             if (*abort) return false;
             if (global_timer_ns() - t0 > kWaitLimitNs) {
                 atomicOr(&g_device_status, kDevErrTimeout);
@@ -76,6 +75,40 @@ __device__ __noinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return bounded_wait_slow(bar, parity, abort);
+}
+
+// Named hardware barrier over `nthreads` threads (whole warps); waiting warps issue
+// nothing until the last one arrives.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also ANDs a predicate over the participating threads.
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(uint32_t(v)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// Group-wide wait: one thread of the group polls the mbarrier, the others block on a
+// named barrier, so only one warp of the group spends issue slots while waiting. All
+// threads of the group must call it together; the barrier's AND hands every one of them
+// the leader's result, so the group never splits.
+__device__ __forceinline__ bool bounded_wait_group(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                                   bool leader, uint32_t barrier_id, uint32_t nthreads) {
+    const bool ok = leader ? bounded_wait(bar, parity, abort) : true;
+    return named_barrier_and(barrier_id, nthreads, ok);
 }
 
 // Warp-uniform variant: lane 0 waits, the outcome is broadcast so that every lane of
@@ -230,6 +263,28 @@ __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
                  : "memory");
 }
 
+// 32 lanes x 16 columns (registers valid after the next tcgen05.wait::ld).
+__device__ __forceinline__ void tmem_ld_32x32_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Waits for this thread's outstanding tensor-memory loads; both register sets are
+// threaded through the asm so that no use of them moves above the wait.
+__device__ __forceinline__ void tmem_wait_ld16x2(uint32_t (&a)[16], uint32_t (&b)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                   "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]),
+                   "+r"(a[15]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]),
+                   "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]),
+                   "+r"(b[14]), "+r"(b[15])
+                 :
+                 : "memory");
+}
+
 // Packed f32 pair arithmetic (sm_100): acc += d * (x * w), lane-wise on two floats, each
 // operation rounded to nearest (no contraction across the multiply and the FMA).
 __device__ __forceinline__ void fma2_scaled(unsigned long long& acc, uint32_t d0, uint32_t d1, float x0, float x1,
@@ -254,6 +309,15 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
     unsigned long long r;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
+}
+// acc += (p0, p1) * (s0, s1), lane-wise, one rounding per lane.
+__device__ __forceinline__ void fma2_pp(unsigned long long& acc, uint32_t p0, uint32_t p1, uint32_t s0, uint32_t s1) {
+    asm("{\n\t.reg .b64 pp, ss;\n\t"
+        "mov.b64 pp, {%1, %2};\n\t"
+        "mov.b64 ss, {%3, %4};\n\t"
+        "fma.rn.f32x2 %0, pp, ss, %0;\n\t}\n"
+        : "+l"(acc)
+        : "r"(p0), "r"(p1), "r"(s0), "r"(s1));
 }
 // acc += b * (z0, z1)
 __device__ __forceinline__ void fma2_bias(unsigned long long& acc, float z0, float z1, unsigned long long b2) {

@@ -5,31 +5,35 @@
 // #2432, "The kernel": Q4_0's per-32-block scales force a per-block rescale; there it
 // is one vector multiply per block over accumulator lanes that each hold one output).
 // Here every block gets its own tensor-memory accumulator: TMEM lane = weight row,
-// TMEM column = token, so each epilogue thread owns one output row and rescales its
-// columns with a per-thread (weight) and a per-column (activation) scale, with no
+// TMEM column = token, so each epilogue thread owns one output row and needs no
 // cross-lane reduction.
 //
-// Operands are fp16 holding small integers, so the MMA (kind::f16, f32 accumulate) is
-// exact: weight codes (q-8 or 16(q-8); affine q or 16q) times activation codes (16q_x or
-// q_x, see quant_act_tc_kernel), every product an integer below 2^15 and every block
-// sum below 2^20. The block dot comes out of TMEM as 16*D in f32 with no conversion.
+// Per block the tensor core produces two 128 x 128 tiles in TMEM:
+//   P = 16 * D      two kind::f16 MMAs on fp16 operands that hold small integers (weight
+//                   codes q-8 or 16(q-8), affine q or 16q; activation codes 16q_x or q_x,
+//                   see quant_act_tc_kernel): every product and block sum is an exact
+//                   integer below 2^20, so P is exact.
+//   S = s_w (x) d_x/16   one kind::tf32 MMA with K = 8: the weight side holds
+//                   (s_w, s_w, s_w, .) per row, the activation side (a, b, c, 0) with
+//                   a + b + c = d_x/16 exactly, the second K-chunk of both points at a
+//                   zero region. So S = s_w * d_x / 16 up to the accumulator's rounding.
+// The epilogue then does acc += P * S per element: one FMA, no per-column scale traffic
+// through shared memory (the outer product of the scales comes from the tensor core).
 //
-// CTA tile: 128 weight rows x 128 tokens; one pipeline stage = 4 quant blocks (K=128),
-// 3 stages; 4 TMEM accumulator buffers of 128 columns (the whole 512-column TMEM).
-// Warp roles (448 threads):
-//   WG0, WG1 (warps 0-7)  epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane
-//                         quarter) and token columns 64(w/4)..+63 of each block's
-//                         accumulator (16x256b loads: each thread 4 rows x 16 columns),
-//                         scales them and accumulates in f32 registers
-//   WG2 (warps 8-11)      producer: load packed 4-bit codes (16 B per row-block, two
-//                         stages ahead), expand to fp16 in the MMA's K-major core-matrix
-//                         layout, store the per-row scales
-//   warp 12               TMEM allocation + single-thread MMA issue
-//   warp 13               one thread issuing the bulk copies of the token operand and
-//                         its scales
-// The kernel runs one CTA per SM with 128 registers per thread.
-// Every wait is bounded (bounded_wait); on a timeout all roles stop, outstanding copies
-// and MMAs are drained, TMEM is freed and the kernel returns.
+// CTA tile: 128 weight rows x 128 tokens; one pipeline stage = 2 quant blocks (K = 64),
+// 4 stages; 2 block buffers in TMEM, each a P tile and an S tile (512 columns in all).
+// Warp roles (704 threads):
+//   warps 0-15   epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane quarter)
+//                and token columns 32(w/4)..+31 of P and S, accumulates in f32 registers
+//   warps 16-19  producer: load packed 4-bit codes (16 B per row-block, two stages
+//                ahead), expand to fp16 in the MMA's K-major core-matrix layout, store
+//                the row's scale operand (and the affine bias) per block
+//   warp 20      TMEM allocation + single-thread MMA issue
+//   warp 21      one thread issuing the bulk copies of the token operand, its scale
+//                operand and (affine) the per-group bias factor
+// Every wait is bounded (bounded_wait); within the epilogue and the producer one thread
+// polls and the other warps block on a named barrier. On a timeout all roles stop,
+// outstanding copies and MMAs are drained, TMEM is freed and the kernel returns.
 #pragma once
 
 #include "device_common.cuh"
@@ -40,42 +44,46 @@ namespace tc {
 
 constexpr int BN = 128;                   // weight rows per CTA (MMA M, TMEM lanes)
 constexpr int TT = tcgeo::kTokTile;       // tokens per CTA (MMA N)
-constexpr int S = 4;                      // quant blocks per stage
-constexpr int NS = 3;                     // stages in the ring
-constexpr int NACC = 4;                   // TMEM accumulator buffers
+constexpr int S = 2;                      // quant blocks per stage
+constexpr int NS = 4;                     // stages in the ring
+constexpr int NBUF = 2;                   // TMEM block buffers (each P + S)
 constexpr int A_BLK = BN * 64;            // fp16 weight operand bytes per block
 constexpr int B_BLK = tcgeo::kTokBlockBytes;
+constexpr int AS_BLK = BN * 16;           // tf32 scale operand, first K-chunk, weight side
+constexpr int BS_BLK = TT * 16;           // tf32 scale operand, first K-chunk, token side
 constexpr int OFF_B = S * A_BLK;
-constexpr int OFF_DX = OFF_B + S * B_BLK;
-constexpr int OFF_WS = OFF_DX + S * TT * 4;
-constexpr int OFF_WB = OFF_WS + S * BN * 4;
-constexpr int OFF_Z = OFF_WB + S * BN * 4;
-constexpr int STAGE_BYTES = OFF_Z + S * TT * 4;
+constexpr int OFF_AS = OFF_B + S * B_BLK;
+constexpr int OFF_BS = OFF_AS + S * AS_BLK;
+constexpr int OFF_Z = OFF_BS + S * BS_BLK;
+constexpr int STAGE_BYTES = OFF_Z + TT * 4;   // + one group's bias factor (affine)
+constexpr int ZERO_BYTES = 128 * 16;          // second K-chunk of both scale operands
 constexpr int CTRL_BYTES = 256;
-constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;  // + alignment slack
-constexpr int TMEM_COLS = NACC * TT;
-constexpr int EPI_WARPS = 8;
-constexpr int EPI_COLS = TT / (EPI_WARPS / 4);   // token columns per epilogue warp (64)
-constexpr int PROD_WARP0 = 8;
-constexpr int MMA_WARP = 12;
-constexpr int COPY_WARP = 13;
-constexpr int NUM_THREADS = 448;
-constexpr int MAX_REGS = 128;
-constexpr uint32_t IDESC = idesc_f16_f32(BN, TT);
-constexpr uint32_t LBO = 128, SBO = 512;  // core-matrix strides (K, M/N)
+constexpr int SMEM_BYTES = NS * STAGE_BYTES + ZERO_BYTES + CTRL_BYTES + 1024;  // + alignment slack
+constexpr int TMEM_COLS = 512;
+constexpr int P_COL0 = 0, S_COL0 = NBUF * TT;  // P tiles in columns 0..255, S tiles 256..511
+constexpr int EPI_WARPS = 16;
+constexpr int EPI_COLS = 32;                   // token columns per epilogue warp
+constexpr int PROD_WARP0 = 16;
+constexpr int MMA_WARP = 20;
+constexpr int COPY_WARP = 21;
+constexpr int NUM_THREADS = 22 * 32;
+constexpr uint32_t IDESC_P = idesc_f16_f32(BN, TT);
+// kind::tf32: D f32, A and B tf32 (format 2), K-major, M x N
+constexpr uint32_t IDESC_S = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(TT >> 3) << 17) | (uint32_t(BN >> 4) << 24);
+constexpr uint32_t LBO = 128, SBO = 512;   // fp16 operands: core-matrix strides (K, M/N)
+constexpr uint32_t SBO_S = 128;            // tf32 scale operands: 8-row groups 128 B apart
 
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-static_assert(TMEM_COLS == 512, "tmem allocation must be a power of two >= 32");
-static_assert(EPI_COLS == 64, "epilogue loads 64 columns per warp");
-static_assert(NUM_THREADS * MAX_REGS <= 65536, "register file");
+static_assert(EPI_WARPS * EPI_COLS == 4 * TT, "epilogue covers the tile");
+static_assert(NBUF * 2 * TT == TMEM_COLS, "tmem columns");
 
 struct Ctrl {
     unsigned long long full_a[NS];    // producer threads (128 arrivals)
     unsigned long long full_b[NS];    // bulk copies (1 arrival + bytes)
     unsigned long long empty[NS];     // MMA commit + one arrival per epilogue warp
-    unsigned long long tfull[NACC];   // MMA commit
-    unsigned long long tempty[NACC];  // one arrival per epilogue warp
+    unsigned long long tfull[NBUF];   // MMA commit
+    unsigned long long tempty[NBUF];  // one arrival per epilogue warp
     unsigned long long drain;         // final MMA drain
     uint32_t tmem_base;
     uint32_t abort;
@@ -104,6 +112,17 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
     return make_uint4(sub(ea, off_lo), sub(eb, off_lo), sub(ec, off_hi), sub(ed, off_hi));
 }
 
+// tf32 MMA: D[tmem] (+)= A[smem] * B[smem]^T, both K-major, f32 accumulator.
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Codes and scales of one stage of one weight row, held in registers until stored.
 struct RowStage {
     uint4 w[S];
@@ -112,13 +131,14 @@ struct RowStage {
 
 template <int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dx16,
+    gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float4* __restrict__ bs,
                    const float* __restrict__ zb, const uint8_t* __restrict__ wq,
                    const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
                    float* __restrict__ y) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + NS * STAGE_BYTES);
+    uint8_t* zero = smem + NS * STAGE_BYTES;
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(zero + ZERO_BYTES);
     volatile uint32_t* abort = &ctrl->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,13 +152,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
     auto bar = [](unsigned long long* p) { return smem_addr(p); };
 
+    for (int i = threadIdx.x; i < ZERO_BYTES / 16; i += NUM_THREADS)
+        reinterpret_cast<uint4*>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(bar(&ctrl->full_a[s]), 128);
             mbar_init(bar(&ctrl->full_b[s]), 1);
             mbar_init(bar(&ctrl->empty[s]), 1 + EPI_WARPS);
         }
-        for (int j = 0; j < NACC; ++j) {
+        for (int j = 0; j < NBUF; ++j) {
             mbar_init(bar(&ctrl->tfull[j]), 1);
             mbar_init(bar(&ctrl->tempty[j]), EPI_WARPS);
         }
@@ -150,6 +172,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc(smem_addr(&ctrl->tmem_base), TMEM_COLS);
         tmem_relinquish();
     }
+    fence_proxy_async_smem();  // the zero region is read by the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -185,7 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Store one stage into shared memory; false if the wait gave up.
         auto produce = [&](int st, const RowStage& rs) {
             const int slot = st % NS;
-            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) return false;
+            if (!bounded_wait_group(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort, p == 0, 2, 128)) return false;
             uint8_t* sp = stage_ptr(slot);
 #pragma unroll
             for (int k = 0; k < S; ++k) {
@@ -193,8 +216,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint8_t* arow = sp + k * A_BLK + (p >> 3) * 512 + (p & 7) * 16;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(arow + c * 128) = expand_word<FMT>(w[c]);
-                reinterpret_cast<float*>(sp + OFF_WS)[k * BN + p] = rs.s[k];
-                if (FMT == 1) reinterpret_cast<float*>(sp + OFF_WB)[k * BN + p] = rs.b[k];
+                // scale operand (s, s, s, bias): the fourth slot meets a zero on the token
+                // side, so it only carries the affine bias to the epilogue
+                reinterpret_cast<float4*>(sp + OFF_AS + k * AS_BLK)[p] = make_float4(rs.s[k], rs.s[k], rs.s[k], rs.b[k]);
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(&ctrl->full_a[slot]));
@@ -216,22 +240,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp >= MMA_WARP) {
         if (warp == COPY_WARP && lane == 0) {
             // -------------------------------------------------------- bulk copies
-            pdl_wait_primary();  // the token operand is written by the preceding kernel
+            pdl_wait_primary();  // the token operands are written by the preceding kernel
             int issued = 0;
             for (int st = 0; st < nstages; ++st) {
                 const int slot = st % NS;
                 if (!bounded_wait(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) break;
                 const int b0 = st * S;
                 const int nb = min(S, B - b0);
-                const uint32_t bytes_tok = nb * B_BLK, bytes_dx = nb * TT * 4;
-                const uint32_t bytes_z = (FMT == 1) ? (nb / bpg) * TT * 4 : 0;
+                // affine: the bias factor of the group whose last block is in this stage
+                const bool zlast = (FMT == 1) && (((b0 + nb) % bpg) == 0);
+                const uint32_t bytes_tok = nb * B_BLK, bytes_bs = nb * BS_BLK;
+                const uint32_t bytes_z = zlast ? TT * 4 : 0;
                 const uint32_t fb = bar(&ctrl->full_b[slot]);
                 uint8_t* sp = stage_ptr(slot);
-                mbar_arrive_expect_tx(fb, bytes_tok + bytes_dx + bytes_z);
+                mbar_arrive_expect_tx(fb, bytes_tok + bytes_bs + bytes_z);
                 bulk_g2s(smem_addr(sp + OFF_B), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * B_BLK,
                          bytes_tok, fb);
-                bulk_g2s(smem_addr(sp + OFF_DX), dx16 + (int64_t(t) * B + b0) * TT, bytes_dx, fb);
-                if (FMT == 1) bulk_g2s(smem_addr(sp + OFF_Z), zb + (int64_t(t) * G + b0 / bpg) * TT, bytes_z, fb);
+                bulk_g2s(smem_addr(sp + OFF_BS), bs + (int64_t(t) * B + b0) * TT, bytes_bs, fb);
+                if (zlast) bulk_g2s(smem_addr(sp + OFF_Z), zb + (int64_t(t) * G + (b0 + nb - 1) / bpg) * TT, bytes_z, fb);
                 issued = st + 1;
             }
             // Let every copy this thread issued land before the CTA can exit (on the
@@ -241,6 +267,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 bounded_wait(bar(&ctrl->full_b[st % NS]), (st / NS) & 1, &local_abort);
         } else if (warp == MMA_WARP && lane == 0) {
             // -------------------------------------------------------- MMA issue
+            const uint32_t zero_addr = smem_addr(zero);
             for (int i = 0; i < B; ++i) {
                 const int st = i / S, k = i - st * S, slot = st % NS;
                 const uint32_t par = (st / NS) & 1;
@@ -248,16 +275,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (!bounded_wait(bar(&ctrl->full_a[slot]), par, abort)) break;
                     if (!bounded_wait(bar(&ctrl->full_b[slot]), par, abort)) break;
                 }
-                const int buf = i % NACC;
-                if (!bounded_wait(bar(&ctrl->tempty[buf]), ((i / NACC) & 1) ^ 1, abort)) break;
+                const int buf = i % NBUF;
+                if (!bounded_wait(bar(&ctrl->tempty[buf]), ((i / NBUF) & 1) ^ 1, abort)) break;
                 tc_fence_after();
-                const uint32_t a_addr = smem_addr(stage_ptr(slot) + k * A_BLK);
-                const uint32_t b_addr = smem_addr(stage_ptr(slot) + OFF_B + k * B_BLK);
+                uint8_t* sp = stage_ptr(slot);
+                const uint32_t a_addr = smem_addr(sp + k * A_BLK);
+                const uint32_t b_addr = smem_addr(sp + OFF_B + k * B_BLK);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    tc_mma_f16(tmem_base + uint32_t(buf * TT), smem_desc_kmajor(a_addr + h * 256, LBO, SBO),
-                               smem_desc_kmajor(b_addr + h * 256, LBO, SBO), IDESC, h);
+                    tc_mma_f16(tmem_base + uint32_t(P_COL0 + buf * TT), smem_desc_kmajor(a_addr + h * 256, LBO, SBO),
+                               smem_desc_kmajor(b_addr + h * 256, LBO, SBO), IDESC_P, h);
                 }
+                const uint32_t as_addr = smem_addr(sp + OFF_AS + k * AS_BLK);
+                const uint32_t bs_addr = smem_addr(sp + OFF_BS + k * BS_BLK);
+                tc_mma_tf32(tmem_base + uint32_t(S_COL0 + buf * TT),
+                            smem_desc_kmajor(as_addr, zero_addr - as_addr, SBO_S),
+                            smem_desc_kmajor(bs_addr, zero_addr - bs_addr, SBO_S), IDESC_S, 0);
                 tc_commit(bar(&ctrl->tfull[buf]));
                 if (k == S - 1 || i == B - 1) tc_commit(bar(&ctrl->empty[slot]));
             }
@@ -269,100 +302,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Warp w covers TMEM lanes 32q..32q+31 (q = w%4, its hardware lane quarter) and
-        // token columns c0..c0+63 (c0 = 64*(w/4)). It reads them as 2 row halves x 2
-        // column groups with tcgen05.ld.16x256b.x4, so thread t owns weight rows
-        // 32q + t/4 + {0, 8, 16, 24} and token columns c0 + 8j + 2(t%4) + {0, 1}
-        // (j = 0..7): 4 row scales and 8 column-scale pairs per block instead of one
-        // broadcast column scale per accumulator.
-        const int q = warp & 3;
-        const int c0 = (warp >> 2) * EPI_COLS;
-        const int tr = lane >> 2, tc = (lane & 3) * 2;
-        unsigned long long acc[4][8];  // [row 0..3][column pair j]
+        const int q = warp & 3;                    // lane quarter: weight rows 32q..32q+31
+        const int c0 = (warp >> 2) * EPI_COLS;     // token columns c0..c0+31
+        const int p = q * 32 + lane;               // this thread's weight row within the tile
+        unsigned long long acc[EPI_COLS / 2];      // f32 pairs
 #pragma unroll
-        for (int r_ = 0; r_ < 4; ++r_)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[r_][j] = 0ull;
+        for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = 0ull;
         const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
         for (int i = 0; i < B; ++i) {
             const int st = i / S, k = i - st * S, slot = st % NS;
-            const int buf = i % NACC;
-            if (!bounded_wait_warp(bar(&ctrl->tfull[buf]), (i / NACC) & 1, abort)) break;
+            const int buf = i % NBUF;
+            if (!bounded_wait_group(bar(&ctrl->tfull[buf]), (i / NBUF) & 1, abort, threadIdx.x == 0, 1,
+                                    EPI_WARPS * 32))
+                break;
             tc_fence_after();
-            const uint8_t* sp = stage_ptr(slot);
-            const float* dxs = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT + c0 + tc;
-            const float* wss = reinterpret_cast<const float*>(sp + OFF_WS) + k * BN + q * 32 + tr;
-            // Four chunks per block, chunk c = (column group g = c/2, row half h = c%2);
-            // the TMEM load of chunk c+1 is issued before chunk c is scaled, so only the
-            // first load of a block is exposed.
-            const uint32_t tbase = lane_base + uint32_t(buf * TT + c0);
-            auto chunk_addr = [&](int c) { return tbase + (uint32_t(16 * (c & 1)) << 16) + uint32_t(32 * (c >> 1)); };
-            unsigned long long dx2[4];
-            auto load_dx = [&](int g) {
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    dx2[jj] = *reinterpret_cast<const unsigned long long*>(dxs + 8 * (4 * g + jj));
-            };
-            auto scale_chunk = [&](int c, const uint32_t (&r)[16]) {
-                const int g = c >> 1, h = c & 1;
-                const float wa = wss[16 * h], wb = wss[16 * h + 8];
-                const unsigned long long wa2 = pack2(wa, wa), wb2 = pack2(wb, wb);
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = 4 * g + jj;
-                    fma2(acc[2 * h][j], r[4 * jj], r[4 * jj + 1], mul2(dx2[jj], wa2));
-                    fma2(acc[2 * h + 1][j], r[4 * jj + 2], r[4 * jj + 3], mul2(dx2[jj], wb2));
+            for (int h = 0; h < EPI_COLS / 16; ++h) {
+                uint32_t pr[16], sr[16];
+                tmem_ld_32x32_x16(lane_base + uint32_t(P_COL0 + buf * TT + c0 + 16 * h), pr);
+                tmem_ld_32x32_x16(lane_base + uint32_t(S_COL0 + buf * TT + c0 + 16 * h), sr);
+                tmem_wait_ld16x2(pr, sr);
+                if (h == EPI_COLS / 16 - 1) {  // TMEM buffer free: every value is in registers
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(&ctrl->tempty[buf]));
                 }
-            };
-            uint32_t ra[16], rb[16];
-            load_dx(0);
-            tmem_ld_16x256_x4(chunk_addr(0), ra);
-            tmem_wait_ld16(ra);
-            tmem_ld_16x256_x4(chunk_addr(1), rb);
-            scale_chunk(0, ra);
-            tmem_wait_ld16(rb);
-            tmem_ld_16x256_x4(chunk_addr(2), ra);
-            scale_chunk(1, rb);
-            tmem_wait_ld16(ra);
-            tmem_ld_16x256_x4(chunk_addr(3), rb);
-            load_dx(1);
-            scale_chunk(2, ra);
-            tmem_wait_ld16(rb);
-            tc_fence_before();  // TMEM buffer free: every value of the block is in registers
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(&ctrl->tempty[buf]));
-            scale_chunk(3, rb);
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) fma2_pp(acc[8 * h + j / 2], pr[j], pr[j + 1], sr[j], sr[j + 1]);
+            }
             if (FMT == 1 && ((i + 1) % bpg) == 0) {  // last block of a group: add bias * Z
-                const float* bss = reinterpret_cast<const float*>(sp + OFF_WB) + k * BN + q * 32 + tr;
-                const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + (k / bpg) * TT + c0 + tc;
+                const uint8_t* sp = stage_ptr(slot);
+                const float bsc = reinterpret_cast<const float4*>(sp + OFF_AS + k * AS_BLK)[p].w;
+                const unsigned long long b2 = pack2(bsc, bsc);
+                const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + c0;
 #pragma unroll
-                for (int r_ = 0; r_ < 4; ++r_) {
-                    const float bv = bss[8 * r_];
-                    const unsigned long long b2 = pack2(bv, bv);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float2 z = *reinterpret_cast<const float2*>(zs + 8 * j);
-                        fma2_bias(acc[r_][j], z.x, z.y, b2);
-                    }
+                for (int j = 0; j < EPI_COLS; j += 4) {
+                    const float4 zv = *reinterpret_cast<const float4*>(zs + j);
+                    fma2_bias(acc[j / 2], zv.x, zv.y, b2);
+                    fma2_bias(acc[j / 2 + 1], zv.z, zv.w, b2);
                 }
             }
             __syncwarp();
             if (lane == 0 && (k == S - 1 || i == B - 1)) mbar_arrive(bar(&ctrl->empty[slot]));
         }
-        if (!*abort) {
+        const int n = n0 + p;
+        if (n < N && !*abort) {
 #pragma unroll
-            for (int r_ = 0; r_ < 4; ++r_) {
-                const int n = n0 + q * 32 + tr + 8 * r_;
-                if (n < N) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        float a, b;
-                        unpack2(acc[r_][j], a, b);
-                        const int m = t * TT + c0 + 8 * j + tc;
-                        if (m < M) y[int64_t(m) * N + n] = a;
-                        if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
-                    }
-                }
+            for (int j = 0; j < EPI_COLS; j += 2) {
+                float a, b;
+                unpack2(acc[j / 2], a, b);
+                const int m = t * TT + c0 + j;
+                if (m < M) y[int64_t(m) * N + n] = a;
+                if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
             }
         }
     }

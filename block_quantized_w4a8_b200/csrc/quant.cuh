@@ -77,12 +77,16 @@ __global__ void __launch_bounds__(256) quant_act_rowmajor_kernel(const void* __r
 //   FMT 1 (affine): 8c, 8c+4, 8c+2, 8c+6, 8c+1, 8c+5, 8c+3, 8c+7
 // Slots 0..3 store 16*q (the weight side holds the plain code there) and slots 4..7
 // store q (the weight side holds 16*code there), so every product is 16*(w_code*q):
-// the GEMM's block dot is exactly 16x the integer dot, and the stored scale is d/16
-// (exact). Rows past M are zero. For FMT 1 it also writes, per token and weight group
-// g, Z = sum over the group's blocks of d*sum(q) (the factor of the bias term).
+// the GEMM's block dot is exactly 16x the integer dot.
+// The block scale goes to `bs` as the tf32 operand of the GEMM's scale MMA: per chunk,
+// token r at 16 bytes (a, b, c, 0) with a + b + c == d/16 exactly (a keeps the top 11
+// significant bits of d/16, b the next 11, c the rest; each is representable in tf32,
+// whose low 13 mantissa bits are zero). Rows past M are zero. For FMT 1 it also writes,
+// per token and weight group g, Z = sum over the group's blocks of d*sum(q) (the factor
+// of the bias term).
 template <bool BF16, int FMT>
 __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restrict__ x, int M, int K, int64_t nblocks,
-                                                           __half* __restrict__ tok, float* __restrict__ dx16,
+                                                           __half* __restrict__ tok, float4* __restrict__ bs,
                                                            float* __restrict__ zb, int group) {
     using namespace tcgeo;
     pdl_launch_dependents();
@@ -137,7 +141,14 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         char* dst = reinterpret_cast<char*>(tok) + chunk * kTokBlockBytes + (r >> 3) * 512 + c * 128 + (r & 7) * 16;
         *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
     }
-    if (valid && sub == 0) dx16[chunk * kTokTile + r] = __fmul_rn(d, 0.0625f);
+    if (valid && sub == 0) {
+        const float d16 = __fmul_rn(d, 0.0625f);
+        const float a = __uint_as_float(__float_as_uint(d16) & 0xFFFFE000u);
+        const float r1 = __fsub_rn(d16, a);  // exact: the low 13 significand bits of d16
+        const float b2 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+        const float c2 = __fsub_rn(r1, b2);  // exact, at most 2 significant bits
+        bs[chunk * kTokTile + r] = make_float4(a, b2, c2, 0.0f);
+    }
     if (FMT == 1) {
         // Blocks of one weight group are adjacent 8-lane groups of this warp (the warp's
         // four blocks start at a multiple of 4 and B is a multiple of group/32).

@@ -54,7 +54,7 @@ GemvWs gemv_ws(void* ws, int M, int K) {
 
 struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
     __half* tok;
-    float* dx16;
+    float4* bs;
     float* z;
     int tiles;
     size_t bytes;
@@ -67,7 +67,7 @@ TcWs tc_ws(void* ws, int M, int K, int group) {
     size_t off = 0;
     char* base = static_cast<char*>(ws);
     w.tok = reinterpret_cast<__half*>(base + off); off = align256(off + size_t(rows) * B * 64);
-    w.dx16 = reinterpret_cast<float*>(base + off); off = align256(off + size_t(rows) * B * 4);
+    w.bs = reinterpret_cast<float4*>(base + off); off = align256(off + size_t(rows) * B * 16);
     w.z = reinterpret_cast<float*>(base + off);
     if (group > 0) off = align256(off + size_t(rows) * (K / group) * 4);
     w.bytes = off;
@@ -106,14 +106,14 @@ w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, 
     const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
     if (group == 0) {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, 0);
+            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, 0);
         else
-            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, 0);
+            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, 0);
     } else {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, group);
+            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, group);
         else
-            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.dx16, w.z, group);
+            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, group);
     }
     return launch_status();
 }
@@ -232,7 +232,7 @@ w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uin
     }
     const dim3 grid(unsigned(cdiv(N, tc::BN)), unsigned(w.tiles));
     cudaError_t e = launch_pdl(tc::gemm_tc_kernel<FMT>, grid, dim3(tc::NUM_THREADS), size_t(tc::SMEM_BYTES), stream,
-                               M, N, K, group, (const __half*)w.tok, (const float*)w.dx16, (const float*)w.z, wq, ws,
+                               M, N, K, group, (const __half*)w.tok, (const float4*)w.bs, (const float*)w.z, wq, ws,
                                wb, y);
     return cuda_status(e);
 }

@@ -54,7 +54,7 @@ def test_workspace_bytes(lib, M, N, K, group):
     B = K // 32
     gemv = _align(M * K) + _align(M * B * 4) + _align(M * B * 4)
     rows = -(-M // 128) * 128
-    tc = _align(rows * B * 64) + _align(rows * B * 4) + (_align(rows * (K // group) * 4) if group else 0)
+    tc = _align(rows * B * 64) + _align(rows * B * 16) + (_align(rows * (K // group) * 4) if group else 0)
     assert w4a8.w4a8_workspace_bytes(M, N, K, group) == max(gemv, tc)
 
 
