@@ -504,8 +504,8 @@ def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
 
 
 def run_probe(args):
-    """A short, fixed sequence of launches for ncu: per step one prepare (act quant) and
-    one contraction, each through the C ABI, on the workload named by --probe."""
+    """A short, fixed sequence of launches for ncu: `--steps` calls of w4a8_gemm (or
+    w4a8_gemm_affine) through the C ABI on the workload named by --probe."""
     import torch
     import block_quantized_w4a8_b200 as w4a8
     from block_quantized_w4a8_b200 import inputs
@@ -528,13 +528,11 @@ def run_probe(args):
     else:
         qs, d = w4a8.pack_q4_0(wd)
     torch.cuda.synchronize()
-    for _ in range(args.steps):
+    for _ in range(args.steps):  # the public call one benchmark step makes
         if g:
-            w4a8.w4a8_prepare_act(xd, ws, g)
-            w4a8.w4a8_gemm_affine_prepared(wl.M, wl.K, g, q, s, b, y, ws)
+            w4a8.w4a8_gemm_affine(xd, q, s, b, y, ws, g)
         else:
-            w4a8.w4a8_prepare_act(xd, ws)
-            w4a8.w4a8_gemm_prepared(wl.M, wl.K, qs, d, y, ws)
+            w4a8.w4a8_gemm(xd, qs, d, y, ws)
     torch.cuda.synchronize()
     assert w4a8.w4a8_last_device_error() == 0
     print(f"probe {wl.name}: {args.steps} steps ok")
