@@ -20,17 +20,17 @@
 // The epilogue then does acc += P * S per element: one FMA, no per-column scale traffic
 // through shared memory (the outer product of the scales comes from the tensor core).
 //
-// CTA tile: 128 weight rows x 128 tokens; one pipeline stage = 2 quant blocks (K = 64),
-// 4 stages; 2 block buffers in TMEM, each a P tile and an S tile (512 columns in all).
-// Warp roles (704 threads):
-//   warps 0-15   epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane quarter)
-//                and token columns 32(w/4)..+31 of P and S, accumulates in f32 registers
-//   warps 16-19  producer: load packed 4-bit codes (16 B per row-block, two stages
-//                ahead), expand to fp16 in the MMA's K-major core-matrix layout, store
-//                the row's scale operand (and the affine bias) per block
-//   warp 20      TMEM allocation + single-thread MMA issue
-//   warp 21      one thread issuing the bulk copies of the token operand, its scale
-//                operand and (affine) the per-group bias factor
+// CTA tile: 128 weight rows x TT tokens (TT = 32, 64 or 128); one pipeline stage = 2
+// quant blocks (K = 64), 4-7 stages; 512/(2 TT) block buffers in TMEM, each a P tile and
+// an S tile. Warp roles (E = TT/8 epilogue warps):
+//   warps 0..E-1   epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane
+//                  quarter) and token columns 32(w/4)..+31 of P and S, accumulates in f32
+//   warps E..E+3   producer: load packed 4-bit codes (16 B per row-block, two stages
+//                  ahead), expand to fp16 in the MMA's K-major core-matrix layout, store
+//                  the row's scale operand (and the affine bias) per block
+//   warp E+4       TMEM allocation + single-thread MMA issue
+//   warp E+5       one thread issuing the bulk copies of the token operand, its scale
+//                  operand and (affine) the per-group bias factor
 // Every wait is bounded (bounded_wait); within the epilogue and the producer one thread
 // polls and the other warps block on a named barrier. On a timeout all roles stop,
 // outstanding copies and MMAs are drained, TMEM is freed and the kernel returns.
@@ -43,47 +43,54 @@ namespace w4a8 {
 namespace tc {
 
 constexpr int BN = 128;                   // weight rows per CTA (MMA M, TMEM lanes)
-constexpr int TT = tcgeo::kTokTile;       // tokens per CTA (MMA N)
 constexpr int S = 2;                      // quant blocks per stage
-constexpr int NS = 4;                     // stages in the ring
-constexpr int NBUF = 2;                   // TMEM block buffers (each P + S)
 constexpr int A_BLK = BN * 64;            // fp16 weight operand bytes per block
-constexpr int B_BLK = tcgeo::kTokBlockBytes;
 constexpr int AS_BLK = BN * 16;           // tf32 scale operand, first K-chunk, weight side
-constexpr int BS_BLK = TT * 16;           // tf32 scale operand, first K-chunk, token side
-constexpr int OFF_B = S * A_BLK;
-constexpr int OFF_AS = OFF_B + S * B_BLK;
-constexpr int OFF_BS = OFF_AS + S * AS_BLK;
-constexpr int OFF_Z = OFF_BS + S * BS_BLK;
-constexpr int STAGE_BYTES = OFF_Z + TT * 4;   // + one group's bias factor (affine)
-constexpr int ZERO_BYTES = 128 * 16;          // second K-chunk of both scale operands
-constexpr int CTRL_BYTES = 256;
-constexpr int SMEM_BYTES = NS * STAGE_BYTES + ZERO_BYTES + CTRL_BYTES + 1024;  // + alignment slack
+constexpr int ZERO_BYTES = 128 * 16;      // second K-chunk of both scale operands
+constexpr int CTRL_BYTES = 512;
 constexpr int TMEM_COLS = 512;
-constexpr int P_COL0 = 0, S_COL0 = NBUF * TT;  // P tiles in columns 0..255, S tiles 256..511
-constexpr int EPI_WARPS = 16;
-constexpr int EPI_COLS = 32;                   // token columns per epilogue warp
-constexpr int PROD_WARP0 = 16;
-constexpr int MMA_WARP = 20;
-constexpr int COPY_WARP = 21;
-constexpr int NUM_THREADS = 22 * 32;
-constexpr uint32_t IDESC_P = idesc_f16_f32(BN, TT);
-// kind::tf32: D f32, A and B tf32 (format 2), K-major, M x N
-constexpr uint32_t IDESC_S = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(TT >> 3) << 17) | (uint32_t(BN >> 4) << 24);
-constexpr uint32_t LBO = 128, SBO = 512;   // fp16 operands: core-matrix strides (K, M/N)
-constexpr uint32_t SBO_S = 128;            // tf32 scale operands: 8-row groups 128 B apart
+constexpr int EPI_COLS = 32;              // token columns per epilogue warp
+constexpr uint32_t LBO = 128, SBO = 512;  // fp16 operands: core-matrix strides (K, M/N)
+constexpr uint32_t SBO_S = 128;           // tf32 scale operands: 8-row groups 128 B apart
 
-static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
-static_assert(SMEM_BYTES <= 232448, "shared memory");
-static_assert(EPI_WARPS * EPI_COLS == 4 * TT, "epilogue covers the tile");
-static_assert(NBUF * 2 * TT == TMEM_COLS, "tmem columns");
+// Geometry for a token tile of TT tokens (32, 64 or 128): TMEM holds NBUF block buffers
+// of a P tile (TT columns) and an S tile (TT columns); TT/8 epilogue warps cover the
+// 128 x TT tile 32 columns each; the shared-memory ring is as deep as fits.
+template <int TT>
+struct Geo {
+    static constexpr int NBUF = TMEM_COLS / (2 * TT);
+    static constexpr int B_BLK = tcgeo::tok_block_bytes(TT);
+    static constexpr int BS_BLK = TT * 16;
+    static constexpr int OFF_B = S * A_BLK;
+    static constexpr int OFF_AS = OFF_B + S * B_BLK;
+    static constexpr int OFF_BS = OFF_AS + S * AS_BLK;
+    static constexpr int OFF_Z = OFF_BS + S * BS_BLK;
+    static constexpr int STAGE_BYTES = OFF_Z + TT * 4;  // + one group's bias factor (affine)
+    static constexpr int NS = (TT == 128) ? 4 : (TT == 64) ? 6 : 7;
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + ZERO_BYTES + CTRL_BYTES + 1024;
+    static constexpr int P_COL0 = 0, S_COL0 = NBUF * TT;
+    static constexpr int EPI_WARPS = TT / 8;
+    static constexpr int PROD_WARP0 = EPI_WARPS;
+    static constexpr int MMA_WARP = EPI_WARPS + 4;
+    static constexpr int COPY_WARP = EPI_WARPS + 5;
+    static constexpr int NUM_THREADS = (EPI_WARPS + 6) * 32;
+    static constexpr uint32_t IDESC_P = idesc_f16_f32(BN, TT);
+    // kind::tf32: D f32, A and B tf32 (format 2), K-major, M x N
+    static constexpr uint32_t IDESC_S =
+        (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(TT >> 3) << 17) | (uint32_t(BN >> 4) << 24);
+    static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(EPI_WARPS * EPI_COLS == 4 * TT, "epilogue covers the tile");
+    static_assert(NBUF * 2 * TT == TMEM_COLS, "tmem columns");
+};
 
+constexpr int MAX_NS = 8, MAX_NBUF = 8;
 struct Ctrl {
-    unsigned long long full_a[NS];    // producer threads (128 arrivals)
-    unsigned long long full_b[NS];    // bulk copies (1 arrival + bytes)
-    unsigned long long empty[NS];     // MMA commit + one arrival per epilogue warp
-    unsigned long long tfull[NBUF];   // MMA commit
-    unsigned long long tempty[NBUF];  // one arrival per epilogue warp
+    unsigned long long full_a[MAX_NS];    // producer threads (128 arrivals)
+    unsigned long long full_b[MAX_NS];    // bulk copies (1 arrival + bytes)
+    unsigned long long empty[MAX_NS];     // MMA commit + one arrival per epilogue warp
+    unsigned long long tfull[MAX_NBUF];   // MMA commit
+    unsigned long long tempty[MAX_NBUF];  // one arrival per epilogue warp
     unsigned long long drain;         // final MMA drain
     uint32_t tmem_base;
     uint32_t abort;
@@ -129,12 +136,18 @@ struct RowStage {
     float s[S], b[S];
 };
 
-template <int FMT>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int FMT, int TT>
+__global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
     gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float4* __restrict__ bs,
                    const float* __restrict__ zb, const uint8_t* __restrict__ wq,
                    const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
                    float* __restrict__ y) {
+    using Gm = Geo<TT>;
+    constexpr int NS = Gm::NS, NBUF = Gm::NBUF, B_BLK = Gm::B_BLK, BS_BLK = Gm::BS_BLK;
+    constexpr int OFF_B = Gm::OFF_B, OFF_AS = Gm::OFF_AS, OFF_BS = Gm::OFF_BS, OFF_Z = Gm::OFF_Z;
+    constexpr int STAGE_BYTES = Gm::STAGE_BYTES, P_COL0 = Gm::P_COL0, S_COL0 = Gm::S_COL0;
+    constexpr int EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0, MMA_WARP = Gm::MMA_WARP;
+    constexpr int COPY_WARP = Gm::COPY_WARP, NUM_THREADS = Gm::NUM_THREADS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* zero = smem + NS * STAGE_BYTES;
@@ -284,13 +297,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     tc_mma_f16(tmem_base + uint32_t(P_COL0 + buf * TT), smem_desc_kmajor(a_addr + h * 256, LBO, SBO),
-                               smem_desc_kmajor(b_addr + h * 256, LBO, SBO), IDESC_P, h);
+                               smem_desc_kmajor(b_addr + h * 256, LBO, SBO), Gm::IDESC_P, h);
                 }
                 const uint32_t as_addr = smem_addr(sp + OFF_AS + k * AS_BLK);
                 const uint32_t bs_addr = smem_addr(sp + OFF_BS + k * BS_BLK);
                 tc_mma_tf32(tmem_base + uint32_t(S_COL0 + buf * TT),
                             smem_desc_kmajor(as_addr, zero_addr - as_addr, SBO_S),
-                            smem_desc_kmajor(bs_addr, zero_addr - bs_addr, SBO_S), IDESC_S, 0);
+                            smem_desc_kmajor(bs_addr, zero_addr - bs_addr, SBO_S), Gm::IDESC_S, 0);
                 tc_commit(bar(&ctrl->tfull[buf]));
                 if (k == S - 1 || i == B - 1) tc_commit(bar(&ctrl->empty[slot]));
             }

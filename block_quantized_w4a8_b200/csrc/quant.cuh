@@ -16,10 +16,10 @@
 
 namespace w4a8 {
 
-// Tensor-core operand geometry shared by the activation kernel and the GEMM.
+// Tensor-core operand geometry shared by the activation kernel and the GEMM: the
+// token tile (tokens per GEMM tile, the MMA's N) is 32, 64 or 128.
 namespace tcgeo {
-constexpr int kTokTile = 128;                 // tokens per GEMM tile (MMA N)
-constexpr int kTokBlockBytes = kTokTile * 64; // one 32-wide block of kTokTile tokens, fp16
+__host__ __device__ constexpr int tok_block_bytes(int tt) { return tt * 64; }  // one 32-wide block, fp16
 }  // namespace tcgeo
 
 // ------------------------------------------------------------------ Q8_0, row-major
@@ -64,8 +64,8 @@ __global__ void __launch_bounds__(256) quant_act_rowmajor_kernel(const void* __r
 // ------------------------------------------------------------------ Q8_0, MMA operand
 // Same quantisation, written as the fp16 B operand of the tcgen05 GEMM.
 //
-// Layout (per token tile t of kTokTile rows and block b): a contiguous chunk of
-// kTokTile x 32 fp16 at chunk index t*B + b. Inside a chunk, token row r and 16-byte
+// Layout (per token tile t of `tt` rows and block b): a contiguous chunk of tt x 32
+// fp16 at chunk index t*B + b. Inside a chunk, token row r and 16-byte
 // segment c (c = 0..3) sit at byte (r/8)*512 + c*128 + (r%8)*16: the K-major,
 // no-swizzle arrangement of 8-row x 16-byte core matrices (K-adjacent core matrices
 // 128 B apart, 8-row groups 512 B apart).
@@ -85,10 +85,10 @@ __global__ void __launch_bounds__(256) quant_act_rowmajor_kernel(const void* __r
 // per token and weight group g, Z = sum over the group's blocks of d*sum(q) (the factor
 // of the bias term).
 template <bool BF16, int FMT>
-__global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restrict__ x, int M, int K, int64_t nblocks,
-                                                           __half* __restrict__ tok, float4* __restrict__ bs,
-                                                           float* __restrict__ zb, int group) {
-    using namespace tcgeo;
+__global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restrict__ x, int M, int K, int tt,
+                                                           int64_t nblocks, __half* __restrict__ tok,
+                                                           float4* __restrict__ bs, float* __restrict__ zb,
+                                                           int group) {
     pdl_launch_dependents();
     const int B = K >> 5;
     const int64_t blk = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
                           ((uint32_t(q[2]) & 0xFFu) << 16) | ((uint32_t(q[3]) & 0xFFu) << 24);
     const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, FMT == 0 ? 4 : 1);
     auto code = [](uint32_t w, int i) { return int(int8_t((w >> (8 * i)) & 0xFFu)); };
-    const int64_t t = m / kTokTile;
-    const int r = int(m - t * kTokTile);
+    const int64_t t = m / tt;
+    const int r = int(m - t * tt);
     const int64_t chunk = t * B + b;
     const bool writer = (FMT == 0) ? (sub < 4) : ((sub & 1) == 0);
     if (valid && writer) {
@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
             const uint32_t hi = __half_as_ushort(__int2half_rn(e[2 * i + 1]));
             h[i] = lo | (hi << 16);
         }
-        char* dst = reinterpret_cast<char*>(tok) + chunk * kTokBlockBytes + (r >> 3) * 512 + c * 128 + (r & 7) * 16;
+        char* dst = reinterpret_cast<char*>(tok) + chunk * tcgeo::tok_block_bytes(tt) + (r >> 3) * 512 + c * 128 +
+                    (r & 7) * 16;
         *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     if (valid && sub == 0) {
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         const float r1 = __fsub_rn(d16, a);  // exact: the low 13 significand bits of d16
         const float b2 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
         const float c2 = __fsub_rn(r1, b2);  // exact, at most 2 significant bits
-        bs[chunk * kTokTile + r] = make_float4(a, b2, c2, 0.0f);
+        bs[chunk * tt + r] = make_float4(a, b2, c2, 0.0f);
     }
     if (FMT == 1) {
         // Blocks of one weight group are adjacent 8-lane groups of this warp (the warp's
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         const int nbg = group >> 5;
         if (valid && sub == 0 && (b % nbg) == 0) {
             const int G = K / group;
-            zb[(t * G + b / nbg) * kTokTile + r] = z;
+            zb[(t * G + b / nbg) * tt + r] = z;
         }
     }
 }

@@ -52,18 +52,24 @@ GemvWs gemv_ws(void* ws, int M, int K) {
     return w;
 }
 
+// Token tile of the tensor-core GEMM for M rows of x: small M gets a small tile (less
+// padding, more TMEM block buffers).
+inline int tc_token_tile(int M) { return M <= 32 ? 32 : (M <= 64 ? 64 : 128); }
+
 struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
     __half* tok;
     float4* bs;
     float* z;
+    int tt;      // tokens per tile
     int tiles;
     size_t bytes;
 };
 TcWs tc_ws(void* ws, int M, int K, int group) {
     const int64_t B = K / 32;
     TcWs w{};
-    w.tiles = int(cdiv(M, tcgeo::kTokTile));
-    const int64_t rows = int64_t(w.tiles) * tcgeo::kTokTile;
+    w.tt = tc_token_tile(M);
+    w.tiles = int(cdiv(M, w.tt));
+    const int64_t rows = int64_t(w.tiles) * w.tt;
     size_t off = 0;
     char* base = static_cast<char*>(ws);
     w.tok = reinterpret_cast<__half*>(base + off); off = align256(off + size_t(rows) * B * 64);
@@ -102,18 +108,18 @@ w4a8_status run_quant_rowmajor(const void* x, w4a8_dtype dt, int M, int K, int8_
 }
 
 w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, const TcWs& w, cudaStream_t stream) {
-    const int64_t nblocks = int64_t(w.tiles) * tcgeo::kTokTile * (K / 32);
+    const int64_t nblocks = int64_t(w.tiles) * w.tt * (K / 32);
     const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
     if (group == 0) {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, 0);
+            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, 0);
         else
-            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, 0);
+            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, 0);
     } else {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, group);
+            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, group);
         else
-            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, nblocks, w.tok, w.bs, w.z, group);
+            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, group);
     }
     return launch_status();
 }
@@ -218,23 +224,35 @@ w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_d
     return cuda_status(e);
 }
 
-template <int FMT>
-w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                        const uint16_t* wb, float* y, cudaStream_t stream) {
+template <int FMT, int TT>
+w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
+                           const uint16_t* wb, float* y, cudaStream_t stream) {
+    using Gm = tc::Geo<TT>;
     static bool configured[64] = {false};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return W4A8_ERR_CUDA;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return cuda_status(ed);
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT, TT>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM_BYTES);
         if (ea != cudaSuccess) return cuda_status(ea);
         configured[dev] = true;
     }
     const dim3 grid(unsigned(cdiv(N, tc::BN)), unsigned(w.tiles));
-    cudaError_t e = launch_pdl(tc::gemm_tc_kernel<FMT>, grid, dim3(tc::NUM_THREADS), size_t(tc::SMEM_BYTES), stream,
-                               M, N, K, group, (const __half*)w.tok, (const float4*)w.bs, (const float*)w.z, wq, ws,
-                               wb, y);
+    cudaError_t e = launch_pdl(tc::gemm_tc_kernel<FMT, TT>, grid, dim3(Gm::NUM_THREADS), size_t(Gm::SMEM_BYTES),
+                               stream, M, N, K, group, (const __half*)w.tok, (const float4*)w.bs, (const float*)w.z,
+                               wq, ws, wb, y);
     return cuda_status(e);
+}
+
+template <int FMT>
+w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
+                        const uint16_t* wb, float* y, cudaStream_t stream) {
+    switch (w.tt) {
+        case 32: return launch_gemm_tc<FMT, 32>(M, N, K, group, w, wq, ws, wb, y, stream);
+        case 64: return launch_gemm_tc<FMT, 64>(M, N, K, group, w, wq, ws, wb, y, stream);
+        default: return launch_gemm_tc<FMT, 128>(M, N, K, group, w, wq, ws, wb, y, stream);
+    }
 }
 
 w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
