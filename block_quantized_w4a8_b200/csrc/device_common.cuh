@@ -57,6 +57,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Probe without a suspend hint: on a completed phase it returns in a fraction of the
+// time of the hinted form, so every wait checks this way first.
+__device__ __forceinline__ bool mbar_try_wait_nohint(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 
 // Wait until the phase with parity `parity` of barrier `bar` has completed. Gives up
 // when `*abort` is raised by another thread or after kWaitLimitNs; in the latter case
@@ -77,8 +90,34 @@ __device__ __noinline__ bool bounded_wait_slow(uint32_t bar, uint32_t parity, vo
     }
 }
 __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_nohint(bar, parity)) return true;
     return bounded_wait_slow(bar, parity, abort);
+}
+
+// Warp-wide wait: every lane probes the barrier and a vote makes the outcome uniform
+// (phase completion is monotonic, so a lane that saw it keeps seeing it), so the warp
+// never diverges. Same limits as bounded_wait. All 32 lanes must call it.
+__device__ __noinline__ bool bounded_wait_warp_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+    const unsigned long long t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        if ((it & 15u) == 0u) {
+            uint32_t stop = *abort;
+            if (!stop && global_timer_ns() - t0 > kWaitLimitNs) stop = 2u;
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop) {
+                if (stop == 2u && (threadIdx.x & 31u) == 0u) {
+                    atomicOr(&g_device_status, kDevErrTimeout);
+                    *abort = 1u;
+                }
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool bounded_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+    if (__all_sync(0xffffffffu, mbar_try_wait_nohint(bar, parity))) return true;
+    return bounded_wait_warp_slow(bar, parity, abort);
 }
 
 // Named hardware barrier over `nthreads` threads (whole warps); waiting warps issue
@@ -111,13 +150,25 @@ __device__ __forceinline__ bool bounded_wait_group(uint32_t bar, uint32_t parity
     return named_barrier_and(barrier_id, nthreads, ok);
 }
 
-// Warp-uniform variant: lane 0 waits, the outcome is broadcast so that every lane of
-// the warp takes the same branch afterwards (needed before .sync.aligned instructions).
-__device__ __forceinline__ bool bounded_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
-    uint32_t ok = 0;
-    if ((threadIdx.x & 31u) == 0u) ok = bounded_wait(bar, parity, abort) ? 1u : 0u;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    return ok != 0;
+// Warp-wide wait used only to drain asynchronous copies before a CTA exits: waits up to
+// `limit_ns` and reports nothing (the caller has already recorded why it stopped).
+__device__ __noinline__ void drain_wait_warp(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+    const unsigned long long t0 = global_timer_ns();
+    while (!__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) {
+        uint32_t stop = (global_timer_ns() - t0 > limit_ns) ? 1u : 0u;
+        if (__shfl_sync(0xffffffffu, stop, 0)) return;
+    }
+}
+
+// True in exactly one lane of the (converged) warp: the lowest active lane.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 // ------------------------------------------------------------------ bulk async copy

@@ -1,163 +1,211 @@
-// Large-M path: tcgen05 tensor-core GEMM with per-block rescaling.
+// Tensor-core path: tcgen05 GEMM with the weight block scale folded into the weight
+// operand and the activation block scale applied per block in the epilogue.
 //
-// y[m][n] = sum_b  s_w[n][b] * d_x[m][b] * D[m][n][b],  D = exact 32-wide block dot.
-// The block dot must stay exact and each block must be rescaled separately (tract PR
-// #2432, "The kernel": Q4_0's per-32-block scales force a per-block rescale; there it
-// is one vector multiply per block over accumulator lanes that each hold one output).
-// Here every block gets its own tensor-memory accumulator: TMEM lane = weight row,
-// TMEM column = token, so each epilogue thread owns one output row and needs no
-// cross-lane reduction.
+// y[m][n] = sum_b  d_x[m][b] * P[m][n][b],   P = d_w[n][b] * D[m][n][b],
+// D = the exact 32-wide integer block dot. The block dot must stay exact and each block
+// must be rescaled separately (tract PR #2432, "The kernel": Q4_0's per-32-block scales
+// force a per-block rescale, one multiply per block over accumulator lanes that each own
+// one output). Here the tensor core produces P directly, exactly up to the f32 rounding
+// of its accumulator, and the epilogue does one f32 FMA per (output, block):
 //
-// Per block the tensor core produces two 128 x 128 tiles in TMEM:
-//   P = 16 * D      two kind::f16 MMAs on fp16 operands that hold small integers (weight
-//                   codes q-8 or 16(q-8), affine q or 16q; activation codes 16q_x or q_x,
-//                   see quant_act_tc_kernel): every product and block sum is an exact
-//                   integer below 2^20, so P is exact.
-//   S = s_w (x) d_x/16   one kind::tf32 MMA with K = 8: the weight side holds
-//                   (s_w, s_w, s_w, .) per row, the activation side (a, b, c, 0) with
-//                   a + b + c = d_x/16 exactly, the second K-chunk of both points at a
-//                   zero region. So S = s_w * d_x / 16 up to the accumulator's rounding.
-// The epilogue then does acc += P * S per element: one FMA, no per-column scale traffic
-// through shared memory (the outer product of the scales comes from the tensor core).
+// Weight operand (fp16, one K-major core-matrix tile per block):
+//   Q4_0:   d_w = d_hi + d_lo, d_hi = d_w with the three lowest significand bits cleared
+//           (8 significant bits), d_lo = the rest (3 bits). The slots hold d_hi*(q-8) and
+//           d_lo*(q-8): an 8-bit times a 3-bit magnitude (|q-8| <= 8) fits the 11-bit fp16
+//           significand, so both parts are exact; they are formed by one fused multiply-add
+//           whose addend 24*d_hi must fit fp16, so |d_hi| <= 2720 (larger, infinite or nan
+//           scales set W4A8_ERR_RANGE in the device status word). Four kind::f16
+//           MMAs (hi and lo parts, two K = 16 halves each) accumulate d_w*D in one TMEM
+//           tile: the hi half-sums are exact, the lo parts add at most two f32 roundings.
+//   affine: s*(q-8) with s the bf16 group scale (8 significant bits): exact in fp16 for
+//           2^-17 <= |s| <= 2720 (or s = 0; others set W4A8_ERR_RANGE). Two MMAs per block
+//           give s*sum (q-8)*q_x; the epilogue adds (b + 8s)*Z per group, where
+//           Z[m][g] = sum over the group's blocks of d_x*sum(q_x) (MLX PR #4802, mode
+//           "affine": scale and bias applied on the original codes, rewritten with the
+//           codes centred at 8 so that the scaled codes stay exact in fp16).
+// Token operand: the Q8_0 codes as fp16 (exact), written by quant_act_tc_kernel in the
+// same K permutation as the weight expansion.
 //
-// CTA tile: 128 weight rows x TT tokens (TT = 32, 64 or 128); one pipeline stage = 2
-// quant blocks (K = 64), 4-7 stages; 512/(2 TT) block buffers in TMEM, each a P tile and
-// an S tile. Warp roles (E = TT/8 epilogue warps):
-//   warps 0..E-1   epilogue: warp w reads TMEM lanes 32(w%4).. (its hardware lane
-//                  quarter) and token columns 32(w/4)..+31 of P and S, accumulates in f32
-//   warps E..E+3   producer: load packed 4-bit codes (16 B per row-block, two stages
-//                  ahead), expand to fp16 in the MMA's K-major core-matrix layout, store
-//                  the row's scale operand (and the affine bias) per block
-//   warp E+4       TMEM allocation + single-thread MMA issue
-//   warp E+5       one thread issuing the bulk copies of the token operand, its scale
-//                  operand and (affine) the per-group bias factor
-// Every wait is bounded (bounded_wait); within the epilogue and the producer one thread
-// polls and the other warps block on a named barrier. On a timeout all roles stop,
-// outstanding copies and MMAs are drained, TMEM is freed and the kernel returns.
+// Two orientations of the same MMA (K-major operands, so A and B just swap roles):
+//   TOKL = true  (large M): TMEM lane = token (128 per tile), TMEM column = weight row
+//                (MN per tile). d_x is a per-thread scalar: the epilogue is acc += d_x * P.
+//   TOKL = false (small M): TMEM lane = weight row (128 per tile), TMEM column = token
+//                (MN = 16..128 per tile, so few MMA rows are padding); d_x comes from a
+//                broadcast shared-memory load per 4 tokens.
+// Warp roles: EPI_WARPS epilogue warps (warp w reads TMEM lane quarter w%4, column chunk
+// w/4 of CW columns, accumulates in f32 registers); PROD_WARPS producer warps (one weight
+// row per thread: 16-B code loads two stages ahead, nibble -> scaled fp16 expansion,
+// store in the core-matrix layout); one MMA-issue warp (also allocates TMEM); one
+// bulk-copy warp (token operand, d_x and Z via plain cp.async.bulk, no multicast). The
+// MMA and copy warps run their loops warp-uniformly with one elected lane issuing. Every
+// wait is bounded and taken by each warp on its own (all lanes probe, a vote keeps the
+// warp converged), so no role is held in lockstep by its slowest warp; the epilogue
+// releases a pipeline stage as soon as it has read the stage's scales. On a timeout all
+// roles stop, outstanding copies and MMAs are drained, TMEM is freed and the kernel
+// returns.
 #pragma once
 
 #include "device_common.cuh"
 #include "quant.cuh"
 
 namespace w4a8 {
+
+// Bit set in the device status word when a weight scale is outside the range in which
+// the tensor-core path's fp16 weight operand is exact.
+constexpr unsigned kDevErrRange = 2u;
+
 namespace tc {
 
-constexpr int BN = 128;                   // weight rows per CTA (MMA M, TMEM lanes)
-constexpr int S = 2;                      // quant blocks per stage
-constexpr int A_BLK = BN * 64;            // fp16 weight operand bytes per block
-constexpr int AS_BLK = BN * 16;           // tf32 scale operand, first K-chunk, weight side
-constexpr int ZERO_BYTES = 128 * 16;      // second K-chunk of both scale operands
-constexpr int CTRL_BYTES = 512;
-constexpr int TMEM_COLS = 512;
-constexpr int EPI_COLS = 32;              // token columns per epilogue warp
-constexpr uint32_t LBO = 128, SBO = 512;  // fp16 operands: core-matrix strides (K, M/N)
-constexpr uint32_t SBO_S = 128;           // tf32 scale operands: 8-row groups 128 B apart
+constexpr int CTRL_BYTES = 1024;
+constexpr uint32_t LBO = 128, SBO = 512;  // core-matrix strides: along K, along rows
+constexpr int SMEM_LIMIT = 232448;
 
-// Geometry for a token tile of TT tokens (32, 64 or 128): TMEM holds NBUF block buffers
-// of a P tile (TT columns) and an S tile (TT columns); TT/8 epilogue warps cover the
-// 128 x TT tile 32 columns each; the shared-memory ring is as deep as fits.
-template <int TT>
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
+
+// Geometry of one instantiation. FMT: 0 = Q4_0, 1 = affine. MN: the MMA's N (weight
+// rows per tile when TOKL, tokens per tile otherwise); the MMA's M is always 128.
+template <int FMT, bool TOKL, int MN>
 struct Geo {
-    static constexpr int NBUF = TMEM_COLS / (2 * TT);
-    static constexpr int B_BLK = tcgeo::tok_block_bytes(TT);
-    static constexpr int BS_BLK = TT * 16;
-    static constexpr int OFF_B = S * A_BLK;
-    static constexpr int OFF_AS = OFF_B + S * B_BLK;
-    static constexpr int OFF_BS = OFF_AS + S * AS_BLK;
-    static constexpr int OFF_Z = OFF_BS + S * BS_BLK;
-    static constexpr int STAGE_BYTES = OFF_Z + TT * 4;  // + one group's bias factor (affine)
-    static constexpr int NS = (TT == 128) ? 4 : (TT == 64) ? 6 : 7;
-    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + ZERO_BYTES + CTRL_BYTES + 1024;
-    static constexpr int P_COL0 = 0, S_COL0 = NBUF * TT;
-    static constexpr int EPI_WARPS = TT / 8;
+    static constexpr int TT = TOKL ? 128 : MN;   // tokens per tile
+    static constexpr int NW = TOKL ? MN : 128;   // weight rows per tile
+    static constexpr int WP = (FMT == 0) ? 2 : 1;  // weight operand parts (hi, lo)
+    static constexpr int W_PART = NW * 64;       // bytes of one part of one block
+    static constexpr int W_BLK = W_PART * WP;
+    static constexpr int T_BLK = TT * 64;
+    static constexpr int DX_BLK = TT * 4;
+    static constexpr int PER_BLK = W_BLK + T_BLK;
+    // Quant blocks per pipeline stage. One tcgen05.commit covers a stage (a commit costs
+    // the tensor pipe about as much as 1.5 MMAs of 128x128x16), so small tiles take more
+    // blocks per stage.
+    static constexpr int S = (!TOKL && MN <= 32) ? 4 : (PER_BLK <= 12288 ? 4 : (PER_BLK <= 24576 ? 2 : 1));
+    static constexpr int OFF_T = S * W_BLK;
+    static constexpr int OFF_DX = OFF_T + S * T_BLK;
+    static constexpr int OFF_C = align_up(OFF_DX + S * DX_BLK, 128);           // affine: b + 8s per row
+    static constexpr int OFF_Z = OFF_C + (FMT == 1 ? S * NW * 4 : 0);          // affine: Z per token
+    static constexpr int STAGE_BYTES = align_up(OFF_Z + (FMT == 1 ? S * TT * 4 : 0), 1024);
+    static constexpr int NS = cmin(8, (SMEM_LIMIT - CTRL_BYTES - 1024) / STAGE_BYTES);
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;
+    static constexpr int NBUF = cmin(16, 512 / MN);  // TMEM accumulator tiles (one per block)
+    static constexpr int NG = NBUF / S;              // TMEM groups: stage st uses group st % NG
+    static constexpr int TMEM_COLS = NBUF * MN;
+    static constexpr int CW = cmin(MN, 64);  // columns per epilogue warp
+    static constexpr int EPI_WARPS = 4 * MN / CW;
+    static constexpr int PROD_WARPS = NW / 32;
     static constexpr int PROD_WARP0 = EPI_WARPS;
-    static constexpr int MMA_WARP = EPI_WARPS + 4;
-    static constexpr int COPY_WARP = EPI_WARPS + 5;
-    static constexpr int NUM_THREADS = (EPI_WARPS + 6) * 32;
-    static constexpr uint32_t IDESC_P = idesc_f16_f32(BN, TT);
-    // kind::tf32: D f32, A and B tf32 (format 2), K-major, M x N
-    static constexpr uint32_t IDESC_S =
-        (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(TT >> 3) << 17) | (uint32_t(BN >> 4) << 24);
-    static_assert(STAGE_BYTES % 16 == 0, "stage alignment");
-    static_assert(SMEM_BYTES <= 232448, "shared memory");
-    static_assert(EPI_WARPS * EPI_COLS == 4 * TT, "epilogue covers the tile");
-    static_assert(NBUF * 2 * TT == TMEM_COLS, "tmem columns");
+    static constexpr int MMA_WARP = PROD_WARP0 + PROD_WARPS;
+    static constexpr int COPY_WARP = MMA_WARP + 1;
+    static constexpr int NUM_THREADS = (COPY_WARP + 1) * 32;
+    // Registers per thread at this size: each SM sub-partition holds ceil(warps/4) warps
+    // of the CTA in 16384 registers. Below 160 the epilogue reads its columns in halves
+    // so that the accumulators and one half of the tile fit.
+    static constexpr int REG_CAP = 16384 / (((NUM_THREADS / 32) + 3) / 4 * 32) / 8 * 8;
+    static constexpr int LD_COLS = (REG_CAP < 160 && CW == 64) ? 32 : CW;
+    static constexpr uint32_t IDESC = idesc_f16_f32(128, MN);
+    static_assert(MN == 16 || MN == 32 || MN == 64 || MN == 128, "MMA N");
+    static_assert(!TOKL || MN >= 64, "token-lane tiles cover 64 or 128 weight rows");
+    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation");
+    static_assert(NS >= 2, "pipeline depth");
+    static_assert(NG >= 2 && NBUF % S == 0, "TMEM groups");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
+    static_assert(OFF_T % 128 == 0 && OFF_DX % 16 == 0 && OFF_Z % 16 == 0, "operand alignment");
 };
 
-constexpr int MAX_NS = 8, MAX_NBUF = 8;
+constexpr int MAX_NS = 8, MAX_NG = 8;
 struct Ctrl {
-    unsigned long long full_a[MAX_NS];    // producer threads (128 arrivals)
-    unsigned long long full_b[MAX_NS];    // bulk copies (1 arrival + bytes)
-    unsigned long long empty[MAX_NS];     // MMA commit + one arrival per epilogue warp
-    unsigned long long tfull[MAX_NBUF];   // MMA commit
-    unsigned long long tempty[MAX_NBUF];  // one arrival per epilogue warp
-    unsigned long long drain;         // final MMA drain
+    unsigned long long full[MAX_NS];    // producer threads (one arrival per weight row) + bulk copies (1 + bytes)
+    unsigned long long empty[MAX_NS];   // one arrival per epilogue warp (after the stage's MMAs completed
+                                        // and the warp read the stage's scales)
+    unsigned long long tfull[MAX_NG];   // MMA commit, once per stage
+    unsigned long long tempty[MAX_NG];  // one arrival per epilogue warp
+    unsigned long long drain;             // final MMA drain
     uint32_t tmem_base;
     uint32_t abort;
 };
 static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
 
-// Expand one 32-bit word of packed codes into four fp16x2 words (8 K-slots).
-// Q4_0 word = bytes 4i..4i+3 of a block: low nibbles elements 4i..4i+3, high nibbles
-// 16+4i..; affine word = elements 8t..8t+7 at bits 4e. Output slot order (both
-// operands use it): low nibbles of bytes 0,2 | of bytes 1,3 | high nibbles of bytes
-// 0,2 | of bytes 1,3. Low-nibble slots hold the code, high-nibble slots 16*code; the
-// Q4_0 codes are shifted by -8 (-128 for the x16 slots). 0x6400 is fp16 1024, so
-// (0x6400 | v) is 1024 + v exactly and one packed subtract removes the offset.
-template <int FMT>
-__device__ __forceinline__ uint4 expand_word(uint32_t w) {
-    const uint32_t ea = (w & 0x000F000Fu) | 0x64006400u;
-    const uint32_t eb = ((w >> 8) & 0x000F000Fu) | 0x64006400u;
-    const uint32_t ec = (w & 0x00F000F0u) | 0x64006400u;
-    const uint32_t ed = ((w >> 8) & 0x00F000F0u) | 0x64006400u;
-    const uint32_t off_lo = (FMT == 0) ? 0x64086408u : 0x64006400u;  // 1032 : 1024
-    const uint32_t off_hi = (FMT == 0) ? 0x64806480u : 0x64006400u;  // 1152 : 1024
-    auto sub = [](uint32_t a, uint32_t b) {
-        __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
-        return *reinterpret_cast<uint32_t*>(&r);
-    };
-    return make_uint4(sub(ea, off_lo), sub(eb, off_lo), sub(ec, off_hi), sub(ed, off_hi));
+
+// One 32-bit word of packed codes as four fp16x2 words holding 8 + q/2: each nibble is
+// moved to mantissa bits 6..9 under the exponent of 8.0 (0x4800). Slot order (both
+// operands use it): Q4_0 word i = bytes 4i..4i+3 of a block gives elements 4i, 4i+2 |
+// 4i+1, 4i+3 | 16+4i, 16+4i+2 | 16+4i+1, 16+4i+3; affine word t (element 8t+e at bits
+// 4e) gives 8t, 8t+4 | 8t+2, 8t+6 | 8t+1, 8t+5 | 8t+3, 8t+7.
+__device__ __forceinline__ void codes_raw(uint32_t w, uint32_t (&r)[4]) {
+    constexpr uint32_t M = 0x03C003C0u, E = 0x48004800u;
+    r[0] = ((w << 6) & M) | E;
+    r[1] = ((w >> 2) & M) | E;
+    r[2] = ((w << 2) & M) | E;
+    r[3] = ((w >> 6) & M) | E;
+}
+// (8 + q/2) * (2d) - 24d = (q - 8) * d in one fused multiply-add per pair. With d of at
+// most 8 significant bits (d_hi, d_lo, or a bf16 scale) the addend 24d and the result
+// (q - 8)*d are representable in fp16, so the single rounding leaves them exact.
+__device__ __forceinline__ uint32_t scaled_codes(uint32_t raw, uint32_t d2x2, uint32_t m24d2) {
+    __half2 r = __hfma2(*reinterpret_cast<const __half2*>(&raw), *reinterpret_cast<const __half2*>(&d2x2),
+                        *reinterpret_cast<const __half2*>(&m24d2));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t pair_of(__half h) { return uint32_t(__half_as_ushort(h)) * 0x10001u; }
+
+// Global loads written as volatile asm so that the compiler issues them where they stand
+// in the program (stages ahead of their use) instead of sinking them to the first use.
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
 }
 
-// tf32 MMA: D[tmem] (+)= A[smem] * B[smem]^T, both K-major, f32 accumulator.
-__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Codes and scales of one stage of one weight row, held in registers until stored.
+// Codes and scale bits of one stage of one weight row, held in registers until stored.
+template <int S>
 struct RowStage {
     uint4 w[S];
-    float s[S], b[S];
+    uint16_t s[S], b[S];
 };
 
-template <int FMT, int TT>
-__global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
-    gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float4* __restrict__ bs,
+// Loads CW TMEM columns of this warp's lane quarter into registers (and waits for them).
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[64]) {
+    tmem_ld_32x32_x64(taddr, r);
+    tmem_wait_ld64(r);
+}
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[32]) {
+    tmem_ld_32x32(taddr, r);
+    tmem_wait_ld(r);
+}
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[16]) {
+    tmem_ld_32x32_x16(taddr, r);
+    tmem_wait_ld16(r);
+}
+
+template <int FMT, bool TOKL, int MN>
+__global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
+    gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dxs,
                    const float* __restrict__ zb, const uint8_t* __restrict__ wq,
                    const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
                    float* __restrict__ y) {
-    using Gm = Geo<TT>;
-    constexpr int NS = Gm::NS, NBUF = Gm::NBUF, B_BLK = Gm::B_BLK, BS_BLK = Gm::BS_BLK;
-    constexpr int OFF_B = Gm::OFF_B, OFF_AS = Gm::OFF_AS, OFF_BS = Gm::OFF_BS, OFF_Z = Gm::OFF_Z;
-    constexpr int STAGE_BYTES = Gm::STAGE_BYTES, P_COL0 = Gm::P_COL0, S_COL0 = Gm::S_COL0;
-    constexpr int EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0, MMA_WARP = Gm::MMA_WARP;
-    constexpr int COPY_WARP = Gm::COPY_WARP, NUM_THREADS = Gm::NUM_THREADS;
+    using Gm = Geo<FMT, TOKL, MN>;
+    constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NW = Gm::NW, CW = Gm::CW;
+    constexpr int W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK, DX_BLK = Gm::DX_BLK;
+    constexpr int OFF_T = Gm::OFF_T, OFF_DX = Gm::OFF_DX, OFF_C = Gm::OFF_C, OFF_Z = Gm::OFF_Z;
+    constexpr int STAGE_BYTES = Gm::STAGE_BYTES, EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0;
+    constexpr int LD_COLS = Gm::LD_COLS;
+    constexpr int PROD_THREADS = Gm::PROD_WARPS * 32;
+    constexpr int MMA_WARP = Gm::MMA_WARP, COPY_WARP = Gm::COPY_WARP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* zero = smem + NS * STAGE_BYTES;
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(zero + ZERO_BYTES);
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + NS * STAGE_BYTES);
     volatile uint32_t* abort = &ctrl->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = K >> 5;
     const int nstages = (B + S - 1) / S;
-    const int n0 = blockIdx.x * BN;
+    const int n0 = blockIdx.x * NW;
     const int t = blockIdx.y;
     const int bpg = (FMT == 1) ? (group >> 5) : 1;  // blocks per affine group
     const int G = (FMT == 1) ? K / group : 0;
@@ -165,15 +213,12 @@ __global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
     auto bar = [](unsigned long long* p) { return smem_addr(p); };
 
-    for (int i = threadIdx.x; i < ZERO_BYTES / 16; i += NUM_THREADS)
-        reinterpret_cast<uint4*>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(bar(&ctrl->full_a[s]), 128);
-            mbar_init(bar(&ctrl->full_b[s]), 1);
-            mbar_init(bar(&ctrl->empty[s]), 1 + EPI_WARPS);
+            mbar_init(bar(&ctrl->full[s]), PROD_THREADS + 1);
+            mbar_init(bar(&ctrl->empty[s]), EPI_WARPS);
         }
-        for (int j = 0; j < NBUF; ++j) {
+        for (int j = 0; j < NG; ++j) {
             mbar_init(bar(&ctrl->tfull[j]), 1);
             mbar_init(bar(&ctrl->tempty[j]), EPI_WARPS);
         }
@@ -182,10 +227,9 @@ __global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
         mbar_init_fence();
     }
     if (warp == MMA_WARP) {
-        tmem_alloc(smem_addr(&ctrl->tmem_base), TMEM_COLS);
+        tmem_alloc(smem_addr(&ctrl->tmem_base), Gm::TMEM_COLS);
         tmem_relinquish();
     }
-    fence_proxy_async_smem();  // the zero region is read by the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -194,50 +238,87 @@ __global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
     // before reading its output.
     pdl_launch_dependents();
 
-    if (warp >= PROD_WARP0 && warp < PROD_WARP0 + 4) {
+    if (warp >= PROD_WARP0 && warp < MMA_WARP) {
         // ------------------------------------------------------------ producer
-        const int p = threadIdx.x - PROD_WARP0 * 32;
+        const int p = threadIdx.x - PROD_WARP0 * 32;  // weight row within the tile
         const int n = n0 + p;
         const bool row_ok = n < N;
         const uint4* wrow = reinterpret_cast<const uint4*>(wq + int64_t(row_ok ? n : 0) * (K >> 1));
-        auto load = [&](int st, RowStage& rs) {
+        bool range_bad = false;
+        auto load = [&](int st, RowStage<S>& rs) {
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 const int b = st * S + k;
-                rs.w[k] = make_uint4(0u, 0u, 0u, 0u);
-                rs.s[k] = 0.0f;
-                rs.b[k] = 0.0f;
+                rs.w[k] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);  // codes 8: zero
+                rs.s[k] = 0;
+                rs.b[k] = 0;
                 if (row_ok && b < B) {
-                    rs.w[k] = __ldg(wrow + b);
+                    rs.w[k] = ld_nc_v4(wrow + b);
                     if (FMT == 0) {
-                        rs.s[k] = __half2float(__ushort_as_half(wscale[int64_t(n) * B + b]));
+                        rs.s[k] = ld_nc_u16(wscale + int64_t(n) * B + b);
                     } else {
-                        rs.s[k] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + b / bpg]));
-                        rs.b[k] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + b / bpg]));
+                        rs.s[k] = ld_nc_u16(wscale + int64_t(n) * G + b / bpg);
+                        rs.b[k] = ld_nc_u16(wbias + int64_t(n) * G + b / bpg);
                     }
                 }
             }
         };
         // Store one stage into shared memory; false if the wait gave up.
-        auto produce = [&](int st, const RowStage& rs) {
+        auto produce = [&](int st, const RowStage<S>& rs) {
             const int slot = st % NS;
-            if (!bounded_wait_group(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort, p == 0, 2, 128)) return false;
+            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) return false;
             uint8_t* sp = stage_ptr(slot);
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 const uint32_t w[4] = {rs.w[k].x, rs.w[k].y, rs.w[k].z, rs.w[k].w};
-                uint8_t* arow = sp + k * A_BLK + (p >> 3) * 512 + (p & 7) * 16;
+                uint8_t* dst = sp + k * W_BLK + (p >> 3) * 512 + (p & 7) * 16;
+                if (FMT == 0) {
+                    const uint32_t sb = rs.s[k];
+                    range_bad |= (sb & 0x7FF8u) > 0x6950u;  // d_hi > 2720 (24 d_hi > 65504), inf or nan
+                    const __half dh = __ushort_as_half(uint16_t(sb & 0xFFF8u));
+                    const __half dl = __hsub(__ushort_as_half(uint16_t(sb)), dh);  // exact
+                    const uint32_t h2 = pair_of(__hmul(dh, __float2half(2.0f)));
+                    const uint32_t h24 = pair_of(__hmul(dh, __float2half(-24.0f)));
+                    const uint32_t l2 = pair_of(__hmul(dl, __float2half(2.0f)));
+                    const uint32_t l24 = pair_of(__hmul(dl, __float2half(-24.0f)));
 #pragma unroll
-                for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(arow + c * 128) = expand_word<FMT>(w[c]);
-                // scale operand (s, s, s, bias): the fourth slot meets a zero on the token
-                // side, so it only carries the affine bias to the epilogue
-                reinterpret_cast<float4*>(sp + OFF_AS + k * AS_BLK)[p] = make_float4(rs.s[k], rs.s[k], rs.s[k], rs.b[k]);
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[4];
+                        codes_raw(w[c], r);
+                        *reinterpret_cast<uint4*>(dst + c * 128) =
+                            make_uint4(scaled_codes(r[0], h2, h24), scaled_codes(r[1], h2, h24),
+                                       scaled_codes(r[2], h2, h24), scaled_codes(r[3], h2, h24));
+                        *reinterpret_cast<uint4*>(dst + W_PART + c * 128) =
+                            make_uint4(scaled_codes(r[0], l2, l24), scaled_codes(r[1], l2, l24),
+                                       scaled_codes(r[2], l2, l24), scaled_codes(r[3], l2, l24));
+                    }
+                } else {
+                    const float sf = __bfloat162float(__ushort_as_bfloat16(rs.s[k]));
+                    const float af = fabsf(sf);
+                    range_bad |= !(af <= 2720.0f) || (af != 0.0f && af < 7.62939453125e-06f);  // 2^-17
+                    const __half sh = __float2half_rn(sf);  // exact in range
+                    const uint32_t s2 = pair_of(__hmul(sh, __float2half(2.0f)));
+                    const uint32_t s24 = pair_of(__hmul(sh, __float2half(-24.0f)));
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[4];
+                        codes_raw(w[c], r);
+                        *reinterpret_cast<uint4*>(dst + c * 128) =
+                            make_uint4(scaled_codes(r[0], s2, s24), scaled_codes(r[1], s2, s24),
+                                       scaled_codes(r[2], s2, s24), scaled_codes(r[3], s2, s24));
+                    }
+                    const int b = st * S + k;
+                    if (((b + 1) % bpg) == 0) {  // last block of a group: its bias factor b + 8s
+                        const float bf = __bfloat162float(__ushort_as_bfloat16(rs.b[k]));
+                        reinterpret_cast<float*>(sp + OFF_C)[k * NW + p] = __fadd_rn(bf, __fmul_rn(8.0f, sf));
+                    }
+                }
             }
             fence_proxy_async_smem();
-            mbar_arrive(bar(&ctrl->full_a[slot]));
+            mbar_arrive(bar(&ctrl->full[slot]));
             return true;
         };
-        RowStage r0, r1, r2;  // stages st, st+1, st+2 in flight
+        RowStage<S> r0, r1, r2;  // stages st, st+1, st+2 in flight
         load(0, r0);
         if (1 < nstages) load(1, r1);
         for (int st = 0; st < nstages; st += 3) {
@@ -250,123 +331,195 @@ __global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
             if (st + 4 < nstages) load(st + 4, r1);
             if (!produce(st + 2, r2)) break;
         }
-    } else if (warp >= MMA_WARP) {
-        if (warp == COPY_WARP && lane == 0) {
-            // -------------------------------------------------------- bulk copies
-            pdl_wait_primary();  // the token operands are written by the preceding kernel
-            int issued = 0;
-            for (int st = 0; st < nstages; ++st) {
-                const int slot = st % NS;
-                if (!bounded_wait(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) break;
-                const int b0 = st * S;
-                const int nb = min(S, B - b0);
-                // affine: the bias factor of the group whose last block is in this stage
-                const bool zlast = (FMT == 1) && (((b0 + nb) % bpg) == 0);
-                const uint32_t bytes_tok = nb * B_BLK, bytes_bs = nb * BS_BLK;
-                const uint32_t bytes_z = zlast ? TT * 4 : 0;
-                const uint32_t fb = bar(&ctrl->full_b[slot]);
+        if (range_bad) atomicOr(&g_device_status, kDevErrRange);
+    } else if (warp == COPY_WARP) {
+        // ------------------------------------------------------------ bulk copies
+        // The whole warp runs the loop (uniform control flow); one elected lane issues.
+        const bool leader = elect_one();
+        pdl_wait_primary();  // the token operands are written by the preceding kernel
+        int issued = 0;
+        for (int st = 0; st < nstages; ++st) {
+            const int slot = st % NS;
+            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) break;
+            const int b0 = st * S;
+            const int nb = min(S, B - b0);
+            if (leader) {
+                int nz = 0;  // affine: group ends in this stage (each brings its Z row)
+                if (FMT == 1)
+                    for (int k = 0; k < nb; ++k) nz += ((b0 + k + 1) % bpg) == 0;
+                const uint32_t fb = bar(&ctrl->full[slot]);
                 uint8_t* sp = stage_ptr(slot);
-                mbar_arrive_expect_tx(fb, bytes_tok + bytes_bs + bytes_z);
-                bulk_g2s(smem_addr(sp + OFF_B), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * B_BLK,
-                         bytes_tok, fb);
-                bulk_g2s(smem_addr(sp + OFF_BS), bs + (int64_t(t) * B + b0) * TT, bytes_bs, fb);
-                if (zlast) bulk_g2s(smem_addr(sp + OFF_Z), zb + (int64_t(t) * G + (b0 + nb - 1) / bpg) * TT, bytes_z, fb);
-                issued = st + 1;
-            }
-            // Let every copy this thread issued land before the CTA can exit (on the
-            // normal path they have, or soon will; after an abort some may not be consumed).
-            uint32_t local_abort = 0;
-            for (int st = max(0, issued - NS); st < issued; ++st)
-                bounded_wait(bar(&ctrl->full_b[st % NS]), (st / NS) & 1, &local_abort);
-        } else if (warp == MMA_WARP && lane == 0) {
-            // -------------------------------------------------------- MMA issue
-            const uint32_t zero_addr = smem_addr(zero);
-            for (int i = 0; i < B; ++i) {
-                const int st = i / S, k = i - st * S, slot = st % NS;
-                const uint32_t par = (st / NS) & 1;
-                if (k == 0) {
-                    if (!bounded_wait(bar(&ctrl->full_a[slot]), par, abort)) break;
-                    if (!bounded_wait(bar(&ctrl->full_b[slot]), par, abort)) break;
-                }
-                const int buf = i % NBUF;
-                if (!bounded_wait(bar(&ctrl->tempty[buf]), ((i / NBUF) & 1) ^ 1, abort)) break;
-                tc_fence_after();
-                uint8_t* sp = stage_ptr(slot);
-                const uint32_t a_addr = smem_addr(sp + k * A_BLK);
-                const uint32_t b_addr = smem_addr(sp + OFF_B + k * B_BLK);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    tc_mma_f16(tmem_base + uint32_t(P_COL0 + buf * TT), smem_desc_kmajor(a_addr + h * 256, LBO, SBO),
-                               smem_desc_kmajor(b_addr + h * 256, LBO, SBO), Gm::IDESC_P, h);
-                }
-                const uint32_t as_addr = smem_addr(sp + OFF_AS + k * AS_BLK);
-                const uint32_t bs_addr = smem_addr(sp + OFF_BS + k * BS_BLK);
-                tc_mma_tf32(tmem_base + uint32_t(S_COL0 + buf * TT),
-                            smem_desc_kmajor(as_addr, zero_addr - as_addr, SBO_S),
-                            smem_desc_kmajor(bs_addr, zero_addr - bs_addr, SBO_S), Gm::IDESC_S, 0);
-                tc_commit(bar(&ctrl->tfull[buf]));
-                if (k == S - 1 || i == B - 1) tc_commit(bar(&ctrl->empty[slot]));
-            }
-            // Wait until every MMA (and the barrier arrivals their commits trigger) is done
-            // before TMEM and shared memory are released.
-            uint32_t local_abort = 0;
-            tc_commit(bar(&ctrl->drain));
-            bounded_wait(bar(&ctrl->drain), 0, &local_abort);
-        }
-    } else {
-        // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;                    // lane quarter: weight rows 32q..32q+31
-        const int c0 = (warp >> 2) * EPI_COLS;     // token columns c0..c0+31
-        const int p = q * 32 + lane;               // this thread's weight row within the tile
-        unsigned long long acc[EPI_COLS / 2];      // f32 pairs
-#pragma unroll
-        for (int j = 0; j < EPI_COLS / 2; ++j) acc[j] = 0ull;
-        const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
-        for (int i = 0; i < B; ++i) {
-            const int st = i / S, k = i - st * S, slot = st % NS;
-            const int buf = i % NBUF;
-            if (!bounded_wait_group(bar(&ctrl->tfull[buf]), (i / NBUF) & 1, abort, threadIdx.x == 0, 1,
-                                    EPI_WARPS * 32))
-                break;
-            tc_fence_after();
-#pragma unroll
-            for (int h = 0; h < EPI_COLS / 16; ++h) {
-                uint32_t pr[16], sr[16];
-                tmem_ld_32x32_x16(lane_base + uint32_t(P_COL0 + buf * TT + c0 + 16 * h), pr);
-                tmem_ld_32x32_x16(lane_base + uint32_t(S_COL0 + buf * TT + c0 + 16 * h), sr);
-                tmem_wait_ld16x2(pr, sr);
-                if (h == EPI_COLS / 16 - 1) {  // TMEM buffer free: every value is in registers
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(&ctrl->tempty[buf]));
-                }
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) fma2_pp(acc[8 * h + j / 2], pr[j], pr[j + 1], sr[j], sr[j + 1]);
-            }
-            if (FMT == 1 && ((i + 1) % bpg) == 0) {  // last block of a group: add bias * Z
-                const uint8_t* sp = stage_ptr(slot);
-                const float bsc = reinterpret_cast<const float4*>(sp + OFF_AS + k * AS_BLK)[p].w;
-                const unsigned long long b2 = pack2(bsc, bsc);
-                const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + c0;
-#pragma unroll
-                for (int j = 0; j < EPI_COLS; j += 4) {
-                    const float4 zv = *reinterpret_cast<const float4*>(zs + j);
-                    fma2_bias(acc[j / 2], zv.x, zv.y, b2);
-                    fma2_bias(acc[j / 2 + 1], zv.z, zv.w, b2);
+                mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK) + nz * TT * 4));
+                bulk_g2s(smem_addr(sp + OFF_T), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK,
+                         uint32_t(nb * T_BLK), fb);
+                bulk_g2s(smem_addr(sp + OFF_DX), dxs + (int64_t(t) * B + b0) * TT, uint32_t(nb * DX_BLK), fb);
+                if (FMT == 1) {
+                    for (int k = 0; k < nb; ++k)
+                        if (((b0 + k + 1) % bpg) == 0)
+                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + (b0 + k) / bpg) * TT,
+                                     TT * 4, fb);
                 }
             }
             __syncwarp();
-            if (lane == 0 && (k == S - 1 || i == B - 1)) mbar_arrive(bar(&ctrl->empty[slot]));
+            issued = st + 1;
         }
-        const int n = n0 + p;
-        if (n < N && !*abort) {
+        // Let every copy this warp issued land before the CTA can exit. On the normal path
+        // the stage barriers complete (the MMA warp has consumed every stage). After an
+        // abort the producer may never arrive, so each wait is capped at 200 us, far longer
+        // than a few-KB copy takes to land.
+        for (int st = max(0, issued - NS); st < issued; ++st)
+            drain_wait_warp(bar(&ctrl->full[st % NS]), (st / NS) & 1, 200000ull);
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------ MMA issue
+        // Uniform loop over the warp; the elected lane issues every MMA and commit (a
+        // commit tracks the MMAs of the thread that issues it).
+        const bool leader = elect_one();
+        const uint32_t smem0 = smem_addr(smem);
+        for (int st = 0; st < nstages; ++st) {
+            const int slot = st % NS, g = st % NG;
+            if (!bounded_wait_warp(bar(&ctrl->full[slot]), (st / NS) & 1, abort)) break;
+            if (!bounded_wait_warp(bar(&ctrl->tempty[g]), ((st / NG) & 1) ^ 1, abort)) break;
+            tc_fence_after();
+            const int nb = min(S, B - st * S);
+            if (leader) {
+                for (int k = 0; k < nb; ++k) {
+                    const uint32_t w_addr = smem0 + uint32_t(slot * STAGE_BYTES + k * W_BLK);
+                    const uint32_t t_addr = smem0 + uint32_t(slot * STAGE_BYTES + OFF_T + k * T_BLK);
+                    const uint32_t d = tmem_base + uint32_t((g * S + k) * MN);
 #pragma unroll
-            for (int j = 0; j < EPI_COLS; j += 2) {
-                float a, b;
-                unpack2(acc[j / 2], a, b);
-                const int m = t * TT + c0 + j;
-                if (m < M) y[int64_t(m) * N + n] = a;
-                if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
+                    for (int part = 0; part < Gm::WP; ++part) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t wd = smem_desc_kmajor(w_addr + part * W_PART + h * 256, LBO, SBO);
+                            const uint64_t td = smem_desc_kmajor(t_addr + h * 256, LBO, SBO);
+                            if (TOKL)
+                                tc_mma_f16(d, td, wd, Gm::IDESC, (part | h) != 0);
+                            else
+                                tc_mma_f16(d, wd, td, Gm::IDESC, (part | h) != 0);
+                        }
+                    }
+                }
+                tc_commit(bar(&ctrl->tfull[g]));  // the stage's accumulators are complete and its operands read
+            }
+            __syncwarp();
+        }
+        // Wait until every MMA (and the barrier arrivals their commits trigger) is done
+        // before TMEM and shared memory are released.
+        uint32_t local_abort = 0;
+        if (leader) tc_commit(bar(&ctrl->drain));
+        __syncwarp();
+        bounded_wait_warp(bar(&ctrl->drain), 0, &local_abort);
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;             // TMEM lane quarter
+        const int c0 = (warp >> 2) * CW;    // first TMEM column of this warp
+        const int r = q * 32 + lane;        // this thread's TMEM lane: token (TOKL) or weight row
+        unsigned long long acc[CW / 2];     // f32 pairs, columns c0 + 2j, c0 + 2j + 1
+#pragma unroll
+        for (int j = 0; j < CW / 2; ++j) acc[j] = 0ull;
+        const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
+        for (int st = 0; st < nstages; ++st) {
+            const int slot = st % NS, g = st % NG;
+            const int nb = min(S, B - st * S);
+            if (!bounded_wait_warp(bar(&ctrl->tfull[g]), (st / NG) & 1, abort)) break;
+            tc_fence_after();
+            const uint8_t* sp = stage_ptr(slot);
+            bool released = false;
+#pragma unroll
+            for (int k = 0; k < S; ++k) {
+                if (k >= nb) break;
+                const int i = st * S + k;
+                const bool last = (k == nb - 1);
+                const float* dxk = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT;
+                const bool group_end = (FMT == 1) && (((i + 1) % bpg) == 0);
+                const float dxr = TOKL ? dxk[r] : 0.0f;
+#pragma unroll
+                for (int h0 = 0; h0 < CW; h0 += LD_COLS) {
+                    uint32_t pr[LD_COLS];
+                    tmem_load_cols(lane_base + uint32_t((g * S + k) * MN + c0 + h0), pr);
+                    if (last && h0 + LD_COLS == CW) {  // the group's tiles are all in registers: free it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(&ctrl->tempty[g]));
+                    }
+                    if (TOKL) {
+                        const unsigned long long dx2 = pack2(dxr, dxr);
+#pragma unroll
+                        for (int j = 0; j < LD_COLS / 2; ++j) fma2(acc[h0 / 2 + j], pr[2 * j], pr[2 * j + 1], dx2);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < LD_COLS; j += 4) {
+                            const float4 dv = *reinterpret_cast<const float4*>(dxk + c0 + h0 + j);
+                            fma2(acc[(h0 + j) / 2], pr[j], pr[j + 1], pack2(dv.x, dv.y));
+                            fma2(acc[(h0 + j) / 2 + 1], pr[j + 2], pr[j + 3], pack2(dv.z, dv.w));
+                        }
+                    }
+                }
+                if (group_end) {  // last block of a group: add (b + 8s) * Z
+                    const float* cs = reinterpret_cast<const float*>(sp + OFF_C) + k * NW;
+                    const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + k * TT;
+                    if (TOKL) {
+                        const float z = zs[r];
+                        const unsigned long long z2 = pack2(z, z);
+#pragma unroll
+                        for (int j = 0; j < CW; j += 4) {
+                            const float4 cv = *reinterpret_cast<const float4*>(cs + c0 + j);
+                            fma2_bias(acc[j / 2], cv.x, cv.y, z2);
+                            fma2_bias(acc[j / 2 + 1], cv.z, cv.w, z2);
+                        }
+                    } else {
+                        const float c = cs[r];
+                        const unsigned long long cc = pack2(c, c);
+#pragma unroll
+                        for (int j = 0; j < CW; j += 4) {
+                            const float4 zv = *reinterpret_cast<const float4*>(zs + c0 + j);
+                            fma2_bias(acc[j / 2], zv.x, zv.y, cc);
+                            fma2_bias(acc[j / 2 + 1], zv.z, zv.w, cc);
+                        }
+                    }
+                }
+            }
+            if (!released) {  // the values read from the stage were consumed above
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(&ctrl->empty[slot]));
+            }
+        }
+        if (!*abort) {
+            if (TOKL) {
+                const int m = t * TT + r;
+                const int nb = n0 + c0;
+                if (m < M) {
+                    float* yr = y + int64_t(m) * N + nb;
+                    if ((N & 3) == 0 && nb + CW <= N) {
+#pragma unroll
+                        for (int j = 0; j < CW; j += 4) {
+                            float a, b, c, e;
+                            unpack2(acc[j / 2], a, b);
+                            unpack2(acc[j / 2 + 1], c, e);
+                            *reinterpret_cast<float4*>(yr + j) = make_float4(a, b, c, e);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < CW; j += 2) {
+                            float a, b;
+                            unpack2(acc[j / 2], a, b);
+                            if (nb + j < N) yr[j] = a;
+                            if (nb + j + 1 < N) yr[j + 1] = b;
+                        }
+                    }
+                }
+            } else {
+                const int n = n0 + r;
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < CW; j += 2) {
+                        float a, b;
+                        unpack2(acc[j / 2], a, b);
+                        const int m = t * TT + c0 + j;
+                        if (m < M) y[int64_t(m) * N + n] = a;
+                        if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
+                    }
+                }
             }
         }
     }
@@ -375,7 +528,7 @@ __global__ void __launch_bounds__(Geo<TT>::NUM_THREADS, 1)
     __syncthreads();
     if (warp == MMA_WARP) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc(tmem_base, Gm::TMEM_COLS);
     }
 }
 

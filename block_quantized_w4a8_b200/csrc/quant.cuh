@@ -17,7 +17,7 @@
 namespace w4a8 {
 
 // Tensor-core operand geometry shared by the activation kernel and the GEMM: the
-// token tile (tokens per GEMM tile, the MMA's N) is 32, 64 or 128.
+// token tile (tokens per GEMM tile) is 16, 32, 64 or 128.
 namespace tcgeo {
 __host__ __device__ constexpr int tok_block_bytes(int tt) { return tt * 64; }  // one 32-wide block, fp16
 }  // namespace tcgeo
@@ -62,32 +62,26 @@ __global__ void __launch_bounds__(256) quant_act_rowmajor_kernel(const void* __r
 }
 
 // ------------------------------------------------------------------ Q8_0, MMA operand
-// Same quantisation, written as the fp16 B operand of the tcgen05 GEMM.
+// Same quantisation, written as the token operand of the tcgen05 GEMM.
 //
 // Layout (per token tile t of `tt` rows and block b): a contiguous chunk of tt x 32
-// fp16 at chunk index t*B + b. Inside a chunk, token row r and 16-byte
-// segment c (c = 0..3) sit at byte (r/8)*512 + c*128 + (r%8)*16: the K-major,
-// no-swizzle arrangement of 8-row x 16-byte core matrices (K-adjacent core matrices
-// 128 B apart, 8-row groups 512 B apart).
+// fp16 at chunk index t*B + b. Inside a chunk, token row r and 16-byte segment c
+// (c = 0..3) sit at byte (r/8)*512 + c*128 + (r%8)*16: the K-major, no-swizzle
+// arrangement of 8-row x 16-byte core matrices (K-adjacent core matrices 128 B apart,
+// 8-row groups 512 B apart).
 //
-// The 8 fp16 slots of segment c hold the block's elements in the order in which the
-// GEMM's weight expansion produces them (a permutation of K within the block, applied
-// identically to both operands, so every block dot is unchanged):
+// The 8 fp16 slots of segment c hold the block's codes q (exact small integers) in the
+// order in which the GEMM's weight expansion produces them (a permutation of K within
+// the block, applied identically to both operands, so every block dot is unchanged):
 //   FMT 0 (Q4_0):   4c, 4c+2, 4c+1, 4c+3, 16+4c, 16+4c+2, 16+4c+1, 16+4c+3
 //   FMT 1 (affine): 8c, 8c+4, 8c+2, 8c+6, 8c+1, 8c+5, 8c+3, 8c+7
-// Slots 0..3 store 16*q (the weight side holds the plain code there) and slots 4..7
-// store q (the weight side holds 16*code there), so every product is 16*(w_code*q):
-// the GEMM's block dot is exactly 16x the integer dot.
-// The block scale goes to `bs` as the tf32 operand of the GEMM's scale MMA: per chunk,
-// token r at 16 bytes (a, b, c, 0) with a + b + c == d/16 exactly (a keeps the top 11
-// significant bits of d/16, b the next 11, c the rest; each is representable in tf32,
-// whose low 13 mantissa bits are zero). Rows past M are zero. For FMT 1 it also writes,
-// per token and weight group g, Z = sum over the group's blocks of d*sum(q) (the factor
-// of the bias term).
+// The block scale d goes to `dxs[chunk*tt + r]` (f32). Rows past M are zero (codes and
+// scale). For FMT 1 it also writes, per token and weight group g, Z = the f32 sum over
+// the group's blocks of d*sum(q) (the factor of the bias term), at zb[(t*G + g)*tt + r].
 template <bool BF16, int FMT>
 __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restrict__ x, int M, int K, int tt,
                                                            int64_t nblocks, __half* __restrict__ tok,
-                                                           float4* __restrict__ bs, float* __restrict__ zb,
+                                                           float* __restrict__ dxs, float* __restrict__ zb,
                                                            int group) {
     pdl_launch_dependents();
     const int B = K >> 5;
@@ -125,10 +119,10 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         const int c = (FMT == 0) ? sub : (sub >> 1);
         int e[8];
         if (FMT == 0) {  // own = elements 4c..4c+3, other = 16+4c..16+4c+3
-            e[0] = 16 * code(mine, 0); e[1] = 16 * code(mine, 2); e[2] = 16 * code(mine, 1); e[3] = 16 * code(mine, 3);
+            e[0] = code(mine, 0); e[1] = code(mine, 2); e[2] = code(mine, 1); e[3] = code(mine, 3);
             e[4] = code(other, 0); e[5] = code(other, 2); e[6] = code(other, 1); e[7] = code(other, 3);
         } else {         // own = elements 8c..8c+3, other = 8c+4..8c+7
-            e[0] = 16 * code(mine, 0); e[1] = 16 * code(other, 0); e[2] = 16 * code(mine, 2); e[3] = 16 * code(other, 2);
+            e[0] = code(mine, 0); e[1] = code(other, 0); e[2] = code(mine, 2); e[3] = code(other, 2);
             e[4] = code(mine, 1); e[5] = code(other, 1); e[6] = code(mine, 3); e[7] = code(other, 3);
         }
         uint32_t h[4];
@@ -142,14 +136,7 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
                     (r & 7) * 16;
         *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
     }
-    if (valid && sub == 0) {
-        const float d16 = __fmul_rn(d, 0.0625f);
-        const float a = __uint_as_float(__float_as_uint(d16) & 0xFFFFE000u);
-        const float r1 = __fsub_rn(d16, a);  // exact: the low 13 significand bits of d16
-        const float b2 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
-        const float c2 = __fsub_rn(r1, b2);  // exact, at most 2 significant bits
-        bs[chunk * tt + r] = make_float4(a, b2, c2, 0.0f);
-    }
+    if (valid && sub == 0) dxs[chunk * tt + r] = d;
     if (FMT == 1) {
         // Blocks of one weight group are adjacent 8-lane groups of this warp (the warp's
         // four blocks start at a multiple of 4 and B is a multiple of group/32).

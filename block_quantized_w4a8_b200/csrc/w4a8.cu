@@ -52,13 +52,14 @@ GemvWs gemv_ws(void* ws, int M, int K) {
     return w;
 }
 
-// Token tile of the tensor-core GEMM for M rows of x: small M gets a small tile (less
-// padding, more TMEM block buffers).
-inline int tc_token_tile(int M) { return M <= 32 ? 32 : (M <= 64 ? 64 : 128); }
+// Token tile of the tensor-core GEMM for M rows of x. Up to 64 rows the tokens are the
+// MMA's N (16, 32 or 64 per tile, little padding); above, tiles of 128 tokens sit on the
+// TMEM lanes and the weight rows are the MMA's N.
+inline int tc_token_tile(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
 struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
     __half* tok;
-    float4* bs;
+    float* dxs;
     float* z;
     int tt;      // tokens per tile
     int tiles;
@@ -73,7 +74,7 @@ TcWs tc_ws(void* ws, int M, int K, int group) {
     size_t off = 0;
     char* base = static_cast<char*>(ws);
     w.tok = reinterpret_cast<__half*>(base + off); off = align256(off + size_t(rows) * B * 64);
-    w.bs = reinterpret_cast<float4*>(base + off); off = align256(off + size_t(rows) * B * 16);
+    w.dxs = reinterpret_cast<float*>(base + off); off = align256(off + size_t(rows) * B * 4);
     w.z = reinterpret_cast<float*>(base + off);
     if (group > 0) off = align256(off + size_t(rows) * (K / group) * 4);
     w.bytes = off;
@@ -81,8 +82,12 @@ TcWs tc_ws(void* ws, int M, int K, int group) {
 }
 
 // ------------------------------------------------------------------ launch helpers
+// Launch with programmatic dependent launch allowed (`pdl`): the kernel may start while
+// the preceding kernel of the stream drains; it reads that kernel's output only after
+// griddepcontrol.wait.
 template <typename Kern, typename... Args>
-cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+cudaError_t launch_pdl_if(bool pdl, Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -92,8 +97,12 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+    return launch_pdl_if(true, kernel, grid, block, smem, stream, args...);
 }
 
 w4a8_status run_quant_rowmajor(const void* x, w4a8_dtype dt, int M, int K, int8_t* qx, float* dx, int32_t* sx,
@@ -112,14 +121,14 @@ w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, 
     const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
     if (group == 0) {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, 0);
+            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0);
         else
-            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, 0);
+            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0);
     } else {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, group);
+            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group);
         else
-            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.bs, w.z, group);
+            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group);
     }
     return launch_status();
 }
@@ -224,34 +233,37 @@ w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_d
     return cuda_status(e);
 }
 
-template <int FMT, int TT>
+template <int FMT, bool TOKL, int MN>
 w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                           const uint16_t* wb, float* y, cudaStream_t stream) {
-    using Gm = tc::Geo<TT>;
+                           const uint16_t* wb, float* y, bool pdl, cudaStream_t stream) {
+    using Gm = tc::Geo<FMT, TOKL, MN>;
     static bool configured[64] = {false};
     int dev = 0;
     const cudaError_t ed = cudaGetDevice(&dev);
     if (ed != cudaSuccess) return cuda_status(ed);
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT, TT>,
+        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT, TOKL, MN>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM_BYTES);
         if (ea != cudaSuccess) return cuda_status(ea);
         configured[dev] = true;
     }
-    const dim3 grid(unsigned(cdiv(N, tc::BN)), unsigned(w.tiles));
-    cudaError_t e = launch_pdl(tc::gemm_tc_kernel<FMT, TT>, grid, dim3(Gm::NUM_THREADS), size_t(Gm::SMEM_BYTES),
-                               stream, M, N, K, group, (const __half*)w.tok, (const float4*)w.bs, (const float*)w.z,
-                               wq, ws, wb, y);
+    const dim3 grid(unsigned(cdiv(N, Gm::NW)), unsigned(w.tiles));
+    cudaError_t e = launch_pdl_if(pdl, tc::gemm_tc_kernel<FMT, TOKL, MN>, grid, dim3(Gm::NUM_THREADS),
+                                  size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
+                                  (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y);
     return cuda_status(e);
 }
 
+// Orientation by token tile: tiles of 16..64 tokens put the tokens on the MMA's N; tiles
+// of 128 tokens put them on the TMEM lanes with 128 weight rows per tile.
 template <int FMT>
 w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                        const uint16_t* wb, float* y, cudaStream_t stream) {
+                        const uint16_t* wb, float* y, bool pdl, cudaStream_t stream) {
     switch (w.tt) {
-        case 32: return launch_gemm_tc<FMT, 32>(M, N, K, group, w, wq, ws, wb, y, stream);
-        case 64: return launch_gemm_tc<FMT, 64>(M, N, K, group, w, wq, ws, wb, y, stream);
-        default: return launch_gemm_tc<FMT, 128>(M, N, K, group, w, wq, ws, wb, y, stream);
+        case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
+        case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
+        case 64: return launch_gemm_tc<FMT, false, 64>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
+        default: return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
     }
 }
 
@@ -288,12 +300,15 @@ w4a8_status prepare_impl(int M, int K, int group, const void* x, w4a8_dtype dt, 
     return run_quant_tc(x, dt, M, K, group, tc_ws(work, M, K, group), stream);
 }
 
-// Contraction from a prepared workspace.
+// Contraction from a prepared workspace. `after_quant`: the preceding kernel in the
+// stream is this call's own activation quantisation, so the contraction may overlap its
+// tail (programmatic dependent launch); otherwise it starts after all prior work.
 template <int FMT>
 w4a8_status contract_impl(int M, int N, int K, int group, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb,
-                          float* y, void* work, bool gemv, cudaStream_t stream) {
+                          float* y, void* work, bool gemv, bool after_quant, cudaStream_t stream) {
     if (gemv) return run_gemv<FMT>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, stream);
-    return run_gemm_tc<FMT>(M, N, K, group, tc_ws(work, M, K, FMT == 1 ? group : 0), wq, ws, wb, y, stream);
+    return run_gemm_tc<FMT>(M, N, K, group, tc_ws(work, M, K, FMT == 1 ? group : 0), wq, ws, wb, y, after_quant,
+                            stream);
 }
 
 template <int FMT>
@@ -306,7 +321,7 @@ w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype 
     if (gemv && gemv_fused(M, K)) return run_gemv_fused<FMT>(M, N, K, group, x, dt, wq, ws, wb, y, stream);
     st = prepare_impl(M, K, FMT == 1 ? group : 0, x, dt, work, gemv, stream);
     if (st != W4A8_OK) return st;
-    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, gemv, stream);
+    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, gemv, true, stream);
 }
 
 }  // namespace
@@ -400,7 +415,8 @@ w4a8_status w4a8_gemm_prepared(int M, int N, int K, const uint8_t* qs, const uin
                                const void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
     w4a8_status st = check_gemm_args(M, N, K, qs, W4A8_F32, qs, d_fp16, nullptr, false, 0, y, ws, ws_bytes, path);
     if (st != W4A8_OK) return st;
-    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, const_cast<void*>(ws), use_gemv(M, path), stream);
+    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, const_cast<void*>(ws), use_gemv(M, path), false,
+                           stream);
 }
 
 w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint32_t* q, const uint16_t* scale_bf16,
@@ -411,7 +427,7 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
         check_gemm_args(M, N, K, wq, W4A8_F32, wq, scale_bf16, bias_bf16, true, group, y, ws, ws_bytes, path);
     if (st != W4A8_OK) return st;
     return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, const_cast<void*>(ws), use_gemv(M, path),
-                            stream);
+                            false, stream);
 }
 
 // Scratch of w4a8_gemm_noalloc. In host code this name is only a stand-in for the
@@ -444,7 +460,8 @@ w4a8_status w4a8_last_device_error(void) {
     if (cudaMemcpyFromSymbol(&v, w4a8::g_device_status, sizeof(v)) != cudaSuccess) return W4A8_ERR_CUDA;
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(w4a8::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return W4A8_ERR_CUDA;
-    return v ? W4A8_ERR_DEVICE_TIMEOUT : W4A8_OK;
+    if (v & w4a8::kDevErrTimeout) return W4A8_ERR_DEVICE_TIMEOUT;
+    return v ? W4A8_ERR_RANGE : W4A8_OK;
 }
 
 const char* w4a8_last_cuda_error_string(void) { return cudaGetErrorString(t_last_cuda_error); }
@@ -458,6 +475,7 @@ const char* w4a8_status_string(w4a8_status s) {
         case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
         case W4A8_ERR_DEVICE_TIMEOUT: return "W4A8_ERR_DEVICE_TIMEOUT";
         case W4A8_ERR_MISALIGNED: return "W4A8_ERR_MISALIGNED";
+        case W4A8_ERR_RANGE: return "W4A8_ERR_RANGE";
     }
     return "W4A8_UNKNOWN_STATUS";
 }

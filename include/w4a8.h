@@ -42,7 +42,9 @@ typedef enum {
     W4A8_ERR_WORKSPACE = 3,      /* workspace pointer null or smaller than w4a8_workspace_bytes() */
     W4A8_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed */
     W4A8_ERR_DEVICE_TIMEOUT = 5, /* a bounded wait inside a kernel ran out (see w4a8_last_device_error) */
-    W4A8_ERR_MISALIGNED = 6      /* a pointer is not 16-byte aligned */
+    W4A8_ERR_MISALIGNED = 6,     /* a pointer is not 16-byte aligned */
+    W4A8_ERR_RANGE = 7           /* a weight scale outside the tensor-core path's exact range
+                                    (see w4a8_gemm); reported by w4a8_last_device_error */
 } w4a8_status;
 
 /* Element type of the unquantised input (x or W). bf16 is widened exactly to f32. */
@@ -101,6 +103,11 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group);
  *            w4a8_workspace_bytes(M, N, K, 0) bytes, owned by the caller; contents on
  *            entry are ignored and are garbage afterwards. Calls that share a workspace
  *            must be ordered on one stream.
+ * Scale range: the tensor-core path (M > 8, or PATH_GEMM) holds d_w * (q - 8) exactly as
+ * two fp16 values, which requires |d_w| <= 8188 (weights of magnitude up to ~65500). A
+ * larger, infinite or NaN scale makes the kernel set W4A8_ERR_RANGE in the device status
+ * word (w4a8_last_device_error) and the affected outputs are not reliable. The GEMV path
+ * (M <= 8, or PATH_GEMV) has no such limit.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, WORKSPACE, CUDA.
  */
 w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype,
@@ -130,6 +137,8 @@ w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int 
  * y = x . W^T with W affine 4-bit (from w4a8_pack_affine) and x quantised to Q8_0 in the
  * call. The contraction runs on the original codes: per activation block b inside
  * group g, y += d_x * (s_g * sum q*q_x + b_g * sum q_x). Tolerance as w4a8_gemm.
+ * Scale range of the tensor-core path: s = 0 or 2^-17 <= |s| <= 8188 (s * (q - 8) is then
+ * exact in fp16); other scales set W4A8_ERR_RANGE as in w4a8_gemm.
  * Arguments and errors as w4a8_gemm, plus `group` (64 or 128).
  */
 w4a8_status w4a8_gemm_affine(int M, int N, int K, int group, const void* x, w4a8_dtype dtype,
@@ -194,9 +203,11 @@ w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dty
 
 /*
  * Reads and clears the device status word that kernels set when a bounded wait runs
- * out. Synchronises the current device. Returns W4A8_OK when no kernel has reported a
- * problem since the last call, W4A8_ERR_DEVICE_TIMEOUT otherwise, W4A8_ERR_CUDA if the
- * read itself failed.
+ * out or a weight scale is outside the tensor-core path's range. Synchronises the
+ * current device. Returns W4A8_OK when no kernel has reported a problem since the last
+ * call, W4A8_ERR_DEVICE_TIMEOUT if a wait ran out (this takes precedence),
+ * W4A8_ERR_RANGE if only a scale was out of range, W4A8_ERR_CUDA if the read itself
+ * failed.
  */
 w4a8_status w4a8_last_device_error(void);
 

@@ -53,9 +53,9 @@ def _align(v):
 def test_workspace_bytes(lib, M, N, K, group):
     B = K // 32
     gemv = _align(M * K) + _align(M * B * 4) + _align(M * B * 4)
-    tt = 32 if M <= 32 else (64 if M <= 64 else 128)
+    tt = 16 if M <= 16 else (32 if M <= 32 else (64 if M <= 64 else 128))
     rows = -(-M // tt) * tt
-    tc = _align(rows * B * 64) + _align(rows * B * 16) + (_align(rows * (K // group) * 4) if group else 0)
+    tc = _align(rows * B * 64) + _align(rows * B * 4) + (_align(rows * (K // group) * 4) if group else 0)
     assert w4a8.w4a8_workspace_bytes(M, N, K, group) == max(gemv, tc)
 
 

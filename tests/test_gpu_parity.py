@@ -112,8 +112,8 @@ def test_pack_affine_bit_exact(group, N, K, dtype):
 
 
 # ------------------------------------------------------------------ Q4_0 matmul, full compare
-SHAPES = [(1, 1, 32), (1, 4096, 4096), (2, 333, 800), (5, 1536, 384), (8, 200, 256), (64, 1536, 384),
-          (300, 333, 800), (129, 128, 128), (130, 257, 4128), (3, 64, 32768)]
+SHAPES = [(1, 1, 32), (1, 4096, 4096), (2, 333, 800), (5, 1536, 384), (8, 200, 256), (17, 96, 640),
+          (32, 520, 1056), (64, 1536, 384), (300, 333, 800), (129, 128, 128), (130, 257, 4128), (3, 64, 32768)]
 
 
 def _q4_0_case(M, N, K, x_dtype="f32", w_std=0.02, seed=0):
@@ -172,6 +172,25 @@ def test_gemm_is_deterministic_and_ignores_workspace_contents():
         assert torch.equal(y1, y2)
 
 
+def test_scale_outside_tensor_core_range_is_reported():
+    """A Q4_0 block scale above 8188 cannot be held exactly by the tensor-core path's fp16
+    weight operand: that path reports W4A8_ERR_RANGE through the device status word, while
+    the GEMV path (no such limit) stays within tolerance."""
+    M, N, K = 40, 128, 256
+    x, w, *_ = _q4_0_case(M, N, K, seed=21)
+    w[5, :32] *= 100000.0 / float(w[5, :32].abs().max())  # block scale 12500
+    rqs, rd = oracle.pack_q4_0(w.numpy())
+    rqx, rdx, _ = oracle.quant_act_q8_0(x.numpy())
+    yref, T = oracle.gemm_q4_0(rqx, rdx, rqs, rd, nthreads=8)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    assert w4a8.w4a8_last_device_error() == 0
+    check_tol(as_np(w4a8.gemm(dev(x), qs, d, path=w4a8.PATH_GEMV)), yref, T, "gemv, large scale")
+    assert w4a8.w4a8_last_device_error() == 0
+    w4a8.gemm(dev(x), qs, d, path=w4a8.PATH_GEMM)
+    assert w4a8.w4a8_last_device_error() == 7  # W4A8_ERR_RANGE, read and cleared
+    assert w4a8.w4a8_last_device_error() == 0
+
+
 def test_empty_input_is_rejected():
     qs = torch.zeros(8, 16, dtype=torch.uint8, device="cuda")
     d = torch.zeros(8, 1, dtype=torch.int16, device="cuda")
@@ -204,7 +223,8 @@ def test_full_size_sampled(wl):
 
 
 # ------------------------------------------------------------------ affine
-AFFINE_SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (64, 1536, 384), (200, 333, 1280), (130, 128, 4096)]
+AFFINE_SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (20, 128, 640), (32, 256, 1024), (64, 1536, 384),
+                 (200, 333, 1280), (130, 128, 4096)]
 
 
 @pytest.mark.parametrize("group", [64, 128])
