@@ -414,9 +414,12 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
         const int q = warp & 3;             // TMEM lane quarter
         const int c0 = (warp >> 2) * CW;    // first TMEM column of this warp
         const int r = q * 32 + lane;        // this thread's TMEM lane: token (TOKL) or weight row
-        unsigned long long acc[CW / 2];     // f32 pairs, columns c0 + 2j, c0 + 2j + 1
+        // f32 accumulators, one per column. Scalar FMAs: the packed f32x2 form does the same
+        // work on the FMA pipe and would need its operands re-paired after each tensor-
+        // memory load, which costs more issue slots than it saves.
+        float acc[CW];
 #pragma unroll
-        for (int j = 0; j < CW / 2; ++j) acc[j] = 0ull;
+        for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
         const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
         for (int st = 0; st < nstages; ++st) {
             const int slot = st % NS, g = st % NG;
@@ -443,15 +446,16 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                         if (lane == 0) mbar_arrive(bar(&ctrl->tempty[g]));
                     }
                     if (TOKL) {
-                        const unsigned long long dx2 = pack2(dxr, dxr);
 #pragma unroll
-                        for (int j = 0; j < LD_COLS / 2; ++j) fma2(acc[h0 / 2 + j], pr[2 * j], pr[2 * j + 1], dx2);
+                        for (int j = 0; j < LD_COLS; ++j) acc[h0 + j] = fmaf(__uint_as_float(pr[j]), dxr, acc[h0 + j]);
                     } else {
 #pragma unroll
                         for (int j = 0; j < LD_COLS; j += 4) {
                             const float4 dv = *reinterpret_cast<const float4*>(dxk + c0 + h0 + j);
-                            fma2(acc[(h0 + j) / 2], pr[j], pr[j + 1], pack2(dv.x, dv.y));
-                            fma2(acc[(h0 + j) / 2 + 1], pr[j + 2], pr[j + 3], pack2(dv.z, dv.w));
+                            acc[h0 + j] = fmaf(__uint_as_float(pr[j]), dv.x, acc[h0 + j]);
+                            acc[h0 + j + 1] = fmaf(__uint_as_float(pr[j + 1]), dv.y, acc[h0 + j + 1]);
+                            acc[h0 + j + 2] = fmaf(__uint_as_float(pr[j + 2]), dv.z, acc[h0 + j + 2]);
+                            acc[h0 + j + 3] = fmaf(__uint_as_float(pr[j + 3]), dv.w, acc[h0 + j + 3]);
                         }
                     }
                 }
@@ -460,21 +464,23 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                     const float* zs = reinterpret_cast<const float*>(sp + OFF_Z) + k * TT;
                     if (TOKL) {
                         const float z = zs[r];
-                        const unsigned long long z2 = pack2(z, z);
 #pragma unroll
                         for (int j = 0; j < CW; j += 4) {
                             const float4 cv = *reinterpret_cast<const float4*>(cs + c0 + j);
-                            fma2_bias(acc[j / 2], cv.x, cv.y, z2);
-                            fma2_bias(acc[j / 2 + 1], cv.z, cv.w, z2);
+                            acc[j] = fmaf(cv.x, z, acc[j]);
+                            acc[j + 1] = fmaf(cv.y, z, acc[j + 1]);
+                            acc[j + 2] = fmaf(cv.z, z, acc[j + 2]);
+                            acc[j + 3] = fmaf(cv.w, z, acc[j + 3]);
                         }
                     } else {
                         const float c = cs[r];
-                        const unsigned long long cc = pack2(c, c);
 #pragma unroll
                         for (int j = 0; j < CW; j += 4) {
                             const float4 zv = *reinterpret_cast<const float4*>(zs + c0 + j);
-                            fma2_bias(acc[j / 2], zv.x, zv.y, cc);
-                            fma2_bias(acc[j / 2 + 1], zv.z, zv.w, cc);
+                            acc[j] = fmaf(zv.x, c, acc[j]);
+                            acc[j + 1] = fmaf(zv.y, c, acc[j + 1]);
+                            acc[j + 2] = fmaf(zv.z, c, acc[j + 2]);
+                            acc[j + 3] = fmaf(zv.w, c, acc[j + 3]);
                         }
                     }
                 }
@@ -492,32 +498,21 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                     float* yr = y + int64_t(m) * N + nb;
                     if ((N & 3) == 0 && nb + CW <= N) {
 #pragma unroll
-                        for (int j = 0; j < CW; j += 4) {
-                            float a, b, c, e;
-                            unpack2(acc[j / 2], a, b);
-                            unpack2(acc[j / 2 + 1], c, e);
-                            *reinterpret_cast<float4*>(yr + j) = make_float4(a, b, c, e);
-                        }
+                        for (int j = 0; j < CW; j += 4)
+                            *reinterpret_cast<float4*>(yr + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < CW; j += 2) {
-                            float a, b;
-                            unpack2(acc[j / 2], a, b);
-                            if (nb + j < N) yr[j] = a;
-                            if (nb + j + 1 < N) yr[j + 1] = b;
-                        }
+                        for (int j = 0; j < CW; ++j)
+                            if (nb + j < N) yr[j] = acc[j];
                     }
                 }
             } else {
                 const int n = n0 + r;
                 if (n < N) {
 #pragma unroll
-                    for (int j = 0; j < CW; j += 2) {
-                        float a, b;
-                        unpack2(acc[j / 2], a, b);
+                    for (int j = 0; j < CW; ++j) {
                         const int m = t * TT + c0 + j;
-                        if (m < M) y[int64_t(m) * N + n] = a;
-                        if (m + 1 < M) y[int64_t(m + 1) * N + n] = b;
+                        if (m < M) y[int64_t(m) * N + n] = acc[j];
                     }
                 }
             }
