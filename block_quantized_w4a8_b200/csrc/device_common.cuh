@@ -181,6 +181,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
+// 2-D tiled tensor copy (TMA) global -> shared of one box of the tensor map at `tmap`
+// (a __grid_constant__ kernel parameter), box origin (c0 = innermost, c1), completing its
+// bytes on mbarrier `bar`. Plain (no multicast). c0 times the element size must be a
+// multiple of 16 bytes; parts of the box outside the tensor are filled with zeros.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -45,6 +45,8 @@
 // returns.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (the type only; maps are encoded by the host code)
+
 #include "device_common.cuh"
 #include "quant.cuh"
 
@@ -75,15 +77,19 @@ struct Geo {
     static constexpr int T_BLK = TT * 64;
     static constexpr int DX_BLK = TT * 4;
     static constexpr int PER_BLK = W_BLK + T_BLK;
-    // Quant blocks per pipeline stage. One tcgen05.commit covers a stage (a commit costs
-    // the tensor pipe about as much as 1.5 MMAs of 128x128x16), so small tiles take more
-    // blocks per stage.
-    static constexpr int S = (!TOKL && MN <= 32) ? 4 : (PER_BLK <= 12288 ? 4 : (PER_BLK <= 24576 ? 2 : 1));
+    // Quant blocks per pipeline stage (one tcgen05.commit covers a stage).
+    static constexpr int S = PER_BLK <= 12288 ? 4 : (PER_BLK <= 24576 ? 2 : 1);
     static constexpr int OFF_T = S * W_BLK;
     static constexpr int OFF_DX = OFF_T + S * T_BLK;
     static constexpr int OFF_C = align_up(OFF_DX + S * DX_BLK, 128);           // affine: b + 8s per row
     static constexpr int OFF_Z = OFF_C + (FMT == 1 ? S * NW * 4 : 0);          // affine: Z per token
-    static constexpr int STAGE_BYTES = align_up(OFF_Z + (FMT == 1 ? S * TT * 4 : 0), 1024);
+    // Packed weights as fetched by TMA: per block of the stage a [NW rows][16 B] box of
+    // codes; the scales (and affine biases) of the 8 blocks (groups) around the stage as a
+    // [NW rows][8 x 16 bit] box each.
+    static constexpr int OFF_RAW = align_up(OFF_Z + (FMT == 1 ? S * TT * 4 : 0), 128);
+    static constexpr int OFF_RSC = OFF_RAW + S * NW * 16;
+    static constexpr int OFF_RBI = OFF_RSC + NW * 16;
+    static constexpr int STAGE_BYTES = align_up(OFF_RBI + (FMT == 1 ? NW * 16 : 0), 1024);
     static constexpr int NS = cmin(8, (SMEM_LIMIT - CTRL_BYTES - 1024) / STAGE_BYTES);
     static constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;
     static constexpr int NBUF = cmin(16, 512 / MN);  // TMEM accumulator tiles (one per block)
@@ -113,6 +119,7 @@ struct Geo {
 
 constexpr int MAX_NS = 8, MAX_NG = 8;
 struct Ctrl {
+    unsigned long long raw[MAX_NS];     // TMA of the packed weights (1 arrival + bytes)
     unsigned long long full[MAX_NS];    // producer threads (one arrival per weight row) + bulk copies (1 + bytes)
     unsigned long long empty[MAX_NS];   // one arrival per epilogue warp (after the stage's MMAs completed
                                         // and the warp read the stage's scales)
@@ -147,27 +154,13 @@ __device__ __forceinline__ uint32_t scaled_codes(uint32_t raw, uint32_t d2x2, ui
 }
 __device__ __forceinline__ uint32_t pair_of(__half h) { return uint32_t(__half_as_ushort(h)) * 0x10001u; }
 
-// Global loads written as volatile asm so that the compiler issues them where they stand
-// in the program (stages ahead of their use) instead of sinking them to the first use.
-__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
+// Global load written as volatile asm so that the compiler issues it where it stands in
+// the program (stages ahead of its use) instead of sinking it to the first use.
 __device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
     uint16_t v;
     asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
 }
-
-// Codes and scale bits of one stage of one weight row, held in registers until stored.
-template <int S>
-struct RowStage {
-    uint4 w[S];
-    uint16_t s[S], b[S];
-};
 
 // Loads CW TMEM columns of this warp's lane quarter into registers (and waits for them).
 __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[64]) {
@@ -188,11 +181,13 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
     gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dxs,
                    const float* __restrict__ zb, const uint8_t* __restrict__ wq,
                    const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
-                   float* __restrict__ y) {
+                   float* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int sc_tma) {
     using Gm = Geo<FMT, TOKL, MN>;
     constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NW = Gm::NW, CW = Gm::CW;
     constexpr int W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK, DX_BLK = Gm::DX_BLK;
     constexpr int OFF_T = Gm::OFF_T, OFF_DX = Gm::OFF_DX, OFF_C = Gm::OFF_C, OFF_Z = Gm::OFF_Z;
+    constexpr int OFF_RAW = Gm::OFF_RAW, OFF_RSC = Gm::OFF_RSC, OFF_RBI = Gm::OFF_RBI;
     constexpr int STAGE_BYTES = Gm::STAGE_BYTES, EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0;
     constexpr int LD_COLS = Gm::LD_COLS;
     constexpr int PROD_THREADS = Gm::PROD_WARPS * 32;
@@ -215,6 +210,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(&ctrl->raw[s]), 1);
             mbar_init(bar(&ctrl->full[s]), PROD_THREADS + 1);
             mbar_init(bar(&ctrl->empty[s]), EPI_WARPS);
         }
@@ -243,37 +239,55 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
         const int p = threadIdx.x - PROD_WARP0 * 32;  // weight row within the tile
         const int n = n0 + p;
         const bool row_ok = n < N;
-        const uint4* wrow = reinterpret_cast<const uint4*>(wq + int64_t(row_ok ? n : 0) * (K >> 1));
         bool range_bad = false;
-        auto load = [&](int st, RowStage<S>& rs) {
+        // Scales of the stages st, st+1, st+2 when they are not fetched by TMA (their row
+        // pitch is not a multiple of 16 bytes): plain loads two stages ahead.
+        uint16_t sA[S], sB[S], sC[S], bA[S], bB[S], bC[S];
+        auto load_sc = [&](int st, uint16_t (&sv)[S], uint16_t (&bv)[S]) {
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 const int b = st * S + k;
-                rs.w[k] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);  // codes 8: zero
-                rs.s[k] = 0;
-                rs.b[k] = 0;
-                if (row_ok && b < B) {
-                    rs.w[k] = ld_nc_v4(wrow + b);
+                sv[k] = 0;
+                bv[k] = 0;
+                if (!sc_tma && row_ok && b < B) {
                     if (FMT == 0) {
-                        rs.s[k] = ld_nc_u16(wscale + int64_t(n) * B + b);
+                        sv[k] = ld_nc_u16(wscale + int64_t(n) * B + b);
                     } else {
-                        rs.s[k] = ld_nc_u16(wscale + int64_t(n) * G + b / bpg);
-                        rs.b[k] = ld_nc_u16(wbias + int64_t(n) * G + b / bpg);
+                        sv[k] = ld_nc_u16(wscale + int64_t(n) * G + b / bpg);
+                        bv[k] = ld_nc_u16(wbias + int64_t(n) * G + b / bpg);
                     }
                 }
             }
         };
-        // Store one stage into shared memory; false if the wait gave up.
-        auto produce = [&](int st, const RowStage<S>& rs) {
+        load_sc(0, sA, bA);
+        load_sc(1, sB, bB);
+        load_sc(2, sC, bC);
+        for (int st = 0; st < nstages; ++st) {
             const int slot = st % NS;
-            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) return false;
+            // The packed weights of this stage are in shared memory (the copy warp took the
+            // slot from the epilogue before fetching them).
+            if (!bounded_wait_warp(bar(&ctrl->raw[slot]), (st / NS) & 1, abort)) break;
             uint8_t* sp = stage_ptr(slot);
+            const int e0 = (FMT == 0) ? (st * S) & ~7 : ((st * S) / bpg) & ~7;  // first scale of the TMA box
 #pragma unroll
             for (int k = 0; k < S; ++k) {
-                const uint32_t w[4] = {rs.w[k].x, rs.w[k].y, rs.w[k].z, rs.w[k].w};
+                const int b = st * S + k;
+                uint4 wv = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);  // codes 8: zero
+                uint32_t sb = 0, bb = 0;
+                if (b < B) {
+                    wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + k * NW * 16 + p * 16);
+                    if (sc_tma) {
+                        const int e = (FMT == 0) ? b : b / bpg;
+                        sb = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + p * 16)[e - e0];
+                        if (FMT == 1) bb = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + p * 16)[e - e0];
+                    } else {
+                        sb = sA[k];
+                        bb = bA[k];
+                    }
+                }
+                const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
                 uint8_t* dst = sp + k * W_BLK + (p >> 3) * 512 + (p & 7) * 16;
                 if (FMT == 0) {
-                    const uint32_t sb = rs.s[k];
                     range_bad |= (sb & 0x7FF8u) > 0x6950u;  // d_hi > 2720 (24 d_hi > 65504), inf or nan
                     const __half dh = __ushort_as_half(uint16_t(sb & 0xFFF8u));
                     const __half dl = __hsub(__ushort_as_half(uint16_t(sb)), dh);  // exact
@@ -293,7 +307,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                                        scaled_codes(r[2], l2, l24), scaled_codes(r[3], l2, l24));
                     }
                 } else {
-                    const float sf = __bfloat162float(__ushort_as_bfloat16(rs.s[k]));
+                    const float sf = __bfloat162float(__ushort_as_bfloat16(uint16_t(sb)));
                     const float af = fabsf(sf);
                     range_bad |= !(af <= 2720.0f) || (af != 0.0f && af < 7.62939453125e-06f);  // 2^-17
                     const __half sh = __float2half_rn(sf);  // exact in range
@@ -307,29 +321,24 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                             make_uint4(scaled_codes(r[0], s2, s24), scaled_codes(r[1], s2, s24),
                                        scaled_codes(r[2], s2, s24), scaled_codes(r[3], s2, s24));
                     }
-                    const int b = st * S + k;
                     if (((b + 1) % bpg) == 0) {  // last block of a group: its bias factor b + 8s
-                        const float bf = __bfloat162float(__ushort_as_bfloat16(rs.b[k]));
+                        const float bf = __bfloat162float(__ushort_as_bfloat16(uint16_t(bb)));
                         reinterpret_cast<float*>(sp + OFF_C)[k * NW + p] = __fadd_rn(bf, __fmul_rn(8.0f, sf));
                     }
                 }
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(&ctrl->full[slot]));
-            return true;
-        };
-        RowStage<S> r0, r1, r2;  // stages st, st+1, st+2 in flight
-        load(0, r0);
-        if (1 < nstages) load(1, r1);
-        for (int st = 0; st < nstages; st += 3) {
-            if (st + 2 < nstages) load(st + 2, r2);
-            if (!produce(st, r0)) break;
-            if (st + 1 >= nstages) break;
-            if (st + 3 < nstages) load(st + 3, r0);
-            if (!produce(st + 1, r1)) break;
-            if (st + 2 >= nstages) break;
-            if (st + 4 < nstages) load(st + 4, r1);
-            if (!produce(st + 2, r2)) break;
+            if (!sc_tma) {
+#pragma unroll
+                for (int k = 0; k < S; ++k) {
+                    sA[k] = sB[k];
+                    sB[k] = sC[k];
+                    bA[k] = bB[k];
+                    bB[k] = bC[k];
+                }
+                load_sc(st + 3, sC, bC);
+            }
         }
         if (range_bad) atomicOr(&g_device_status, kDevErrRange);
     } else if (warp == COPY_WARP) {
@@ -347,8 +356,18 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 int nz = 0;  // affine: group ends in this stage (each brings its Z row)
                 if (FMT == 1)
                     for (int k = 0; k < nb; ++k) nz += ((b0 + k + 1) % bpg) == 0;
-                const uint32_t fb = bar(&ctrl->full[slot]);
                 uint8_t* sp = stage_ptr(slot);
+                // packed weights of the stage (codes, and scales when their pitch allows TMA)
+                const uint32_t rb = bar(&ctrl->raw[slot]);
+                const int e0 = (FMT == 0) ? b0 & ~7 : (b0 / bpg) & ~7;
+                mbar_arrive_expect_tx(rb, uint32_t(nb * NW * 16 + (sc_tma ? NW * 16 * (FMT == 1 ? 2 : 1) : 0)));
+                for (int k = 0; k < nb; ++k)
+                    tma_load_2d(smem_addr(sp + OFF_RAW + k * NW * 16), &tm_q, (b0 + k) * 16, n0, rb);
+                if (sc_tma) {
+                    tma_load_2d(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
+                    if (FMT == 1) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
+                }
+                const uint32_t fb = bar(&ctrl->full[slot]);
                 mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK) + nz * TT * 4));
                 bulk_g2s(smem_addr(sp + OFF_T), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK,
                          uint32_t(nb * T_BLK), fb);
@@ -367,8 +386,10 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
         // the stage barriers complete (the MMA warp has consumed every stage). After an
         // abort the producer may never arrive, so each wait is capped at 200 us, far longer
         // than a few-KB copy takes to land.
-        for (int st = max(0, issued - NS); st < issued; ++st)
+        for (int st = max(0, issued - NS); st < issued; ++st) {
+            drain_wait_warp(bar(&ctrl->raw[st % NS]), (st / NS) & 1, 200000ull);
             drain_wait_warp(bar(&ctrl->full[st % NS]), (st / NS) & 1, 200000ull);
+        }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issue
         // Uniform loop over the warp; the elected lane issues every MMA and commit (a

@@ -2,7 +2,11 @@
 // Declarations and the contract of each call: include/w4a8.h.
 #include "w4a8.h"
 
+#include <string.h>
+
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "device_common.cuh"
 #include "gemm_tc.cuh"
@@ -233,6 +237,38 @@ w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_d
     return cuda_status(e);
 }
 
+// cuTensorMapEncodeTiled, resolved once through the runtime (no link against the driver
+// library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D tensor map over a row-major [rows][cols] array of `esize`-byte elements with row
+// pitch `pitch` bytes, box [box_rows][box_cols]; no swizzle, zero fill outside.
+bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols, uint64_t rows,
+               uint64_t pitch, uint32_t box_cols, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    (void)esize;
+    return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int FMT, bool TOKL, int MN>
 w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
                            const uint16_t* wb, float* y, bool pdl, cudaStream_t stream) {
@@ -247,10 +283,29 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
         if (ea != cudaSuccess) return cuda_status(ea);
         configured[dev] = true;
     }
+    // Tensor maps of the packed weights: codes as bytes [N][K/2] in boxes of 16 bytes (one
+    // quant block) x NW rows; scales (affine: scales and biases) as 16-bit [N][E] in boxes
+    // of 8 x NW, fetched by TMA only when the row pitch 2E is a multiple of 16 bytes.
+    CUtensorMap tq, tsc, tbi;
+    memset(&tsc, 0, sizeof(tsc));
+    memset(&tbi, 0, sizeof(tbi));
+    if (!encode_2d(&tq, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 16,
+                   Gm::NW))
+        return W4A8_ERR_CUDA;
+    const int E = (FMT == 0) ? K / 32 : K / group;  // scales per row
+    int sc_tma = ((E * 2) % 16) == 0 ? 1 : 0;
+    if (sc_tma) {
+        if (!encode_2d(&tsc, ws, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N), uint64_t(E) * 2, 8,
+                       Gm::NW))
+            return W4A8_ERR_CUDA;
+        if (FMT == 1 && !encode_2d(&tbi, wb, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N),
+                                   uint64_t(E) * 2, 8, Gm::NW))
+            return W4A8_ERR_CUDA;
+    }
     const dim3 grid(unsigned(cdiv(N, Gm::NW)), unsigned(w.tiles));
     cudaError_t e = launch_pdl_if(pdl, tc::gemm_tc_kernel<FMT, TOKL, MN>, grid, dim3(Gm::NUM_THREADS),
                                   size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
-                                  (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y);
+                                  (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y, tq, tsc, tbi, sc_tma);
     return cuda_status(e);
 }
 
