@@ -104,10 +104,10 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group);
  *            entry are ignored and are garbage afterwards. Calls that share a workspace
  *            must be ordered on one stream.
  * Scale range: the tensor-core path (M > 8, or PATH_GEMM) holds d_w * (q - 8) exactly as
- * two fp16 values, which requires |d_w| <= 8188 (weights of magnitude up to ~65500). A
- * larger, infinite or NaN scale makes the kernel set W4A8_ERR_RANGE in the device status
- * word (w4a8_last_device_error) and the affected outputs are not reliable. The GEMV path
- * (M <= 8, or PATH_GEMV) has no such limit.
+ * two fp16 values formed by one fused multiply-add each, which requires |d_w| < 2728
+ * (weights of magnitude up to ~21800). A larger, infinite or NaN scale makes the kernel
+ * set W4A8_ERR_RANGE in the device status word (w4a8_last_device_error) and the affected
+ * outputs are not reliable. The GEMV path (M <= 8, or PATH_GEMV) has no such limit.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, WORKSPACE, CUDA.
  */
 w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype,
@@ -137,7 +137,7 @@ w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int 
  * y = x . W^T with W affine 4-bit (from w4a8_pack_affine) and x quantised to Q8_0 in the
  * call. The contraction runs on the original codes: per activation block b inside
  * group g, y += d_x * (s_g * sum q*q_x + b_g * sum q_x). Tolerance as w4a8_gemm.
- * Scale range of the tensor-core path: s = 0 or 2^-17 <= |s| <= 8188 (s * (q - 8) is then
+ * Scale range of the tensor-core path: s = 0 or 2^-17 <= |s| <= 2720 (s * (q - 8) is then
  * exact in fp16); other scales set W4A8_ERR_RANGE as in w4a8_gemm.
  * Arguments and errors as w4a8_gemm, plus `group` (64 or 128).
  */
