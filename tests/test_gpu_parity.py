@@ -173,7 +173,7 @@ def test_gemm_is_deterministic_and_ignores_workspace_contents():
 
 
 def test_scale_outside_tensor_core_range_is_reported():
-    """A Q4_0 block scale above 8188 cannot be held exactly by the tensor-core path's fp16
+    """A Q4_0 block scale above 2720 cannot be held exactly by the tensor-core path's fp16
     weight operand: that path reports W4A8_ERR_RANGE through the device status word, while
     the GEMV path (no such limit) stays within tolerance."""
     M, N, K = 40, 128, 256
