@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                    const float* __restrict__ zb, const uint8_t* __restrict__ wq,
                    const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
                    float* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int sc_tma) {
+                   const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int sc_tma,
+                   int bsplit, float* __restrict__ ypart) {
     using Gm = Geo<FMT, TOKL, MN>;
     constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NW = Gm::NW, CW = Gm::CW;
     constexpr int W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK, DX_BLK = Gm::DX_BLK;
@@ -199,7 +200,13 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = K >> 5;
-    const int nstages = (B + S - 1) / S;
+    // Split of K over blockIdx.z: this CTA contracts blocks [kb0, kb0 + Bl) (bsplit is a
+    // multiple of 8) and, when K is split, writes its partial sums to ypart[z] for the
+    // reduction kernel instead of y.
+    const int kb0 = blockIdx.z * bsplit;
+    const int Bl = min(B, kb0 + bsplit) - kb0;
+    const int nstages = (Bl + S - 1) / S;
+    float* __restrict__ yo = (gridDim.z > 1) ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : y;
     const int n0 = blockIdx.x * NW;
     const int t = blockIdx.y;
     const int bpg = (FMT == 1) ? (group >> 5) : 1;  // blocks per affine group
@@ -246,10 +253,10 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
         auto load_sc = [&](int st, uint16_t (&sv)[S], uint16_t (&bv)[S]) {
 #pragma unroll
             for (int k = 0; k < S; ++k) {
-                const int b = st * S + k;
+                const int b = kb0 + st * S + k;
                 sv[k] = 0;
                 bv[k] = 0;
-                if (!sc_tma && row_ok && b < B) {
+                if (!sc_tma && row_ok && st * S + k < Bl) {
                     if (FMT == 0) {
                         sv[k] = ld_nc_u16(wscale + int64_t(n) * B + b);
                     } else {
@@ -268,13 +275,14 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
             // slot from the epilogue before fetching them).
             if (!bounded_wait_warp(bar(&ctrl->raw[slot]), (st / NS) & 1, abort)) break;
             uint8_t* sp = stage_ptr(slot);
-            const int e0 = (FMT == 0) ? (st * S) & ~7 : ((st * S) / bpg) & ~7;  // first scale of the TMA box
+            const int sb0 = kb0 + st * S;  // first block of the stage
+            const int e0 = (FMT == 0) ? sb0 & ~7 : (sb0 / bpg) & ~7;  // first scale of the TMA box
 #pragma unroll
             for (int k = 0; k < S; ++k) {
-                const int b = st * S + k;
+                const int b = sb0 + k;
                 uint4 wv = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);  // codes 8: zero
                 uint32_t sb = 0, bb = 0;
-                if (b < B) {
+                if (st * S + k < Bl) {
                     wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + k * NW * 16 + p * 16);
                     if (sc_tma) {
                         const int e = (FMT == 0) ? b : b / bpg;
@@ -350,8 +358,8 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
         for (int st = 0; st < nstages; ++st) {
             const int slot = st % NS;
             if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) break;
-            const int b0 = st * S;
-            const int nb = min(S, B - b0);
+            const int b0 = kb0 + st * S;
+            const int nb = min(S, kb0 + Bl - b0);
             if (leader) {
                 int nz = 0;  // affine: group ends in this stage (each brings its Z row)
                 if (FMT == 1)
@@ -401,7 +409,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
             if (!bounded_wait_warp(bar(&ctrl->full[slot]), (st / NS) & 1, abort)) break;
             if (!bounded_wait_warp(bar(&ctrl->tempty[g]), ((st / NG) & 1) ^ 1, abort)) break;
             tc_fence_after();
-            const int nb = min(S, B - st * S);
+            const int nb = min(S, Bl - st * S);
             if (leader) {
                 for (int k = 0; k < nb; ++k) {
                     const uint32_t w_addr = smem0 + uint32_t(slot * STAGE_BYTES + k * W_BLK);
@@ -444,7 +452,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
         const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
         for (int st = 0; st < nstages; ++st) {
             const int slot = st % NS, g = st % NG;
-            const int nb = min(S, B - st * S);
+            const int nb = min(S, Bl - st * S);
             if (!bounded_wait_warp(bar(&ctrl->tfull[g]), (st / NG) & 1, abort)) break;
             tc_fence_after();
             const uint8_t* sp = stage_ptr(slot);
@@ -452,7 +460,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 if (k >= nb) break;
-                const int i = st * S + k;
+                const int i = kb0 + st * S + k;
                 const bool last = (k == nb - 1);
                 const float* dxk = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT;
                 const bool group_end = (FMT == 1) && (((i + 1) % bpg) == 0);
@@ -516,7 +524,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 const int m = t * TT + r;
                 const int nb = n0 + c0;
                 if (m < M) {
-                    float* yr = y + int64_t(m) * N + nb;
+                    float* yr = yo + int64_t(m) * N + nb;
                     if ((N & 3) == 0 && nb + CW <= N) {
 #pragma unroll
                         for (int j = 0; j < CW; j += 4)
@@ -533,7 +541,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < CW; ++j) {
                         const int m = t * TT + c0 + j;
-                        if (m < M) y[int64_t(m) * N + n] = acc[j];
+                        if (m < M) yo[int64_t(m) * N + n] = acc[j];
                     }
                 }
             }
@@ -545,6 +553,24 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
     if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Gm::TMEM_COLS);
+    }
+}
+
+// Sum of the K-split partial outputs in split order: y = part[0] + part[1] + ... (the
+// same order on every call, so results do not depend on scheduling). n4 = M*N/4.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ part, int ks, int64_t n4,
+                                                             float4* __restrict__ y) {
+    pdl_wait_primary();  // the partials are written by the preceding GEMM
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
+        float4 a = part[i];
+        for (int z = 1; z < ks; ++z) {
+            const float4 b = part[int64_t(z) * n4 + i];
+            a.x = __fadd_rn(a.x, b.x);
+            a.y = __fadd_rn(a.y, b.y);
+            a.z = __fadd_rn(a.z, b.z);
+            a.w = __fadd_rn(a.w, b.w);
+        }
+        y[i] = a;
     }
 }
 

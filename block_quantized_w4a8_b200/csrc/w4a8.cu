@@ -237,6 +237,43 @@ w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_d
     return cuda_status(e);
 }
 
+// ------------------------------------------------------------------ split of K
+// When the output tiles do not fill the SMs, K is split over blockIdx.z (at least 16
+// blocks per split, splits of a multiple of 8 blocks) and a reduction kernel sums the
+// partial outputs, kept in the workspace after the operand region, in split order.
+struct KSplit {
+    int ks;      // splits actually used
+    int bsplit;  // blocks per split
+};
+inline int64_t tc_tiles(int M, int N) {
+    const int tt = tc_token_tile(M);
+    return cdiv(N, 128) * cdiv(M, tt);
+}
+inline size_t partial_bytes(int ks, int M, int N) { return ks > 1 ? align256(size_t(ks) * M * N * 4) : 0; }
+int tc_split_pref(int M, int N, int K) {
+    if ((int64_t(M) * N) % 4 != 0) return 1;  // the reduction works on float4
+    const int64_t tiles = tc_tiles(M, N);
+    const int sms = sm_count();
+    if (tiles >= sms) return 1;
+    int ks = int(sms / tiles);
+    const int by_k = (K / 32) / 16;
+    if (ks > by_k) ks = by_k;
+    return ks < 1 ? 1 : ks;
+}
+// The split for this call: the preferred one, reduced until its partials fit `work_bytes`.
+KSplit tc_split(int M, int N, int K, size_t base_bytes, size_t work_bytes) {
+    const int B = K / 32;
+    int ks = tc_split_pref(M, N, K);
+    while (ks > 1 && base_bytes + partial_bytes(ks, M, N) > work_bytes) --ks;
+    KSplit sp{1, B};
+    if (ks > 1) {
+        sp.bsplit = int((cdiv(B, ks) + 7) / 8 * 8);
+        sp.ks = int(cdiv(B, sp.bsplit));
+        if (sp.ks < 2) sp = KSplit{1, B};
+    }
+    return sp;
+}
+
 // cuTensorMapEncodeTiled, resolved once through the runtime (no link against the driver
 // library).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -271,7 +308,7 @@ bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e
 
 template <int FMT, bool TOKL, int MN>
 w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                           const uint16_t* wb, float* y, bool pdl, cudaStream_t stream) {
+                           const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
     using Gm = tc::Geo<FMT, TOKL, MN>;
     static bool configured[64] = {false};
     int dev = 0;
@@ -302,10 +339,19 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
                                    uint64_t(E) * 2, 8, Gm::NW))
             return W4A8_ERR_CUDA;
     }
-    const dim3 grid(unsigned(cdiv(N, Gm::NW)), unsigned(w.tiles));
+    const KSplit sp = tc_split(M, N, K, w.bytes, work_bytes);
+    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(w.tok) + w.bytes);
+    const dim3 grid(unsigned(cdiv(N, Gm::NW)), unsigned(w.tiles), unsigned(sp.ks));
     cudaError_t e = launch_pdl_if(pdl, tc::gemm_tc_kernel<FMT, TOKL, MN>, grid, dim3(Gm::NUM_THREADS),
                                   size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
-                                  (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y, tq, tsc, tbi, sc_tma);
+                                  (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y, tq, tsc, tbi, sc_tma,
+                                  sp.bsplit, part);
+    if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
+    const int64_t n4 = int64_t(M) * N / 4;
+    int64_t rb = cdiv(n4, 256);
+    if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
+    e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, (const float4*)part, sp.ks, n4,
+                   reinterpret_cast<float4*>(y));
     return cuda_status(e);
 }
 
@@ -313,13 +359,21 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
 // of 128 tokens put them on the TMEM lanes with 128 weight rows per tile.
 template <int FMT>
 w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                        const uint16_t* wb, float* y, bool pdl, cudaStream_t stream) {
+                        const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
     switch (w.tt) {
-        case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
-        case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
-        case 64: return launch_gemm_tc<FMT, false, 64>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
-        default: return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, pdl, stream);
+        case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+        case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+        case 64: return launch_gemm_tc<FMT, false, 64>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+        default: return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
     }
+}
+
+// Smallest workspace any call of this shape accepts (no split of K); a larger one, up to
+// w4a8_workspace_bytes, lets the tensor-core path split K.
+size_t min_workspace_bytes(int M, int K, int group) {
+    const size_t a = gemv_ws(nullptr, M, K).bytes;
+    const size_t b = tc_ws(nullptr, M, K, group).bytes;
+    return a > b ? a : b;
 }
 
 w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
@@ -337,7 +391,7 @@ w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, c
         return W4A8_ERR_MISALIGNED;
     if (!work) return W4A8_ERR_WORKSPACE;
     if (!aligned16(work)) return W4A8_ERR_MISALIGNED;
-    if (work_bytes < w4a8_workspace_bytes(M, N, K, affine ? group : 0)) return W4A8_ERR_WORKSPACE;
+    if (work_bytes < min_workspace_bytes(M, K, affine ? group : 0)) return W4A8_ERR_WORKSPACE;
     return W4A8_OK;
 }
 
@@ -360,10 +414,10 @@ w4a8_status prepare_impl(int M, int K, int group, const void* x, w4a8_dtype dt, 
 // tail (programmatic dependent launch); otherwise it starts after all prior work.
 template <int FMT>
 w4a8_status contract_impl(int M, int N, int K, int group, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb,
-                          float* y, void* work, bool gemv, bool after_quant, cudaStream_t stream) {
+                          float* y, void* work, size_t work_bytes, bool gemv, bool after_quant, cudaStream_t stream) {
     if (gemv) return run_gemv<FMT>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, stream);
     return run_gemm_tc<FMT>(M, N, K, group, tc_ws(work, M, K, FMT == 1 ? group : 0), wq, ws, wb, y, after_quant,
-                            stream);
+                            work_bytes, stream);
 }
 
 template <int FMT>
@@ -376,7 +430,7 @@ w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype 
     if (gemv && gemv_fused(M, K)) return run_gemv_fused<FMT>(M, N, K, group, x, dt, wq, ws, wb, y, stream);
     st = prepare_impl(M, K, FMT == 1 ? group : 0, x, dt, work, gemv, stream);
     if (st != W4A8_OK) return st;
-    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, gemv, true, stream);
+    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, work_bytes, gemv, true, stream);
 }
 
 }  // namespace
@@ -410,7 +464,7 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group) {
     if (group != 0 && (group != 64 && group != 128)) return 0;
     if (group != 0 && (K % group) != 0) return 0;
     const size_t a = gemv_ws(nullptr, M, K).bytes;
-    const size_t b = tc_ws(nullptr, M, K, group).bytes;
+    const size_t b = tc_ws(nullptr, M, K, group).bytes + partial_bytes(tc_split_pref(M, N, K), M, N);
     return a > b ? a : b;
 }
 
@@ -470,8 +524,8 @@ w4a8_status w4a8_gemm_prepared(int M, int N, int K, const uint8_t* qs, const uin
                                const void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
     w4a8_status st = check_gemm_args(M, N, K, qs, W4A8_F32, qs, d_fp16, nullptr, false, 0, y, ws, ws_bytes, path);
     if (st != W4A8_OK) return st;
-    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, const_cast<void*>(ws), use_gemv(M, path), false,
-                           stream);
+    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, const_cast<void*>(ws), ws_bytes, use_gemv(M, path),
+                            false, stream);
 }
 
 w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint32_t* q, const uint16_t* scale_bf16,
@@ -481,8 +535,8 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
     w4a8_status st =
         check_gemm_args(M, N, K, wq, W4A8_F32, wq, scale_bf16, bias_bf16, true, group, y, ws, ws_bytes, path);
     if (st != W4A8_OK) return st;
-    return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, const_cast<void*>(ws), use_gemv(M, path),
-                            false, stream);
+    return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, const_cast<void*>(ws), ws_bytes,
+                            use_gemv(M, path), false, stream);
 }
 
 // Scratch of w4a8_gemm_noalloc. In host code this name is only a stand-in for the
@@ -492,7 +546,7 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_
 w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
                               const uint16_t* d_fp16, float* y, cudaStream_t stream) {
     static void* scratch_ptr[64] = {nullptr};
-    const size_t need = w4a8_workspace_bytes(M, N, K, 0);
+    const size_t need = (dims_ok(M, N) && dims_ok(K, 1) && K % 32 == 0) ? min_workspace_bytes(M, K, 0) : 0;
     if (need == 0) return W4A8_ERR_INVALID_ARG;
     if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
     int dev = 0;

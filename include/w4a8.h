@@ -87,9 +87,13 @@ w4a8_status w4a8_quant_act_q8_0(const void* x, w4a8_dtype dtype, int M, int K,
                                 int8_t* qx, float* dx, int32_t* sx, cudaStream_t stream);
 
 /*
- * Size in bytes of the workspace w4a8_gemm / w4a8_gemm_affine need for this shape
- * (group = 0 for Q4_0, else the affine group size). Covers every path, so one
- * allocation serves AUTO and both forced paths. Returns 0 for invalid sizes.
+ * Size in bytes of the workspace w4a8_gemm / w4a8_gemm_affine use for this shape
+ * (group = 0 for Q4_0, else the affine group size) on the current device. Covers every
+ * path, so one allocation serves AUTO and both forced paths. It includes room for the
+ * tensor-core path to split K when the output tiles do not fill the SMs (partial sums,
+ * reduced in a fixed order). A smaller workspace is accepted down to the unsplit minimum
+ * (the split then shrinks to what fits, which can change the last bits of the result);
+ * below that minimum the calls return W4A8_ERR_WORKSPACE. Returns 0 for invalid sizes.
  */
 size_t w4a8_workspace_bytes(int M, int N, int K, int group);
 
@@ -99,10 +103,10 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group);
  * D = sum_{j<32} (q_w - 8) * q_x computed exactly. The sum over blocks is taken in f32;
  * each output is within 1e-5 * sum_b |term_b| of the exact value.
  * x        : M x K, f32 or bf16.       qs, d_fp16 : as produced by w4a8_pack_q4_0.
- * y        : out, M x N f32.           ws, ws_bytes : scratch of at least
- *            w4a8_workspace_bytes(M, N, K, 0) bytes, owned by the caller; contents on
- *            entry are ignored and are garbage afterwards. Calls that share a workspace
- *            must be ordered on one stream.
+ * y        : out, M x N f32.           ws, ws_bytes : scratch of w4a8_workspace_bytes(M, N,
+ *            K, 0) bytes (or at least the unsplit minimum, see there), owned by the
+ *            caller; contents on entry are ignored and are garbage afterwards. Calls
+ *            that share a workspace must be ordered on one stream.
  * Scale range: the tensor-core path (M > 8, or PATH_GEMM) holds d_w * (q - 8) exactly as
  * two fp16 values formed by one fused multiply-add each, which requires |d_w| < 2728
  * (weights of magnitude up to ~21800). A larger, infinite or NaN scale makes the kernel
@@ -187,8 +191,9 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
  * exits). The library itself never calls cudaMalloc or cudaFree here.
  *  - The first call on each device looks up that array's device address (with that device
  *    current), so that first call should come before any stream capture.
- *  - Shapes whose workspace (w4a8_workspace_bytes(M, N, K, 0)) exceeds the array are
- *    rejected with W4A8_ERR_WORKSPACE; nothing is launched.
+ *  - Shapes whose minimum workspace (see w4a8_workspace_bytes) exceeds the array are
+ *    rejected with W4A8_ERR_WORKSPACE; nothing is launched. Within the array the
+ *    tensor-core path splits K only as far as its partial sums fit.
  *  - Every call on a device shares the one array and the array keeps whatever the last call
  *    left in it (the kernels overwrite what they read, nothing needs to start at zero).
  *    Calls whose work overlaps on the GPU (different streams, or several host threads
