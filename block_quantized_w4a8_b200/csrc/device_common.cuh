@@ -46,28 +46,49 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 // phase completes or the hint runs out, instead of spinning on shared memory.
 constexpr uint32_t kTryWaitHintNs = 1000000u;
 
+// CLUSTER: acquire at cluster scope, for barriers that other CTAs of the cluster arrive on.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kTryWaitHintNs)
-        : "memory");
+    if (CLUSTER)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(kTryWaitHintNs)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(kTryWaitHintNs)
+            : "memory");
     return ok != 0;
 }
 // Probe without a suspend hint: on a completed phase it returns in a fraction of the
 // time of the hinted form, so every wait checks this way first.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_try_wait_nohint(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+    if (CLUSTER)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 
@@ -97,10 +118,11 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, vola
 // Warp-wide wait: every lane probes the barrier and a vote makes the outcome uniform
 // (phase completion is monotonic, so a lane that saw it keeps seeing it), so the warp
 // never diverges. Same limits as bounded_wait. All 32 lanes must call it.
+template <bool CLUSTER = false>
 __device__ __noinline__ bool bounded_wait_warp_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
     const unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        if (__all_sync(0xffffffffu, mbar_try_wait<CLUSTER>(bar, parity))) return true;
         if ((it & 15u) == 0u) {
             uint32_t stop = *abort;
             if (!stop && global_timer_ns() - t0 > kWaitLimitNs) stop = 2u;
@@ -115,9 +137,10 @@ __device__ __noinline__ bool bounded_wait_warp_slow(uint32_t bar, uint32_t parit
         }
     }
 }
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool bounded_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
-    if (__all_sync(0xffffffffu, mbar_try_wait_nohint(bar, parity))) return true;
-    return bounded_wait_warp_slow(bar, parity, abort);
+    if (__all_sync(0xffffffffu, mbar_try_wait_nohint<CLUSTER>(bar, parity))) return true;
+    return bounded_wait_warp_slow<CLUSTER>(bar, parity, abort);
 }
 
 // Named hardware barrier over `nthreads` threads (whole warps); waiting warps issue
@@ -212,6 +235,18 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
+// The same for a CTA pair (cta_group::2): one warp of each CTA of the pair executes it,
+// and the pair's tensor memory is allocated at the same columns in both CTAs.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -230,6 +265,57 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// CTA-pair MMA, issued by one thread of the even CTA: M = 256 rows of A, 128 from each
+// CTA's shared memory at the descriptor's address; B's N columns split in halves, the
+// first half staged by the even CTA, the second by the odd one; each CTA's tensor memory
+// receives its own 128 rows of D (all N columns).
+__device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on the barrier at offset `bar` in each CTA of `cta_mask` when the pair MMAs
+// this thread issued so far are done.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// ------------------------------------------------------------------ clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Barrier over all threads of all CTAs of the cluster (release/acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// Arrive on a barrier of another CTA of the cluster (address from mapa_shared), releasing
+// this thread's earlier memory operations at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+// Remote arrive with the default (CTA-scope) release: enough to signal that tensor-memory
+// reads ordered before it by tcgen05.fence::before_thread_sync are done. The cluster-
+// scope release costs several hundred cycles more per arrival.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 
 // Shared-memory matrix descriptor for a K-major operand without swizzle: core matrices

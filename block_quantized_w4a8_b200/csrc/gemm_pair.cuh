@@ -1,0 +1,409 @@
+// Tensor-core path on CTA pairs (cta_group::2) for token tiles on the TMEM lanes.
+//
+// Same arithmetic as the token-lane instantiation of gemm_tc_kernel (exact fp16 weight
+// operand with the weight scale folded in, one f32 FMA per output and block for the
+// activation scale; tract PR #2432, "The kernel": a separate rescale per 32-block), but
+// two CTAs of a cluster share each weight tile: the pair's MMA is 256 tokens x 128 weight
+// rows, the even CTA holding tokens 0..127 of the pair and weight rows 0..63, the odd CTA
+// tokens 128..255 and weight rows 64..127. Each CTA therefore expands and stores only half
+// of the weight rows for the same MMA work, which halves the shared-memory stores that
+// bound the single-CTA kernel (the expanded operand is 128 B per row and block), while the
+// epilogue is unchanged: each CTA's tensor memory holds its 128 tokens x all 128 rows.
+//
+// Roles per CTA (448 threads): 8 epilogue warps, 4 producer warps (one thread per (row of
+// the CTA's half, block of the stage), two stages at a time), one MMA warp, one bulk-copy
+// warp. Only the even
+// CTA's MMA warp issues MMAs; the odd CTA's MMA warp forwards its stage-ready signal to the
+// even CTA (one remote arrive per stage). The even CTA's MMA warp waits for its own stage,
+// the forwarded one and both CTAs' epilogues (TMEM groups), issues the stage's MMAs and
+// one commit that arrives on both CTAs' barriers. All waits are bounded as in the
+// single-CTA kernel; both CTAs meet at a cluster barrier before the pair's tensor memory
+// is freed, so neither exits while the other or the tensor core may still touch it.
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace w4a8 {
+namespace tc {
+
+template <int FMT>
+struct PairGeo {
+    static constexpr int TT = 128;                  // tokens per CTA (256 per pair)
+    static constexpr int NWT = 128;                 // weight rows per pair tile (the MMA's N)
+    static constexpr int NWH = NWT / 2;             // weight rows each CTA expands and stages
+    static constexpr int MN = NWT;                  // TMEM columns per accumulator tile
+    static constexpr int WP = (FMT == 0) ? 2 : 1;   // weight operand parts (hi, lo)
+    static constexpr int W_PART = NWH * 64;
+    static constexpr int W_BLK = W_PART * WP;
+    static constexpr int T_BLK = TT * 64;
+    static constexpr int DX_BLK = TT * 4;
+    static constexpr int S = 2;                     // quant blocks per stage (one commit)
+    static constexpr int OFF_T = S * W_BLK;
+    static constexpr int OFF_DX = OFF_T + S * T_BLK;
+    static constexpr int OFF_C = align_up(OFF_DX + S * DX_BLK, 128);            // affine: b + 8s, all 128 rows
+    static constexpr int OFF_Z = OFF_C + (FMT == 1 ? S * NWT * 4 : 0);          // affine: Z per token
+    static constexpr int OFF_RAW = align_up(OFF_Z + (FMT == 1 ? S * TT * 4 : 0), 128);  // codes, own half
+    static constexpr int OFF_RSC = OFF_RAW + S * NWH * 16;                      // scales, all 128 rows
+    static constexpr int OFF_RBI = OFF_RSC + NWT * 16;                          // affine biases
+    static constexpr int STAGE_BYTES = align_up(OFF_RBI + (FMT == 1 ? NWT * 16 : 0), 1024);
+    static constexpr int NS = cmin(8, (SMEM_LIMIT - CTRL_BYTES - 1024) / STAGE_BYTES);
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;
+    static constexpr int NBUF = 512 / MN;           // accumulator tiles (one per block)
+    static constexpr int NG = NBUF / S;             // TMEM groups: stage st uses group st % NG
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int CW = 64;                   // columns per epilogue warp
+    static constexpr int EPI_WARPS = 4 * MN / CW;
+    static constexpr int PROD_WARPS = NWH * S / 32;
+    static constexpr int PROD_WARP0 = EPI_WARPS;
+    static constexpr int MMA_WARP = PROD_WARP0 + PROD_WARPS;
+    static constexpr int COPY_WARP = MMA_WARP + 1;
+    static constexpr int NUM_THREADS = (COPY_WARP + 1) * 32;
+    static constexpr int LD_COLS = 32;              // TMEM columns per load (registers: 64 accumulators + 32)
+    static constexpr uint32_t IDESC = idesc_f16_f32(256, NWT);
+    static_assert(NS >= 3 && NS <= 8, "pipeline depth");
+    static_assert(NG == 2 && NBUF % S == 0, "TMEM groups");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
+    static_assert(OFF_T % 128 == 0 && OFF_DX % 16 == 0 && OFF_Z % 16 == 0 && OFF_RSC % 16 == 0, "alignment");
+};
+
+struct PairCtrl {
+    unsigned long long raw[MAX_NS];     // TMA of the packed weights (1 arrival + bytes)
+    unsigned long long full[MAX_NS];    // producer warps + bulk copies (1 arrival + bytes)
+    unsigned long long empty[MAX_NS];   // one arrival per epilogue warp of this CTA
+    unsigned long long pfull[MAX_NS];   // even CTA: the odd CTA's stage is ready (1 remote arrival)
+    unsigned long long tfull[MAX_NG];   // pair commit, once per stage, on both CTAs
+    unsigned long long tempty[MAX_NG];  // even CTA: one arrival per epilogue warp of both CTAs
+    unsigned long long drain;           // final pair commit, on both CTAs
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+static_assert(sizeof(PairCtrl) <= CTRL_BYTES, "control block");
+
+// Grid: x = token tile (pairs of consecutive tiles form a cluster), y = 128-row weight
+// tile, z = split of K. The scale (and affine bias) tensor maps have boxes of 128 rows x 8
+// entries, the code map boxes of 64 rows x 16 bytes; both require the rows' pitch to be a
+// multiple of 16 bytes, which the host checks before choosing this kernel.
+template <int FMT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_THREADS, 1)
+    gemm_pair_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dxs,
+                     const float* __restrict__ zb, float* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int bsplit,
+                     float* __restrict__ ypart) {
+    using Gm = PairGeo<FMT>;
+    constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NWT = Gm::NWT, NWH = Gm::NWH;
+    constexpr int MN = Gm::MN, CW = Gm::CW, W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK;
+    constexpr int DX_BLK = Gm::DX_BLK, OFF_T = Gm::OFF_T, OFF_DX = Gm::OFF_DX, OFF_C = Gm::OFF_C;
+    constexpr int OFF_Z = Gm::OFF_Z, OFF_RAW = Gm::OFF_RAW, OFF_RSC = Gm::OFF_RSC, OFF_RBI = Gm::OFF_RBI;
+    constexpr int STAGE_BYTES = Gm::STAGE_BYTES, EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0;
+    constexpr int PROD_WARPS = Gm::PROD_WARPS, MMA_WARP = Gm::MMA_WARP, COPY_WARP = Gm::COPY_WARP;
+    constexpr int LD_COLS = Gm::LD_COLS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PairCtrl* ctrl = reinterpret_cast<PairCtrl*>(smem + NS * STAGE_BYTES);
+    volatile uint32_t* abort = &ctrl->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
+    const int B = K >> 5;
+    const int kb0 = blockIdx.z * bsplit;  // this pair contracts blocks [kb0, kb0 + Bl)
+    const int Bl = min(B, kb0 + bsplit) - kb0;
+    const int nstages = (Bl + S - 1) / S;
+    float* __restrict__ yo = (gridDim.z > 1) ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : y;
+    const int t = blockIdx.x;                // token tile
+    const int n0 = blockIdx.y * NWT;         // the pair's weight rows
+    const int nh0 = n0 + int(rank) * NWH;    // the rows this CTA stages
+    const int bpg = (FMT == 1) ? (group >> 5) : 1;
+    const int G = (FMT == 1) ? K / group : 0;
+
+    auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
+    auto bar = [](unsigned long long* p) { return smem_addr(p); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(&ctrl->raw[s]), 1);
+            mbar_init(bar(&ctrl->full[s]), PROD_WARPS + 1);
+            mbar_init(bar(&ctrl->empty[s]), EPI_WARPS);
+            mbar_init(bar(&ctrl->pfull[s]), 1);
+        }
+        for (int j = 0; j < NG; ++j) {
+            mbar_init(bar(&ctrl->tfull[j]), 1);
+            mbar_init(bar(&ctrl->tempty[j]), 2 * EPI_WARPS);
+        }
+        mbar_init(bar(&ctrl->drain), 1);
+        ctrl->abort = 0;
+        mbar_init_fence();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc_pair(smem_addr(&ctrl->tmem_base), Gm::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem_base = ctrl->tmem_base;
+    pdl_launch_dependents();
+
+    if (warp >= PROD_WARP0 && warp < MMA_WARP) {
+        // ------------------------------------------------------------ producer
+        // Two stages per iteration: their loads, expansions and stores interleave, and one
+        // proxy fence covers both (a single row-block per thread leaves the warp waiting on
+        // one dependent chain at a time).
+        const int tid = threadIdx.x - PROD_WARP0 * 32;
+        const int p = tid % NWH;   // weight row within this CTA's half
+        const int kq = tid / NWH;  // block of the stage this thread expands
+        bool range_bad = false;
+        auto expand = [&](int st) {
+            uint8_t* sp = stage_ptr(st % NS);
+            const int sb0 = kb0 + st * S;
+            const int e0 = (FMT == 0) ? sb0 & ~7 : (sb0 / bpg) & ~7;  // first scale of the TMA box
+            if (st * S + kq < Bl) {
+                const int b = sb0 + kq;
+                const int e = (FMT == 0) ? b : b / bpg;
+                const uint4 wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
+                const uint32_t sb =
+                    reinterpret_cast<const uint16_t*>(sp + OFF_RSC + (int(rank) * NWH + p) * 16)[e - e0];
+                const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+                uint8_t* dst = sp + kq * W_BLK + (p >> 3) * 512 + (p & 7) * 16;
+                if (FMT == 0) {
+                    range_bad |= (sb & 0x7FF8u) > 0x6950u;  // d_hi > 2720 (24 d_hi > 65504), inf or nan
+                    const __half dh = __ushort_as_half(uint16_t(sb & 0xFFF8u));
+                    const __half dl = __hsub(__ushort_as_half(uint16_t(sb)), dh);  // exact
+                    const uint32_t h2 = pair_of(__hmul(dh, __float2half(2.0f)));
+                    const uint32_t h24 = pair_of(__hmul(dh, __float2half(-24.0f)));
+                    const uint32_t l2 = pair_of(__hmul(dl, __float2half(2.0f)));
+                    const uint32_t l24 = pair_of(__hmul(dl, __float2half(-24.0f)));
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[4];
+                        codes_raw(w[c], r);
+                        *reinterpret_cast<uint4*>(dst + c * 128) =
+                            make_uint4(scaled_codes(r[0], h2, h24), scaled_codes(r[1], h2, h24),
+                                       scaled_codes(r[2], h2, h24), scaled_codes(r[3], h2, h24));
+                        *reinterpret_cast<uint4*>(dst + W_PART + c * 128) =
+                            make_uint4(scaled_codes(r[0], l2, l24), scaled_codes(r[1], l2, l24),
+                                       scaled_codes(r[2], l2, l24), scaled_codes(r[3], l2, l24));
+                    }
+                } else {
+                    const float sf = __bfloat162float(__ushort_as_bfloat16(uint16_t(sb)));
+                    const float af = fabsf(sf);
+                    range_bad |= !(af <= 2720.0f) || (af != 0.0f && af < 7.62939453125e-06f);  // 2^-17
+                    const __half sh = __float2half_rn(sf);  // exact in range
+                    const uint32_t s2 = pair_of(__hmul(sh, __float2half(2.0f)));
+                    const uint32_t s24 = pair_of(__hmul(sh, __float2half(-24.0f)));
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[4];
+                        codes_raw(w[c], r);
+                        *reinterpret_cast<uint4*>(dst + c * 128) =
+                            make_uint4(scaled_codes(r[0], s2, s24), scaled_codes(r[1], s2, s24),
+                                       scaled_codes(r[2], s2, s24), scaled_codes(r[3], s2, s24));
+                    }
+                }
+            }
+            if (FMT == 1) {
+                // Bias factors b + 8s of all 128 rows of the pair tile (the epilogue of each
+                // CTA covers all of them): thread tid takes row tid for each group ending in
+                // the stage.
+#pragma unroll
+                for (int k = 0; k < S; ++k) {
+                    const int b = sb0 + k;
+                    if (st * S + k < Bl && ((b + 1) % bpg) == 0) {
+                        const int e = b / bpg;
+                        const uint16_t sv = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + tid * 16)[e - e0];
+                        const uint16_t bv = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + tid * 16)[e - e0];
+                        const float sf = __bfloat162float(__ushort_as_bfloat16(sv));
+                        const float bf = __bfloat162float(__ushort_as_bfloat16(bv));
+                        reinterpret_cast<float*>(sp + OFF_C)[k * NWT + tid] = __fadd_rn(bf, __fmul_rn(8.0f, sf));
+                    }
+                }
+            }
+        };
+        for (int st = 0; st < nstages; st += 2) {
+            const bool two = st + 1 < nstages;  // warp-uniform
+            if (!bounded_wait_warp(bar(&ctrl->raw[st % NS]), (st / NS) & 1, abort)) break;
+            if (two && !bounded_wait_warp(bar(&ctrl->raw[(st + 1) % NS]), ((st + 1) / NS) & 1, abort)) break;
+            expand(st);
+            if (two) expand(st + 1);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(&ctrl->full[st % NS]));
+                if (two) mbar_arrive(bar(&ctrl->full[(st + 1) % NS]));
+            }
+        }
+        if (range_bad) atomicOr(&g_device_status, kDevErrRange);
+    } else if (warp == COPY_WARP) {
+        // ------------------------------------------------------------ bulk copies
+        const bool leader = elect_one();
+        pdl_wait_primary();  // the token operands are written by the preceding kernel
+        int issued = 0;
+        for (int st = 0; st < nstages; ++st) {
+            const int slot = st % NS;
+            if (!bounded_wait_warp(bar(&ctrl->empty[slot]), ((st / NS) & 1) ^ 1, abort)) break;
+            const int b0 = kb0 + st * S;
+            const int nb = min(S, kb0 + Bl - b0);
+            if (leader) {
+                int nz = 0;  // affine: groups ending in this stage (each brings its Z row)
+                if (FMT == 1)
+                    for (int k = 0; k < nb; ++k) nz += ((b0 + k + 1) % bpg) == 0;
+                uint8_t* sp = stage_ptr(slot);
+                const uint32_t rb = bar(&ctrl->raw[slot]);
+                const int e0 = (FMT == 0) ? b0 & ~7 : (b0 / bpg) & ~7;
+                mbar_arrive_expect_tx(rb, uint32_t(nb * NWH * 16 + NWT * 16 * (FMT == 1 ? 2 : 1)));
+                for (int k = 0; k < nb; ++k)
+                    tma_load_2d(smem_addr(sp + OFF_RAW + k * NWH * 16), &tm_q, (b0 + k) * 16, nh0, rb);
+                tma_load_2d(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
+                if (FMT == 1) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
+                const uint32_t fb = bar(&ctrl->full[slot]);
+                mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK) + nz * TT * 4));
+                bulk_g2s(smem_addr(sp + OFF_T), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK,
+                         uint32_t(nb * T_BLK), fb);
+                bulk_g2s(smem_addr(sp + OFF_DX), dxs + (int64_t(t) * B + b0) * TT, uint32_t(nb * DX_BLK), fb);
+                if (FMT == 1) {
+                    for (int k = 0; k < nb; ++k)
+                        if (((b0 + k + 1) % bpg) == 0)
+                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + (b0 + k) / bpg) * TT,
+                                     TT * 4, fb);
+                }
+            }
+            __syncwarp();
+            issued = st + 1;
+        }
+        // Let every copy this warp issued land before the CTA can exit (capped waits, as in
+        // the single-CTA kernel).
+        for (int st = max(0, issued - NS); st < issued; ++st) {
+            drain_wait_warp(bar(&ctrl->raw[st % NS]), (st / NS) & 1, 200000ull);
+            drain_wait_warp(bar(&ctrl->full[st % NS]), (st / NS) & 1, 200000ull);
+        }
+    } else if (warp == MMA_WARP) {
+        const bool leader = elect_one();
+        uint32_t local_abort = 0;
+        if (rank == 0) {
+            // -------------------------------------------------------- MMA issue (even CTA)
+            const uint32_t smem0 = smem_addr(smem);
+            for (int st = 0; st < nstages; ++st) {
+                const int slot = st % NS, g = st % NG;
+                if (!bounded_wait_warp(bar(&ctrl->full[slot]), (st / NS) & 1, abort)) break;
+                if (!bounded_wait_warp<true>(bar(&ctrl->pfull[slot]), (st / NS) & 1, abort)) break;
+                if (!bounded_wait_warp<true>(bar(&ctrl->tempty[g]), ((st / NG) & 1) ^ 1, abort)) break;
+                tc_fence_after();
+                if (leader) {
+                    // Straight-line issue of all S blocks (blocks past the end of a short
+                    // last stage fill TMEM tiles that the epilogue never reads).
+#pragma unroll
+                    for (int k = 0; k < S; ++k) {
+                        const uint32_t w_addr = smem0 + uint32_t(slot * STAGE_BYTES + k * W_BLK);
+                        const uint32_t t_addr = smem0 + uint32_t(slot * STAGE_BYTES + OFF_T + k * T_BLK);
+                        const uint32_t d = tmem_base + uint32_t((g * S + k) * MN);
+#pragma unroll
+                        for (int part = 0; part < Gm::WP; ++part) {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint64_t wd = smem_desc_kmajor(w_addr + part * W_PART + h * 256, LBO, SBO);
+                                const uint64_t td = smem_desc_kmajor(t_addr + h * 256, LBO, SBO);
+                                tc_mma_f16_pair(d, td, wd, Gm::IDESC, (part | h) != 0);
+                            }
+                        }
+                    }
+                    tc_commit_pair(bar(&ctrl->tfull[g]), 3);
+                }
+                __syncwarp();
+            }
+            if (leader) tc_commit_pair(bar(&ctrl->drain), 3);
+        } else {
+            // -------------------------------------------------------- stage relay (odd CTA)
+            const uint32_t pfull0 = mapa_shared(bar(&ctrl->pfull[0]), 0);
+            for (int st = 0; st < nstages; ++st) {
+                const int slot = st % NS;
+                if (!bounded_wait_warp(bar(&ctrl->full[slot]), (st / NS) & 1, abort)) break;
+                if (leader) mbar_arrive_remote(pfull0 + uint32_t(slot) * 8u);
+                __syncwarp();
+            }
+        }
+        // Both CTAs: every MMA of the pair (and the arrivals of its commits) is done before
+        // the tensor memory and the shared memory are released.
+        __syncwarp();
+        bounded_wait_warp(bar(&ctrl->drain), 0, &local_abort);
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;           // TMEM lane quarter
+        const int c0 = (warp >> 2) * CW;  // first TMEM column of this warp
+        const int r = q * 32 + lane;      // this thread's TMEM lane: token within the tile
+        const uint32_t tempty0 = (rank == 0) ? bar(&ctrl->tempty[0]) : mapa_shared(bar(&ctrl->tempty[0]), 0);
+        float acc[CW];
+#pragma unroll
+        for (int j = 0; j < CW; ++j) acc[j] = 0.0f;
+        const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
+        for (int st = 0; st < nstages; ++st) {
+            const int slot = st % NS, g = st % NG;
+            const int nb = min(S, Bl - st * S);
+            if (!bounded_wait_warp(bar(&ctrl->tfull[g]), (st / NG) & 1, abort)) break;
+            tc_fence_after();
+            const uint8_t* sp = stage_ptr(slot);
+#pragma unroll
+            for (int k = 0; k < S; ++k) {
+                if (k >= nb) break;
+                const int i = kb0 + st * S + k;
+                const bool last = (k == nb - 1);
+                const float dxr = reinterpret_cast<const float*>(sp + OFF_DX)[k * TT + r];
+                const bool group_end = (FMT == 1) && (((i + 1) % bpg) == 0);
+#pragma unroll
+                for (int h0 = 0; h0 < CW; h0 += LD_COLS) {
+                    uint32_t pr[LD_COLS];
+                    tmem_load_cols(lane_base + uint32_t((g * S + k) * MN + c0 + h0), pr);
+                    if (last && h0 + LD_COLS == CW) {  // the group's tiles are all read: free it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (rank == 0)
+                                mbar_arrive(tempty0 + uint32_t(g) * 8u);
+                            else
+                                mbar_arrive_remote(tempty0 + uint32_t(g) * 8u);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < LD_COLS; ++j) acc[h0 + j] = fmaf(__uint_as_float(pr[j]), dxr, acc[h0 + j]);
+                }
+                if (group_end) {  // last block of a group: add (b + 8s) * Z
+                    const float* cs = reinterpret_cast<const float*>(sp + OFF_C) + k * NWT;
+                    const float z = reinterpret_cast<const float*>(sp + OFF_Z)[k * TT + r];
+#pragma unroll
+                    for (int j = 0; j < CW; j += 4) {
+                        const float4 cv = *reinterpret_cast<const float4*>(cs + c0 + j);
+                        acc[j] = fmaf(cv.x, z, acc[j]);
+                        acc[j + 1] = fmaf(cv.y, z, acc[j + 1]);
+                        acc[j + 2] = fmaf(cv.z, z, acc[j + 2]);
+                        acc[j + 3] = fmaf(cv.w, z, acc[j + 3]);
+                    }
+                }
+            }
+            __syncwarp();  // the values read from the stage were consumed above
+            if (lane == 0) mbar_arrive(bar(&ctrl->empty[slot]));
+        }
+        if (!*abort) {
+            const int m = t * TT + r;
+            const int nb = n0 + c0;
+            if (m < M) {
+                float* yr = yo + int64_t(m) * N + nb;
+                if ((N & 3) == 0 && nb + CW <= N) {
+#pragma unroll
+                    for (int j = 0; j < CW; j += 4)
+                        *reinterpret_cast<float4*>(yr + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < CW; ++j)
+                        if (nb + j < N) yr[j] = acc[j];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();  // neither CTA frees the pair's tensor memory or exits while the other may use it
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, Gm::TMEM_COLS);
+    }
+}
+
+}  // namespace tc
+}  // namespace w4a8

@@ -409,9 +409,12 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
             if (!bounded_wait_warp(bar(&ctrl->full[slot]), (st / NS) & 1, abort)) break;
             if (!bounded_wait_warp(bar(&ctrl->tempty[g]), ((st / NG) & 1) ^ 1, abort)) break;
             tc_fence_after();
-            const int nb = min(S, Bl - st * S);
             if (leader) {
-                for (int k = 0; k < nb; ++k) {
+                // Straight-line issue of all S blocks: a branch between two MMAs lets the
+                // issue stall until the earlier one completes. In a short last stage the
+                // blocks past the end fill TMEM tiles that the epilogue never reads.
+#pragma unroll
+                for (int k = 0; k < S; ++k) {
                     const uint32_t w_addr = smem0 + uint32_t(slot * STAGE_BYTES + k * W_BLK);
                     const uint32_t t_addr = smem0 + uint32_t(slot * STAGE_BYTES + OFF_T + k * T_BLK);
                     const uint32_t d = tmem_base + uint32_t((g * S + k) * MN);

@@ -10,6 +10,7 @@
 
 #include "device_common.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_pair.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
 
@@ -60,6 +61,13 @@ GemvWs gemv_ws(void* ws, int M, int K) {
 // MMA's N (16, 32 or 64 per tile, little padding); above, tiles of 128 tokens sit on the
 // TMEM lanes and the weight rows are the MMA's N.
 inline int tc_token_tile(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
+// Token tiles: 128-token tiles are processed by CTA pairs, so their count is rounded up
+// to even (the padding tile holds zero codes and scales).
+inline int tc_token_tiles(int M) {
+    const int tt = tc_token_tile(M);
+    const int n = int(cdiv(M, tt));
+    return (tt == 128) ? (n + 1) / 2 * 2 : n;
+}
 
 struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
     __half* tok;
@@ -73,7 +81,7 @@ TcWs tc_ws(void* ws, int M, int K, int group) {
     const int64_t B = K / 32;
     TcWs w{};
     w.tt = tc_token_tile(M);
-    w.tiles = int(cdiv(M, w.tt));
+    w.tiles = tc_token_tiles(M);
     const int64_t rows = int64_t(w.tiles) * w.tt;
     size_t off = 0;
     char* base = static_cast<char*>(ws);
@@ -245,10 +253,7 @@ struct KSplit {
     int ks;      // splits actually used
     int bsplit;  // blocks per split
 };
-inline int64_t tc_tiles(int M, int N) {
-    const int tt = tc_token_tile(M);
-    return cdiv(N, 128) * cdiv(M, tt);
-}
+inline int64_t tc_tiles(int M, int N) { return cdiv(N, 128) * tc_token_tiles(M); }
 inline size_t partial_bytes(int ks, int M, int N) { return ks > 1 ? align256(size_t(ks) * M * N * 4) : 0; }
 int tc_split_pref(int M, int N, int K) {
     if ((int64_t(M) * N) % 4 != 0) return 1;  // the reduction works on float4
@@ -355,8 +360,51 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
     return cuda_status(e);
 }
 
+// CTA-pair kernel for 128-token tiles: two consecutive token tiles share one 128-row
+// weight tile, each CTA staging half of its rows.
+template <int FMT>
+w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
+                             const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
+    using Gm = tc::PairGeo<FMT>;
+    static bool configured[64] = {false};
+    int dev = 0;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return cuda_status(ed);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_pair_kernel<FMT>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM_BYTES);
+        if (ea != cudaSuccess) return cuda_status(ea);
+        configured[dev] = true;
+    }
+    CUtensorMap tq, tsc, tbi;
+    memset(&tbi, 0, sizeof(tbi));
+    const int E = (FMT == 0) ? K / 32 : K / group;  // scales per row (a multiple of 8 here)
+    if (!encode_2d(&tq, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 16,
+                   Gm::NWH) ||
+        !encode_2d(&tsc, ws, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N), uint64_t(E) * 2, 8,
+                   Gm::NWT))
+        return W4A8_ERR_CUDA;
+    if (FMT == 1 && !encode_2d(&tbi, wb, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N),
+                               uint64_t(E) * 2, 8, Gm::NWT))
+        return W4A8_ERR_CUDA;
+    const KSplit sp = tc_split(M, N, K, w.bytes, work_bytes);
+    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(w.tok) + w.bytes);
+    const dim3 grid(unsigned(w.tiles), unsigned(cdiv(N, Gm::NWT)), unsigned(sp.ks));
+    cudaError_t e = launch_pdl_if(pdl, tc::gemm_pair_kernel<FMT>, grid, dim3(Gm::NUM_THREADS),
+                                  size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
+                                  (const float*)w.dxs, (const float*)w.z, y, tq, tsc, tbi, sp.bsplit, part);
+    if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
+    const int64_t n4 = int64_t(M) * N / 4;
+    int64_t rb = cdiv(n4, 256);
+    if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
+    e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, (const float4*)part, sp.ks, n4,
+                   reinterpret_cast<float4*>(y));
+    return cuda_status(e);
+}
+
 // Orientation by token tile: tiles of 16..64 tokens put the tokens on the MMA's N; tiles
-// of 128 tokens put them on the TMEM lanes with 128 weight rows per tile.
+// of 128 tokens put them on the TMEM lanes with 128 weight rows per tile, on CTA pairs
+// when the scale rows can be fetched by TMA (their pitch a multiple of 16 bytes).
 template <int FMT>
 w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
                         const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
@@ -364,7 +412,12 @@ w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uin
         case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
         case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
         case 64: return launch_gemm_tc<FMT, false, 64>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
-        default: return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+        default: {
+            const int E = (FMT == 0) ? K / 32 : K / group;
+            if ((E * 2) % 16 == 0)
+                return launch_gemm_pair<FMT>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+            return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+        }
     }
 }
 

@@ -54,11 +54,14 @@ def test_workspace_bytes(lib, M, N, K, group):
     B = K // 32
     gemv = _align(M * K) + _align(M * B * 4) + _align(M * B * 4)
     tt = 16 if M <= 16 else (32 if M <= 32 else (64 if M <= 64 else 128))
-    rows = -(-M // tt) * tt
+    ntok = -(-M // tt)
+    if tt == 128:  # 128-token tiles go to CTA pairs: an even count
+        ntok += ntok % 2
+    rows = ntok * tt
     tc = _align(rows * B * 64) + _align(rows * B * 4) + (_align(rows * (K // group) * 4) if group else 0)
     # split of K when the output tiles do not fill the SMs (148 without a GPU): partial
     # outputs of M*N f32 per split, at least 16 quant blocks per split
-    tiles = -(-N // 128) * -(-M // tt)
+    tiles = -(-N // 128) * ntok
     ks = 1
     if (M * N) % 4 == 0 and tiles < 148:
         ks = max(1, min(148 // tiles, B // 16))
