@@ -151,17 +151,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
         const int p = tid % NWH;   // weight row within this CTA's half
         const int kq = tid / NWH;  // block of the stage this thread expands
         bool range_bad = false;
-        auto expand = [&](int st) {
-            uint8_t* sp = stage_ptr(st % NS);
+        // The packed codes and scale of this thread's (row, block) task, read from the stage
+        // before any expanded value is stored (the stores of one stage could alias the next
+        // stage's loads, so the loads of both stages are issued first).
+        struct Raw {
+            uint4 wv;
+            uint32_t sb;
+        };
+        auto load_raw = [&](int st) {
+            Raw rw{make_uint4(0u, 0u, 0u, 0u), 0u};
+            const uint8_t* sp = stage_ptr(st % NS);
             const int sb0 = kb0 + st * S;
             const int e0 = (FMT == 0) ? sb0 & ~7 : (sb0 / bpg) & ~7;  // first scale of the TMA box
             if (st * S + kq < Bl) {
                 const int b = sb0 + kq;
                 const int e = (FMT == 0) ? b : b / bpg;
-                const uint4 wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
-                const uint32_t sb =
-                    reinterpret_cast<const uint16_t*>(sp + OFF_RSC + (int(rank) * NWH + p) * 16)[e - e0];
-                const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+                rw.wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
+                rw.sb = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + (int(rank) * NWH + p) * 16)[e - e0];
+            }
+            return rw;
+        };
+        auto expand = [&](int st, const Raw& rw) {
+            uint8_t* sp = stage_ptr(st % NS);
+            const int sb0 = kb0 + st * S;
+            if (st * S + kq < Bl) {
+                const uint32_t sb = rw.sb;
+                const uint32_t w[4] = {rw.wv.x, rw.wv.y, rw.wv.z, rw.wv.w};
                 uint8_t* dst = sp + kq * W_BLK + (p >> 3) * 512 + (p & 7) * 16;
                 if (FMT == 0) {
                     range_bad |= (sb & 0x7FF8u) > 0x6950u;  // d_hi > 2720 (24 d_hi > 65504), inf or nan
@@ -203,6 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 // Bias factors b + 8s of all 128 rows of the pair tile (the epilogue of each
                 // CTA covers all of them): thread tid takes row tid for each group ending in
                 // the stage.
+                const int e0 = (sb0 / bpg) & ~7;
 #pragma unroll
                 for (int k = 0; k < S; ++k) {
                     const int b = sb0 + k;
@@ -221,8 +237,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             const bool two = st + 1 < nstages;  // warp-uniform
             if (!bounded_wait_warp(bar(&ctrl->raw[st % NS]), (st / NS) & 1, abort)) break;
             if (two && !bounded_wait_warp(bar(&ctrl->raw[(st + 1) % NS]), ((st + 1) / NS) & 1, abort)) break;
-            expand(st);
-            if (two) expand(st + 1);
+            const Raw r0 = load_raw(st);
+            const Raw r1 = two ? load_raw(st + 1) : Raw{make_uint4(0u, 0u, 0u, 0u), 0u};
+            expand(st, r0);
+            if (two) expand(st + 1, r1);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -339,12 +357,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             if (!bounded_wait_warp(bar(&ctrl->tfull[g]), (st / NG) & 1, abort)) break;
             tc_fence_after();
             const uint8_t* sp = stage_ptr(slot);
+            // Q4_0 needs only d_x from the stage: read it, then hand the stage back to the
+            // copy warp (the stage's MMAs are complete). Affine also reads C and Z at group
+            // ends and releases the stage after the FMAs.
+            float dxv[S];
+#pragma unroll
+            for (int k = 0; k < S; ++k) dxv[k] = reinterpret_cast<const float*>(sp + OFF_DX)[k * TT + r];
+            if (FMT == 0) {
+                const float dep = dxv[0] + dxv[S - 1];  // one warp instruction: waits for the loads
+                __syncwarp();
+                if (lane == 0) mbar_arrive_after(bar(&ctrl->empty[slot]), dep);
+            }
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 if (k >= nb) break;
                 const int i = kb0 + st * S + k;
                 const bool last = (k == nb - 1);
-                const float dxr = reinterpret_cast<const float*>(sp + OFF_DX)[k * TT + r];
+                const float dxr = dxv[k];
                 const bool group_end = (FMT == 1) && (((i + 1) % bpg) == 0);
 #pragma unroll
                 for (int h0 = 0; h0 < CW; h0 += LD_COLS) {
@@ -376,8 +405,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                     }
                 }
             }
-            __syncwarp();  // the values read from the stage were consumed above
-            if (lane == 0) mbar_arrive(bar(&ctrl->empty[slot]));
+            if (FMT == 1) {
+                __syncwarp();  // the values read from the stage were consumed above
+                if (lane == 0) mbar_arrive(bar(&ctrl->empty[slot]));
+            }
         }
         if (!*abort) {
             const int m = t * TT + r;
