@@ -34,9 +34,10 @@
 //                broadcast shared-memory load per 4 tokens.
 // Warp roles: EPI_WARPS epilogue warps (warp w reads TMEM lane quarter w%4, column chunk
 // w/4 of CW columns, accumulates in f32 registers); PROD_WARPS producer warps (one weight
-// row per thread: 16-B code loads two stages ahead, nibble -> scaled fp16 expansion,
-// store in the core-matrix layout); one MMA-issue warp (also allocates TMEM); one
-// bulk-copy warp (token operand, d_x and Z via plain cp.async.bulk, no multicast). The
+// row per thread: reads the stage's packed codes and scales, nibble -> scaled fp16
+// expansion, store in the core-matrix layout); one MMA-issue warp (also allocates TMEM);
+// one copy warp (2-D TMA boxes of the packed weights; token operand, d_x and Z via plain
+// cp.async.bulk; no multicast). The
 // MMA and copy warps run their loops warp-uniformly with one elected lane issuing. Every
 // wait is bounded and taken by each warp on its own (all lanes probe, a vote keeps the
 // warp converged), so no role is held in lockstep by its slowest warp; the epilogue
