@@ -111,7 +111,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
     const int t = blockIdx.x;                // token tile
     const int n0 = blockIdx.y * NWT;         // the pair's weight rows
     const int nh0 = n0 + int(rank) * NWH;    // the rows this CTA stages
-    const int bpg = (FMT == 1) ? (group >> 5) : 1;
+    // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
+    // a run-time divisor cost hundreds of cycles on the copy and producer paths.
+    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;
+    const int bpm = (1 << bsh) - 1;  // block index & bpm == bpm: last block of its group
     const int G = (FMT == 1) ? K / group : 0;
 
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
@@ -162,10 +165,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             Raw rw{make_uint4(0u, 0u, 0u, 0u), 0u};
             const uint8_t* sp = stage_ptr(st % NS);
             const int sb0 = kb0 + st * S;
-            const int e0 = (FMT == 0) ? sb0 & ~7 : (sb0 / bpg) & ~7;  // first scale of the TMA box
+            const int e0 = (FMT == 0) ? sb0 & ~7 : ((sb0 >> bsh)) & ~7;  // first scale of the TMA box
             if (st * S + kq < Bl) {
                 const int b = sb0 + kq;
-                const int e = (FMT == 0) ? b : b / bpg;
+                const int e = (FMT == 0) ? b : (b >> bsh);
                 rw.wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
                 rw.sb = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + (int(rank) * NWH + p) * 16)[e - e0];
             }
@@ -218,12 +221,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 // Bias factors b + 8s of all 128 rows of the pair tile (the epilogue of each
                 // CTA covers all of them): thread tid takes row tid for each group ending in
                 // the stage.
-                const int e0 = (sb0 / bpg) & ~7;
+                const int e0 = ((sb0 >> bsh)) & ~7;
 #pragma unroll
                 for (int k = 0; k < S; ++k) {
                     const int b = sb0 + k;
-                    if (st * S + k < Bl && ((b + 1) % bpg) == 0) {
-                        const int e = b / bpg;
+                    if (st * S + k < Bl && (b & bpm) == bpm) {
+                        const int e = (b >> bsh);
                         const uint16_t sv = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + tid * 16)[e - e0];
                         const uint16_t bv = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + tid * 16)[e - e0];
                         const float sf = __bfloat162float(__ushort_as_bfloat16(sv));
@@ -262,10 +265,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             if (leader) {
                 int nz = 0;  // affine: groups ending in this stage (each brings its Z row)
                 if (FMT == 1)
-                    for (int k = 0; k < nb; ++k) nz += ((b0 + k + 1) % bpg) == 0;
+                    for (int k = 0; k < nb; ++k) nz += ((b0 + k) & bpm) == bpm;
                 uint8_t* sp = stage_ptr(slot);
                 const uint32_t rb = bar(&ctrl->raw[slot]);
-                const int e0 = (FMT == 0) ? b0 & ~7 : (b0 / bpg) & ~7;
+                const int e0 = (FMT == 0) ? b0 & ~7 : ((b0 >> bsh)) & ~7;
                 mbar_arrive_expect_tx(rb, uint32_t(nb * NWH * 16 + NWT * 16 * (FMT == 1 ? 2 : 1)));
                 for (int k = 0; k < nb; ++k)
                     tma_load_2d(smem_addr(sp + OFF_RAW + k * NWH * 16), &tm_q, (b0 + k) * 16, nh0, rb);
@@ -278,8 +281,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 bulk_g2s(smem_addr(sp + OFF_DX), dxs + (int64_t(t) * B + b0) * TT, uint32_t(nb * DX_BLK), fb);
                 if (FMT == 1) {
                     for (int k = 0; k < nb; ++k)
-                        if (((b0 + k + 1) % bpg) == 0)
-                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + (b0 + k) / bpg) * TT,
+                        if (((b0 + k) & bpm) == bpm)
+                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + ((b0 + k) >> bsh)) * TT,
                                      TT * 4, fb);
                 }
             }
@@ -374,7 +377,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 const int i = kb0 + st * S + k;
                 const bool last = (k == nb - 1);
                 const float dxr = dxv[k];
-                const bool group_end = (FMT == 1) && (((i + 1) % bpg) == 0);
+                const bool group_end = (FMT == 1) && ((i & bpm) == bpm);
 #pragma unroll
                 for (int h0 = 0; h0 < CW; h0 += LD_COLS) {
                     uint32_t pr[LD_COLS];

@@ -210,7 +210,10 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
     float* __restrict__ yo = (gridDim.z > 1) ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : y;
     const int n0 = blockIdx.x * NW;
     const int t = blockIdx.y;
-    const int bpg = (FMT == 1) ? (group >> 5) : 1;  // blocks per affine group
+    // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
+    // a run-time divisor cost hundreds of cycles on the copy and producer paths.
+    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;
+    const int bpm = (1 << bsh) - 1;  // block index & bpm == bpm: last block of its group
     const int G = (FMT == 1) ? K / group : 0;
 
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
@@ -261,8 +264,8 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                     if (FMT == 0) {
                         sv[k] = ld_nc_u16(wscale + int64_t(n) * B + b);
                     } else {
-                        sv[k] = ld_nc_u16(wscale + int64_t(n) * G + b / bpg);
-                        bv[k] = ld_nc_u16(wbias + int64_t(n) * G + b / bpg);
+                        sv[k] = ld_nc_u16(wscale + int64_t(n) * G + (b >> bsh));
+                        bv[k] = ld_nc_u16(wbias + int64_t(n) * G + (b >> bsh));
                     }
                 }
             }
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
             if (!bounded_wait_warp(bar(&ctrl->raw[slot]), (st / NS) & 1, abort)) break;
             uint8_t* sp = stage_ptr(slot);
             const int sb0 = kb0 + st * S;  // first block of the stage
-            const int e0 = (FMT == 0) ? sb0 & ~7 : (sb0 / bpg) & ~7;  // first scale of the TMA box
+            const int e0 = (FMT == 0) ? sb0 & ~7 : (sb0 >> bsh) & ~7;  // first scale of the TMA box
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 const int b = sb0 + k;
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 if (st * S + k < Bl) {
                     wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + k * NW * 16 + p * 16);
                     if (sc_tma) {
-                        const int e = (FMT == 0) ? b : b / bpg;
+                        const int e = (FMT == 0) ? b : b >> bsh;
                         sb = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + p * 16)[e - e0];
                         if (FMT == 1) bb = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + p * 16)[e - e0];
                     } else {
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                             make_uint4(scaled_codes(r[0], s2, s24), scaled_codes(r[1], s2, s24),
                                        scaled_codes(r[2], s2, s24), scaled_codes(r[3], s2, s24));
                     }
-                    if (((b + 1) % bpg) == 0) {  // last block of a group: its bias factor b + 8s
+                    if ((b & bpm) == bpm) {  // last block of a group: its bias factor b + 8s
                         const float bf = __bfloat162float(__ushort_as_bfloat16(uint16_t(bb)));
                         reinterpret_cast<float*>(sp + OFF_C)[k * NW + p] = __fadd_rn(bf, __fmul_rn(8.0f, sf));
                     }
@@ -364,11 +367,11 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
             if (leader) {
                 int nz = 0;  // affine: group ends in this stage (each brings its Z row)
                 if (FMT == 1)
-                    for (int k = 0; k < nb; ++k) nz += ((b0 + k + 1) % bpg) == 0;
+                    for (int k = 0; k < nb; ++k) nz += ((b0 + k) & bpm) == bpm;
                 uint8_t* sp = stage_ptr(slot);
                 // packed weights of the stage (codes, and scales when their pitch allows TMA)
                 const uint32_t rb = bar(&ctrl->raw[slot]);
-                const int e0 = (FMT == 0) ? b0 & ~7 : (b0 / bpg) & ~7;
+                const int e0 = (FMT == 0) ? b0 & ~7 : (b0 >> bsh) & ~7;
                 mbar_arrive_expect_tx(rb, uint32_t(nb * NW * 16 + (sc_tma ? NW * 16 * (FMT == 1 ? 2 : 1) : 0)));
                 for (int k = 0; k < nb; ++k)
                     tma_load_2d(smem_addr(sp + OFF_RAW + k * NW * 16), &tm_q, (b0 + k) * 16, n0, rb);
@@ -383,8 +386,8 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 bulk_g2s(smem_addr(sp + OFF_DX), dxs + (int64_t(t) * B + b0) * TT, uint32_t(nb * DX_BLK), fb);
                 if (FMT == 1) {
                     for (int k = 0; k < nb; ++k)
-                        if (((b0 + k + 1) % bpg) == 0)
-                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + (b0 + k) / bpg) * TT,
+                        if (((b0 + k) & bpm) == bpm)
+                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + ((b0 + k) >> bsh)) * TT,
                                      TT * 4, fb);
                 }
             }
@@ -467,7 +470,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 const int i = kb0 + st * S + k;
                 const bool last = (k == nb - 1);
                 const float* dxk = reinterpret_cast<const float*>(sp + OFF_DX) + k * TT;
-                const bool group_end = (FMT == 1) && (((i + 1) % bpg) == 0);
+                const bool group_end = (FMT == 1) && ((i & bpm) == bpm);
                 const float dxr = TOKL ? dxk[r] : 0.0f;
 #pragma unroll
                 for (int h0 = 0; h0 < CW; h0 += LD_COLS) {

@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(int M, int N, int
     if (n >= N) return;
     const int B = K >> 5;
     const int G = (FMT == 1) ? K / group : 0;
-    const int bpg = (FMT == 1) ? (group >> 5) : 1;
+    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;  // log2(blocks per group): no run-time division
     const uint4* wrow = reinterpret_cast<const uint4*>(wq + int64_t(n) * (K >> 1));
     float acc[MT];
 #pragma unroll
@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(int M, int N, int
                 if (FMT == 0) {
                     ws[u] = __half2float(__ushort_as_half(wscale[int64_t(n) * B + b]));
                 } else {
-                    const int g = b / bpg;
+                    const int g = b >> bsh;
                     ws[u] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + g]));
                     wb[u] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + g]));
                 }
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kGemv2Threads, 1)
     const int rows_w = (gw < N) ? (N - 1 - gw) / W + 1 : 0;
     const int T = rows_w * C;
     const int G = (FMT == 1) ? K / group : 0;
-    const int bpg = (FMT == 1) ? (group >> 5) : 1;
+    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;  // log2(blocks per group): no run-time division
 
     struct Item {
         uint4 w[4];
@@ -182,8 +182,8 @@ __global__ void __launch_bounds__(kGemv2Threads, 1)
                 if (FMT == 0) {
                     it.s[u] = __half2float(__ushort_as_half(wscale[int64_t(n) * B + b]));
                 } else {
-                    it.s[u] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + b / bpg]));
-                    it.b[u] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + b / bpg]));
+                    it.s[u] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + (b >> bsh)]));
+                    it.b[u] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + (b >> bsh)]));
                 }
             }
         }

@@ -143,10 +143,10 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         float z = __fmul_rn(d, float(s));
         z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, 8));
         if (group == 128) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, 16));
-        const int nbg = group >> 5;
-        if (valid && sub == 0 && (b % nbg) == 0) {
-            const int G = K / group;
-            zb[(t * G + b / nbg) * tt + r] = z;
+        const int gsh = (group == 128) ? 2 : 1;  // log2(blocks per group)
+        if (valid && sub == 0 && (b & ((1 << gsh) - 1)) == 0) {
+            const int G = K >> (gsh + 5);
+            zb[(t * G + (b >> gsh)) * tt + r] = z;
         }
     }
 }
