@@ -112,8 +112,12 @@ def test_pack_affine_bit_exact(group, N, K, dtype):
 
 
 # ------------------------------------------------------------------ Q4_0 matmul, full compare
+# M > 64 with K a multiple of 256 runs on CTA pairs: (300, 333, 1024) has an odd token-tile
+# count (padded to a pair) and a ragged weight tile, (200, 512, 4096) splits K over the
+# pairs; the other M > 64 shapes take the single-CTA kernel (scale rows not 16-B aligned).
 SHAPES = [(1, 1, 32), (1, 4096, 4096), (2, 333, 800), (5, 1536, 384), (8, 200, 256), (17, 96, 640),
-          (32, 520, 1056), (64, 1536, 384), (300, 333, 800), (129, 128, 128), (130, 257, 4128), (3, 64, 32768)]
+          (32, 520, 1056), (64, 1536, 384), (300, 333, 800), (129, 128, 128), (130, 257, 4128), (3, 64, 32768),
+          (300, 333, 1024), (200, 512, 4096)]
 
 
 def _q4_0_case(M, N, K, x_dtype="f32", w_std=0.02, seed=0):
@@ -224,7 +228,7 @@ def test_full_size_sampled(wl):
 
 # ------------------------------------------------------------------ affine
 AFFINE_SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (20, 128, 640), (32, 256, 1024), (64, 1536, 384),
-                 (200, 333, 1280), (130, 128, 4096)]
+                 (200, 333, 1280), (130, 128, 4096), (300, 333, 1024), (200, 512, 4096)]
 
 
 @pytest.mark.parametrize("group", [64, 128])
