@@ -27,7 +27,8 @@ W4A8_F32, W4A8_BF16 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 
 EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a8_gemm", "w4a8_gemm_ex",
-           "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_prepare_act",
+           "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_gemm_epi", "w4a8_gemm_affine_epi",
+           "w4a8_prepare_act",
            "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_gemm_noalloc", "w4a8_last_device_error",
            "w4a8_last_cuda_error_string", "w4a8_status_string"]
 
@@ -60,6 +61,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_pack_affine": (I, [P, I, I, I, I, P, P, P, P]),
         "w4a8_gemm_affine": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, P]),
         "w4a8_gemm_affine_ex": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, I, P]),
+        "w4a8_gemm_epi": (I, [I, I, I, P, I, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
+        "w4a8_gemm_affine_epi": (I, [I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
         "w4a8_prepare_act": (I, [I, I, I, P, I, P, Z, I, P]),
         "w4a8_gemm_prepared": (I, [I, I, I, P, P, P, P, Z, I, P]),
         "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
@@ -74,6 +77,19 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn.argtypes = args
     _lib = lib
     return lib
+
+
+class Epilogue(ctypes.Structure):
+    """w4a8_epilogue: bias (N values or NULL), its element type, the element type of y."""
+    _fields_ = [("bias", ctypes.c_void_p), ("bias_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+def _epilogue(bias: torch.Tensor | None, out_dtype: torch.dtype) -> Epilogue:
+    e = Epilogue()
+    e.bias = _ptr(bias).value if bias is not None else None
+    e.bias_dtype = _dtype(bias) if bias is not None else W4A8_F32
+    e.out_dtype = W4A8_BF16 if out_dtype == torch.bfloat16 else (W4A8_F32 if out_dtype == torch.float32 else 99)
+    return e
 
 
 def _ptr(t: torch.Tensor | None):
@@ -135,6 +151,28 @@ def w4a8_gemm(x, qs, d, y, ws, stream=None) -> None:
     N = qs.shape[0]
     _check("w4a8_gemm", load_library().w4a8_gemm(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d), _ptr(y), _ptr(ws),
                                                  ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def w4a8_gemm_epi(x, qs, d, y, ws, bias=None, path: int = PATH_AUTO, stream=None) -> None:
+    """y (f32 or bf16, M x N) = x . W^T + bias (bias: N values, f32 or bf16, or None)."""
+    M, K = x.shape
+    N = qs.shape[0]
+    epi = _epilogue(bias, y.dtype)
+    _check("w4a8_gemm_epi", load_library().w4a8_gemm_epi(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d),
+                                                         ctypes.byref(epi), _ptr(y), _ptr(ws),
+                                                         ws.numel() * ws.element_size(), path, _stream(stream)))
+
+
+def w4a8_gemm_affine_epi(x, q, scale, bias_w, y, ws, group: int, bias=None, path: int = PATH_AUTO,
+                         stream=None) -> None:
+    """Affine weights (scale, bias_w from w4a8_pack_affine) with the output epilogue."""
+    M, K = x.shape
+    N = q.shape[0]
+    epi = _epilogue(bias, y.dtype)
+    _check("w4a8_gemm_affine_epi",
+           load_library().w4a8_gemm_affine_epi(M, N, K, group, _ptr(x), _dtype(x), _ptr(q), _ptr(scale), _ptr(bias_w),
+                                               ctypes.byref(epi), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                                               path, _stream(stream)))
 
 
 def w4a8_pack_affine(w, group: int, q, scale, bias, stream=None) -> None:

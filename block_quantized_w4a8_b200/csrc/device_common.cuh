@@ -226,6 +226,48 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ output epilogue
+// What the contraction kernels store: y[m][n] = product + bias[n] (one f32 addition, the
+// bias of a linear layer as in the C-Kernel-Engine Q4_K GEMM wrapper), written as f32 or
+// rounded to bf16 (round to nearest even). Without a bias the product is stored as is.
+struct Epilogue {
+    const void* bias;  // N values, or nullptr
+    int bias_bf16;     // bias elements: 0 = f32, 1 = bf16
+    int out_bf16;      // y elements: 0 = f32, 1 = bf16
+};
+__device__ __forceinline__ float epi_value(const Epilogue& e, int n, float v) {
+    if (!e.bias) return v;
+    const float b = e.bias_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(e.bias)[n])
+                                : reinterpret_cast<const float*>(e.bias)[n];
+    return __fadd_rn(v, b);
+}
+// y[idx] for output column n.
+__device__ __forceinline__ void epi_store(void* y, int64_t idx, int n, float v, const Epilogue& e) {
+    const float r = epi_value(e, n, v);
+    if (e.out_bf16)
+        reinterpret_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(r);
+    else
+        reinterpret_cast<float*>(y)[idx] = r;
+}
+// y[idx .. idx+3] for columns n .. n+3 of one row (idx a multiple of 4: one 16-byte f32
+// or 8-byte bf16 store).
+__device__ __forceinline__ void epi_store4(void* y, int64_t idx, int n, float a, float b, float c, float d,
+                                           const Epilogue& e) {
+    a = epi_value(e, n, a);
+    b = epi_value(e, n + 1, b);
+    c = epi_value(e, n + 2, c);
+    d = epi_value(e, n + 3, d);
+    if (e.out_bf16) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+        uint2 v;
+        v.x = *reinterpret_cast<const uint32_t*>(&lo);
+        v.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + idx) = v;
+    } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + idx) = make_float4(a, b, c, d);
+    }
+}
+
 // ------------------------------------------------------------------ PDL
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

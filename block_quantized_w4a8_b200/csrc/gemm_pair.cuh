@@ -86,9 +86,9 @@ static_assert(sizeof(PairCtrl) <= CTRL_BYTES, "control block");
 template <int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_THREADS, 1)
     gemm_pair_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dxs,
-                     const float* __restrict__ zb, float* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
+                     const float* __restrict__ zb, void* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int bsplit,
-                     float* __restrict__ ypart) {
+                     float* __restrict__ ypart, Epilogue epi) {
     using Gm = PairGeo<FMT>;
     constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NWT = Gm::NWT, NWH = Gm::NWH;
     constexpr int MN = Gm::MN, CW = Gm::CW, W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK;
@@ -107,7 +107,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
     const int kb0 = blockIdx.z * bsplit;  // this pair contracts blocks [kb0, kb0 + Bl)
     const int Bl = min(B, kb0 + bsplit) - kb0;
     const int nstages = (Bl + S - 1) / S;
-    float* __restrict__ yo = (gridDim.z > 1) ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : y;
+    // Split of K: partial sums (f32, no epilogue) to ypart[z] for the reduction kernel.
+    const bool split = gridDim.z > 1;
+    float* __restrict__ yp = split ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : nullptr;
     const int t = blockIdx.x;                // token tile
     const int n0 = blockIdx.y * NWT;         // the pair's weight rows
     const int nh0 = n0 + int(rank) * NWH;    // the rows this CTA stages
@@ -417,15 +419,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             const int m = t * TT + r;
             const int nb = n0 + c0;
             if (m < M) {
-                float* yr = yo + int64_t(m) * N + nb;
+                const int64_t row = int64_t(m) * N;
                 if ((N & 3) == 0 && nb + CW <= N) {
 #pragma unroll
-                    for (int j = 0; j < CW; j += 4)
-                        *reinterpret_cast<float4*>(yr + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                    for (int j = 0; j < CW; j += 4) {
+                        if (split)
+                            *reinterpret_cast<float4*>(yp + row + nb + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                        else
+                            epi_store4(y, row + nb + j, nb + j, acc[j], acc[j + 1], acc[j + 2], acc[j + 3], epi);
+                    }
                 } else {
 #pragma unroll
                     for (int j = 0; j < CW; ++j)
-                        if (nb + j < N) yr[j] = acc[j];
+                        if (nb + j < N) {
+                            if (split)
+                                yp[row + nb + j] = acc[j];
+                            else
+                                epi_store(y, row + nb + j, nb + j, acc[j], epi);
+                        }
                 }
             }
         }

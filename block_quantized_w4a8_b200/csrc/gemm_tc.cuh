@@ -182,9 +182,9 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
     gemm_tc_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dxs,
                    const float* __restrict__ zb, const uint8_t* __restrict__ wq,
                    const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias,
-                   float* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
+                   void* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int sc_tma,
-                   int bsplit, float* __restrict__ ypart) {
+                   int bsplit, float* __restrict__ ypart, Epilogue epi) {
     using Gm = Geo<FMT, TOKL, MN>;
     constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NW = Gm::NW, CW = Gm::CW;
     constexpr int W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK, DX_BLK = Gm::DX_BLK;
@@ -207,7 +207,9 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
     const int kb0 = blockIdx.z * bsplit;
     const int Bl = min(B, kb0 + bsplit) - kb0;
     const int nstages = (Bl + S - 1) / S;
-    float* __restrict__ yo = (gridDim.z > 1) ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : y;
+    // Split of K: partial sums (f32, no epilogue) to ypart[z] for the reduction kernel.
+    const bool split = gridDim.z > 1;
+    float* __restrict__ yp = split ? ypart + size_t(blockIdx.z) * size_t(M) * size_t(N) : nullptr;
     const int n0 = blockIdx.x * NW;
     const int t = blockIdx.y;
     // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
@@ -531,15 +533,24 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 const int m = t * TT + r;
                 const int nb = n0 + c0;
                 if (m < M) {
-                    float* yr = yo + int64_t(m) * N + nb;
+                    const int64_t row = int64_t(m) * N;
                     if ((N & 3) == 0 && nb + CW <= N) {
 #pragma unroll
-                        for (int j = 0; j < CW; j += 4)
-                            *reinterpret_cast<float4*>(yr + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                        for (int j = 0; j < CW; j += 4) {
+                            if (split)
+                                *reinterpret_cast<float4*>(yp + row + nb + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                            else
+                                epi_store4(y, row + nb + j, nb + j, acc[j], acc[j + 1], acc[j + 2], acc[j + 3], epi);
+                        }
                     } else {
 #pragma unroll
                         for (int j = 0; j < CW; ++j)
-                            if (nb + j < N) yr[j] = acc[j];
+                            if (nb + j < N) {
+                                if (split)
+                                    yp[row + nb + j] = acc[j];
+                                else
+                                    epi_store(y, row + nb + j, nb + j, acc[j], epi);
+                            }
                     }
                 }
             } else {
@@ -548,7 +559,12 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < CW; ++j) {
                         const int m = t * TT + c0 + j;
-                        if (m < M) yo[int64_t(m) * N + n] = acc[j];
+                        if (m < M) {
+                            if (split)
+                                yp[int64_t(m) * N + n] = acc[j];
+                            else
+                                epi_store(y, int64_t(m) * N + n, n, acc[j], epi);
+                        }
                     }
                 }
             }
@@ -566,7 +582,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
 // Sum of the K-split partial outputs in split order: y = part[0] + part[1] + ... (the
 // same order on every call, so results do not depend on scheduling). n4 = M*N/4.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ part, int ks, int64_t n4,
-                                                             float4* __restrict__ y) {
+                                                             int N, void* __restrict__ y, Epilogue epi) {
     pdl_wait_primary();  // the partials are written by the preceding GEMM
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
         float4 a = part[i];
@@ -577,7 +593,15 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __rest
             a.z = __fadd_rn(a.z, b.z);
             a.w = __fadd_rn(a.w, b.w);
         }
-        y[i] = a;
+        if (!epi.bias && !epi.out_bf16) {
+            reinterpret_cast<float4*>(y)[i] = a;
+        } else if ((N & 3) == 0) {  // the four outputs lie in one row
+            epi_store4(y, 4 * i, int((4 * i) % N), a.x, a.y, a.z, a.w, epi);
+        } else {
+            const float v[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) epi_store(y, 4 * i + j, int((4 * i + j) % N), v[j], epi);
+        }
     }
 }
 

@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(int M, int N, int
                                                              const uint8_t* __restrict__ wq,
                                                              const uint16_t* __restrict__ wscale,
                                                              const uint16_t* __restrict__ wbias,
-                                                             float* __restrict__ y) {
+                                                             void* __restrict__ y, Epilogue epi) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = blockIdx.x * kGemvWarps + warp;
     if (n >= N) return;
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(int M, int N, int
         float v = acc[m];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0 && m < M) y[int64_t(m) * N + n] = v;
+        if (lane == 0 && m < M) epi_store(y, int64_t(m) * N + n, n, v, epi);
     }
 }
 
@@ -147,7 +147,8 @@ template <int MT, int FMT, int XMODE>
 __global__ void __launch_bounds__(kGemv2Threads, 1)
     gemv2_kernel(int M, int N, int K, int group, const void* __restrict__ x, const int8_t* __restrict__ qx,
                  const float* __restrict__ dx, const int32_t* __restrict__ sx, const uint8_t* __restrict__ wq,
-                 const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias, float* __restrict__ y) {
+                 const uint16_t* __restrict__ wscale, const uint16_t* __restrict__ wbias, void* __restrict__ y,
+                 Epilogue epi) {
     extern __shared__ __align__(16) uint8_t g2_smem[];
     const int B = K >> 5;
     int8_t* qs_ = reinterpret_cast<int8_t*>(g2_smem);
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(kGemv2Threads, 1)
                 float v = acc[m];
 #pragma unroll
                 for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0 && m < M) y[int64_t(m) * N + n] = v;
+                if (lane == 0 && m < M) epi_store(y, int64_t(m) * N + n, n, v, epi);
                 acc[m] = 0.0f;
             }
         }

@@ -167,8 +167,8 @@ inline int gemv_mt(int mc) { return mc == 1 ? 1 : mc == 2 ? 2 : mc <= 4 ? 4 : 8;
 // Launch one persistent-GEMV instantiation (sets its shared-memory limit once per device).
 template <int MT, int FMT, int XMODE>
 cudaError_t launch_gemv2(int M, int N, int K, int group, const void* x, const int8_t* qx, const float* dx,
-                         const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, float* y,
-                         cudaStream_t stream) {
+                         const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, void* y,
+                         const Epilogue& epi, cudaStream_t stream) {
     static bool configured[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -182,18 +182,18 @@ cudaError_t launch_gemv2(int M, int N, int K, int group, const void* x, const in
     const int64_t ctas = cdiv(N, kGemv2Warps);
     const dim3 grid(unsigned(ctas < sm_count() ? ctas : sm_count()));
     return launch_pdl(gemv2_kernel<MT, FMT, XMODE>, grid, dim3(kGemv2Threads), smem, stream, M, N, K, group, x, qx,
-                      dx, sx, wq, ws, wb, y);
+                      dx, sx, wq, ws, wb, y, epi);
 }
 
 template <int FMT, int XMODE>
 cudaError_t launch_gemv2_mt(int mt, int M, int N, int K, int group, const void* x, const int8_t* qx, const float* dx,
-                            const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, float* y,
-                            cudaStream_t stream) {
+                            const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, void* y,
+                            const Epilogue& epi, cudaStream_t stream) {
     switch (mt) {
-        case 1: return launch_gemv2<1, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
-        case 2: return launch_gemv2<2, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
-        case 4: return launch_gemv2<4, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
-        default: return launch_gemv2<8, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, stream);
+        case 1: return launch_gemv2<1, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, epi, stream);
+        case 2: return launch_gemv2<2, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, epi, stream);
+        case 4: return launch_gemv2<4, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, epi, stream);
+        default: return launch_gemv2<8, FMT, XMODE>(M, N, K, group, x, qx, dx, sx, wq, ws, wb, y, epi, stream);
     }
 }
 
@@ -205,7 +205,7 @@ inline bool gemv_fused(int M, int K) {
 // GEMV contraction from a prepared row-major Q8_0 workspace, in chunks of 8 rows of x.
 template <int FMT>
 w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint8_t* wq, const uint16_t* ws,
-                     const uint16_t* wb, float* y, cudaStream_t stream) {
+                     const uint16_t* wb, void* y, const Epilogue& epi, cudaStream_t stream) {
     const int B = K / 32;
     for (int m0 = 0; m0 < M; m0 += 8) {
         const int mc = (M - m0 < 8) ? (M - m0) : 8;
@@ -213,21 +213,21 @@ w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint
         const int8_t* qx = a.qx + int64_t(m0) * K;
         const float* dx = a.dx + int64_t(m0) * B;
         const int32_t* sx = a.sx + int64_t(m0) * B;
-        float* yy = y + int64_t(m0) * N;
+        void* yy = static_cast<char*>(y) + int64_t(m0) * N * (epi.out_bf16 ? 2 : 4);
         cudaError_t e;
         if (gemv2_smem_bytes(mt, K) <= kGemv2MaxSmem) {
-            e = launch_gemv2_mt<FMT, 0>(mt, mc, N, K, group, nullptr, qx, dx, sx, wq, ws, wb, yy, stream);
+            e = launch_gemv2_mt<FMT, 0>(mt, mc, N, K, group, nullptr, qx, dx, sx, wq, ws, wb, yy, epi, stream);
         } else {  // activation too large for shared memory: stream it from L1/L2
             const dim3 grid(unsigned(cdiv(N, kGemvWarps)));
             const dim3 block(kGemvWarps * 32);
             if (mt == 1)
-                e = launch_pdl(gemv_kernel<1, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+                e = launch_pdl(gemv_kernel<1, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
             else if (mt == 2)
-                e = launch_pdl(gemv_kernel<2, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+                e = launch_pdl(gemv_kernel<2, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
             else if (mt == 4)
-                e = launch_pdl(gemv_kernel<4, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+                e = launch_pdl(gemv_kernel<4, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
             else
-                e = launch_pdl(gemv_kernel<8, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy);
+                e = launch_pdl(gemv_kernel<8, FMT>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
         }
         if (e != cudaSuccess) return cuda_status(e);
     }
@@ -237,11 +237,11 @@ w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint
 // One-launch GEMV that quantises x itself (requires gemv_fused(M, K)).
 template <int FMT>
 w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
-                           const uint16_t* ws, const uint16_t* wb, float* y, cudaStream_t stream) {
+                           const uint16_t* ws, const uint16_t* wb, void* y, const Epilogue& epi, cudaStream_t stream) {
     const int mt = gemv_mt(M);
     cudaError_t e = (dt == W4A8_BF16)
-                        ? launch_gemv2_mt<FMT, 2>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, stream)
-                        : launch_gemv2_mt<FMT, 1>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, stream);
+                        ? launch_gemv2_mt<FMT, 2>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, epi, stream)
+                        : launch_gemv2_mt<FMT, 1>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, epi, stream);
     return cuda_status(e);
 }
 
@@ -313,7 +313,8 @@ bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e
 
 template <int FMT, bool TOKL, int MN>
 w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                           const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
+                           const uint16_t* wb, void* y, const Epilogue& epi, bool pdl, size_t work_bytes,
+                           cudaStream_t stream) {
     using Gm = tc::Geo<FMT, TOKL, MN>;
     static bool configured[64] = {false};
     int dev = 0;
@@ -350,13 +351,13 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
     cudaError_t e = launch_pdl_if(pdl, tc::gemm_tc_kernel<FMT, TOKL, MN>, grid, dim3(Gm::NUM_THREADS),
                                   size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
                                   (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y, tq, tsc, tbi, sc_tma,
-                                  sp.bsplit, part);
+                                  sp.bsplit, part, epi);
     if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
     const int64_t n4 = int64_t(M) * N / 4;
     int64_t rb = cdiv(n4, 256);
     if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
     e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, (const float4*)part, sp.ks, n4,
-                   reinterpret_cast<float4*>(y));
+                   N, y, epi);
     return cuda_status(e);
 }
 
@@ -364,7 +365,8 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
 // weight tile, each CTA staging half of its rows.
 template <int FMT>
 w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                             const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
+                             const uint16_t* wb, void* y, const Epilogue& epi, bool pdl, size_t work_bytes,
+                             cudaStream_t stream) {
     using Gm = tc::PairGeo<FMT>;
     static bool configured[64] = {false};
     int dev = 0;
@@ -392,13 +394,13 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
     const dim3 grid(unsigned(w.tiles), unsigned(cdiv(N, Gm::NWT)), unsigned(sp.ks));
     cudaError_t e = launch_pdl_if(pdl, tc::gemm_pair_kernel<FMT>, grid, dim3(Gm::NUM_THREADS),
                                   size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
-                                  (const float*)w.dxs, (const float*)w.z, y, tq, tsc, tbi, sp.bsplit, part);
+                                  (const float*)w.dxs, (const float*)w.z, y, tq, tsc, tbi, sp.bsplit, part, epi);
     if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
     const int64_t n4 = int64_t(M) * N / 4;
     int64_t rb = cdiv(n4, 256);
     if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
     e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, (const float4*)part, sp.ks, n4,
-                   reinterpret_cast<float4*>(y));
+                   N, y, epi);
     return cuda_status(e);
 }
 
@@ -407,16 +409,17 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
 // when the scale rows can be fetched by TMA (their pitch a multiple of 16 bytes).
 template <int FMT>
 w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
-                        const uint16_t* wb, float* y, bool pdl, size_t work_bytes, cudaStream_t stream) {
+                        const uint16_t* wb, void* y, const Epilogue& epi, bool pdl, size_t work_bytes,
+                        cudaStream_t stream) {
     switch (w.tt) {
-        case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
-        case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
-        case 64: return launch_gemm_tc<FMT, false, 64>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+        case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
+        case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
+        case 64: return launch_gemm_tc<FMT, false, 64>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
         default: {
             const int E = (FMT == 0) ? K / 32 : K / group;
             if ((E * 2) % 16 == 0)
-                return launch_gemm_pair<FMT>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
-            return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, pdl, work_bytes, stream);
+                return launch_gemm_pair<FMT>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
+            return launch_gemm_tc<FMT, true, 128>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
         }
     }
 }
@@ -430,7 +433,7 @@ size_t min_workspace_bytes(int M, int K, int group) {
 }
 
 w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
-                            const void* wb, bool affine, int group, const float* y, const void* work,
+                            const void* wb, bool affine, int group, const void* y, const void* work,
                             size_t work_bytes, w4a8_path path) {
     if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 32) != 0) return W4A8_ERR_INVALID_ARG;
     if (!x || !wq || !ws || !y || (affine && !wb)) return W4A8_ERR_INVALID_ARG;
@@ -445,6 +448,24 @@ w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, c
     if (!work) return W4A8_ERR_WORKSPACE;
     if (!aligned16(work)) return W4A8_ERR_MISALIGNED;
     if (work_bytes < min_workspace_bytes(M, K, affine ? group : 0)) return W4A8_ERR_WORKSPACE;
+    return W4A8_OK;
+}
+
+// The epilogue of the entry points without one: f32 output, no bias.
+const Epilogue kPlain{nullptr, 0, 0};
+
+// Checks a caller's epilogue and converts it (nullptr: f32 output, no bias).
+w4a8_status make_epilogue(const w4a8_epilogue* in, Epilogue* out) {
+    *out = kPlain;
+    if (!in) return W4A8_OK;
+    if ((in->bias_dtype != W4A8_F32 && in->bias_dtype != W4A8_BF16) ||
+        (in->out_dtype != W4A8_F32 && in->out_dtype != W4A8_BF16))
+        return W4A8_ERR_UNSUPPORTED;
+    if (in->bias && (reinterpret_cast<uintptr_t>(in->bias) & (in->bias_dtype == W4A8_BF16 ? 1u : 3u)) != 0)
+        return W4A8_ERR_MISALIGNED;
+    out->bias = in->bias;
+    out->bias_bf16 = in->bias_dtype == W4A8_BF16 ? 1 : 0;
+    out->out_bf16 = in->out_dtype == W4A8_BF16 ? 1 : 0;
     return W4A8_OK;
 }
 
@@ -467,23 +488,24 @@ w4a8_status prepare_impl(int M, int K, int group, const void* x, w4a8_dtype dt, 
 // tail (programmatic dependent launch); otherwise it starts after all prior work.
 template <int FMT>
 w4a8_status contract_impl(int M, int N, int K, int group, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb,
-                          float* y, void* work, size_t work_bytes, bool gemv, bool after_quant, cudaStream_t stream) {
-    if (gemv) return run_gemv<FMT>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, stream);
-    return run_gemm_tc<FMT>(M, N, K, group, tc_ws(work, M, K, FMT == 1 ? group : 0), wq, ws, wb, y, after_quant,
-                            work_bytes, stream);
+                          void* y, const Epilogue& epi, void* work, size_t work_bytes, bool gemv, bool after_quant,
+                          cudaStream_t stream) {
+    if (gemv) return run_gemv<FMT>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, epi, stream);
+    return run_gemm_tc<FMT>(M, N, K, group, tc_ws(work, M, K, FMT == 1 ? group : 0), wq, ws, wb, y, epi,
+                            after_quant, work_bytes, stream);
 }
 
 template <int FMT>
 w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
-                      const uint16_t* ws, const uint16_t* wb, float* y, void* work, size_t work_bytes,
-                      w4a8_path path, cudaStream_t stream) {
+                      const uint16_t* ws, const uint16_t* wb, void* y, const Epilogue& epi, void* work,
+                      size_t work_bytes, w4a8_path path, cudaStream_t stream) {
     w4a8_status st = check_gemm_args(M, N, K, x, dt, wq, ws, wb, FMT == 1, group, y, work, work_bytes, path);
     if (st != W4A8_OK) return st;
     const bool gemv = use_gemv(M, path);
-    if (gemv && gemv_fused(M, K)) return run_gemv_fused<FMT>(M, N, K, group, x, dt, wq, ws, wb, y, stream);
+    if (gemv && gemv_fused(M, K)) return run_gemv_fused<FMT>(M, N, K, group, x, dt, wq, ws, wb, y, epi, stream);
     st = prepare_impl(M, K, FMT == 1 ? group : 0, x, dt, work, gemv, stream);
     if (st != W4A8_OK) return st;
-    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, work, work_bytes, gemv, true, stream);
+    return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, epi, work, work_bytes, gemv, true, stream);
 }
 
 }  // namespace
@@ -524,7 +546,7 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group) {
 w4a8_status w4a8_gemm_ex(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
                          const uint16_t* d_fp16, float* y, void* ws, size_t ws_bytes, w4a8_path path,
                          cudaStream_t stream) {
-    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, ws, ws_bytes, path, stream);
+    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, kPlain, ws, ws_bytes, path, stream);
 }
 
 w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
@@ -552,7 +574,7 @@ w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int 
 w4a8_status w4a8_gemm_affine_ex(int M, int N, int K, int group, const void* x, w4a8_dtype dtype, const uint32_t* q,
                                 const uint16_t* scale_bf16, const uint16_t* bias_bf16, float* y, void* ws,
                                 size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
-    return gemm_impl<1>(M, N, K, group, x, dtype, reinterpret_cast<const uint8_t*>(q), scale_bf16, bias_bf16, y, ws,
+    return gemm_impl<1>(M, N, K, group, x, dtype, reinterpret_cast<const uint8_t*>(q), scale_bf16, bias_bf16, y, kPlain, ws,
                         ws_bytes, path, stream);
 }
 
@@ -573,11 +595,30 @@ w4a8_status w4a8_prepare_act(int M, int K, int group, const void* x, w4a8_dtype 
     return prepare_impl(M, K, group, x, dtype, ws, use_gemv(M, path), stream);
 }
 
+w4a8_status w4a8_gemm_epi(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
+                          const uint16_t* d_fp16, const w4a8_epilogue* epi, void* y, void* ws, size_t ws_bytes,
+                          w4a8_path path, cudaStream_t stream) {
+    Epilogue e;
+    const w4a8_status st = make_epilogue(epi, &e);
+    if (st != W4A8_OK) return st;
+    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, e, ws, ws_bytes, path, stream);
+}
+
+w4a8_status w4a8_gemm_affine_epi(int M, int N, int K, int group, const void* x, w4a8_dtype dtype, const uint32_t* q,
+                                 const uint16_t* scale_bf16, const uint16_t* bias_bf16, const w4a8_epilogue* epi,
+                                 void* y, void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
+    Epilogue e;
+    const w4a8_status st = make_epilogue(epi, &e);
+    if (st != W4A8_OK) return st;
+    return gemm_impl<1>(M, N, K, group, x, dtype, reinterpret_cast<const uint8_t*>(q), scale_bf16, bias_bf16, y, e,
+                        ws, ws_bytes, path, stream);
+}
+
 w4a8_status w4a8_gemm_prepared(int M, int N, int K, const uint8_t* qs, const uint16_t* d_fp16, float* y,
                                const void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
     w4a8_status st = check_gemm_args(M, N, K, qs, W4A8_F32, qs, d_fp16, nullptr, false, 0, y, ws, ws_bytes, path);
     if (st != W4A8_OK) return st;
-    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, const_cast<void*>(ws), ws_bytes, use_gemv(M, path),
+    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, kPlain, const_cast<void*>(ws), ws_bytes, use_gemv(M, path),
                             false, stream);
 }
 
@@ -588,7 +629,7 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
     w4a8_status st =
         check_gemm_args(M, N, K, wq, W4A8_F32, wq, scale_bf16, bias_bf16, true, group, y, ws, ws_bytes, path);
     if (st != W4A8_OK) return st;
-    return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, const_cast<void*>(ws), ws_bytes,
+    return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, kPlain, const_cast<void*>(ws), ws_bytes,
                             use_gemv(M, path), false, stream);
 }
 
@@ -612,7 +653,7 @@ w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dty
         if (e != cudaSuccess) return cuda_status(e);
         scratch_ptr[dev] = p;
     }
-    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, scratch_ptr[dev], W4A8_NOALLOC_SCRATCH_BYTES,
+    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, kPlain, scratch_ptr[dev], W4A8_NOALLOC_SCRATCH_BYTES,
                         W4A8_PATH_AUTO, stream);
 }
 

@@ -157,6 +157,38 @@ w4a8_status w4a8_gemm_affine_ex(int M, int N, int K, int group, const void* x, w
                                 w4a8_path path, cudaStream_t stream);
 
 /*
+ * Output epilogue of a linear layer: y[m][n] = P[m][n] + bias[n], stored as f32 or bf16,
+ * where P is the product w4a8_gemm / w4a8_gemm_affine compute. The bias is added in f32
+ * (one rounding) to every row, as the Q4_K GEMM wrapper of the C-Kernel-Engine page
+ * (gemm_kernels_q4k.c, "Engine-compatible wrapper: GEMM_NT with Q4_K weights") adds its
+ * optional bias after the product; a bf16 output is that f32 value rounded to the nearest
+ * bf16 (ties to even; NaN stays NaN, overflow gives infinity).
+ *  bias      : N values of bias_dtype (W4A8_F32 or W4A8_BF16), naturally aligned, or NULL
+ *              (no bias: P is stored unchanged).
+ *  out_dtype : element type of y: W4A8_F32 (float) or W4A8_BF16 (bf16 bit patterns).
+ * The struct is read during the call only; the bias must stay valid until the work
+ * enqueued on `stream` has run.
+ */
+typedef struct {
+    const void* bias;
+    w4a8_dtype bias_dtype;
+    w4a8_dtype out_dtype;
+} w4a8_epilogue;
+
+/*
+ * w4a8_gemm_ex / w4a8_gemm_affine_ex with an epilogue (NULL: as w4a8_gemm_ex). y is M x N
+ * elements of epi->out_dtype, 16-byte aligned. Errors: as w4a8_gemm, plus UNSUPPORTED for
+ * an unknown bias or output type and MISALIGNED for a bias not aligned to its element size.
+ */
+w4a8_status w4a8_gemm_epi(int M, int N, int K, const void* x, w4a8_dtype dtype,
+                          const uint8_t* qs, const uint16_t* d_fp16, const w4a8_epilogue* epi, void* y,
+                          void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream);
+w4a8_status w4a8_gemm_affine_epi(int M, int N, int K, int group, const void* x, w4a8_dtype dtype,
+                                 const uint32_t* q, const uint16_t* scale_bf16, const uint16_t* bias_bf16,
+                                 const w4a8_epilogue* epi, void* y, void* ws, size_t ws_bytes, w4a8_path path,
+                                 cudaStream_t stream);
+
+/*
  * Split form of w4a8_gemm / w4a8_gemm_affine for an activation that feeds several
  * weight matrices (e.g. projections sharing one input): the activation is quantised
  * once and the per-call re-quantisation the tract page identifies as per-op overhead

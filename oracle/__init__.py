@@ -21,6 +21,9 @@ Functions and the definitions they follow (see the header of ``oracle.cpp``):
 * ``pack_affine`` / ``gemm_affine`` -- MLX PR #4802 "mx.qqmm ... mode=affine": codes
   q in [0,15], per-group bf16 scale (max-min)/15 and bias min; the contraction runs on
   the original codes and applies d_x * (s * sum q q_x + b * sum q_x) per block.
+* ``epilogue`` -- the output of a linear layer: the optional per-column bias added to
+  every row of the f32 product in f32 (C-Kernel-Engine gemm_kernels_q4k.c, "Engine-
+  compatible wrapper: GEMM_NT with Q4_K weights"), then f32 or bf16 (nearest even).
 """
 from __future__ import annotations
 
@@ -259,3 +262,19 @@ def gemm_affine_sampled(qx, dx, sx, q, scale, bias, group: int, ms, ns) -> tuple
                                     _p(np.ascontiguousarray(scale, dtype=np.uint16)),
                                     _p(np.ascontiguousarray(bias, dtype=np.uint16)), _p(y), _p(T))
     return y, T
+
+
+def epilogue(p, bias=None, bias_bf16: bool = False, out_bf16: bool = False) -> np.ndarray:
+    """Output epilogue: y[m][n] = f32(p[m][n]) + f32(bias[n]) with one f32 rounding
+    (C-Kernel-Engine gemm_kernels_q4k.c, "Engine-compatible wrapper: GEMM_NT with Q4_K
+    weights": after the product, ``row[j] += bias[j]`` for every row), no addition when
+    ``bias`` is None; a bf16 output is that value narrowed to bf16 with round-to-nearest-even
+    (returned as uint16 bit patterns). ``bias`` is f32 values, or bf16 bit patterns when
+    ``bias_bf16``."""
+    y = np.asarray(p, dtype=np.float32)
+    if bias is not None:
+        b = bf16_to_f32(bias) if bias_bf16 else np.asarray(bias, dtype=np.float32)
+        y = (y + b.reshape(1, -1)).astype(np.float32)  # IEEE single-precision addition
+    if out_bf16:
+        return f32_to_bf16(y)
+    return y
