@@ -505,7 +505,59 @@ def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
         results.append(entry)
         del sets
         torch.cuda.empty_cache()
+    results += run_epilogue(args, torch, w4a8, oracle, inputs, steps, dev)
     return results
+
+
+def run_epilogue(args, torch, w4a8, oracle, inputs, steps, dev):
+    """The output epilogue (per-column f32 bias, bf16 output) on the decode GEMV and the
+    prefill GEMM, through w4a8_gemm_epi, timed beside the plain call on the same inputs."""
+    import numpy as np
+    out = []
+    for wl in (inputs.DECODE, inputs.PREFILL):
+        M, N, K = wl.M, wl.N, wl.K
+        x, w = inputs.make(wl)
+        xd = x.to(dev)
+        bias = inputs.randn((N,), seed=5, std=1.0)
+        bd = bias.to(dev)
+        qs, d = w4a8.pack_q4_0(w.to(dev))
+        R = copies_for(weight_bytes(N, K))
+        sets = [(qs.clone(), d.clone()) for _ in range(R)]
+        ws = w4a8.workspace(M, N, K, 0, dev)
+        y = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+        yp = torch.empty(M, N, device=dev)
+        w4a8.w4a8_gemm_epi(xd, qs, d, y, ws, bias=bd)
+        torch.cuda.synchronize()
+        rqx, rdx, _ = oracle.quant_act_q8_0(x.float().numpy())
+        rqs, rd = oracle.pack_q4_0(w.numpy())
+        ms, ns = (np.asarray(t) for t in inputs.sample_indices(M, N, 400, 7))
+        yref, T = oracle.gemm_q4_0_sampled(rqx, rdx, rqs, rd, ms, ns)
+        ref = oracle.bf16_to_f32(oracle.epilogue(yref.astype(np.float32)[None, :], bias.numpy()[ns],
+                                                 out_bf16=True)[0]).astype(np.float64)
+        got = y.float().cpu().numpy()[ms, ns].astype(np.float64)
+        ok = bool(np.all(np.abs(got - ref) <= 1e-5 * T + np.abs(ref) * 2.0 ** -7))
+        entry = {"workload": wl.name + "_bias_bf16out", "M": M, "N": N, "K": K,
+                 "path": "gemv" if M <= 8 else "gemm_tc", "epilogue": "f32 bias per column, bf16 output",
+                 "parity": "pass" if ok else "FAIL"}
+        if ok:
+            def step(i):
+                qq, dd = sets[i % R]
+                w4a8.w4a8_gemm_epi(xd, qq, dd, y, ws, bias=bd)
+
+            def plain(i):
+                qq, dd = sets[i % R]
+                w4a8.w4a8_gemm(xd, qq, dd, yp, ws)
+            for i in range(3):
+                step(i)
+                plain(i)
+            us = timed(step, steps, torch, graph=True) / steps * 1e3
+            us_plain = timed(plain, steps, torch, graph=True) / steps * 1e3
+            entry.update({"us_per_call": us, "us_per_call_plain": us_plain,
+                          "tops_call": 2.0 * M * N * K / (us * 1e-6) / 1e12, "l2": f"{R} rotating weight copies"})
+        out.append(entry)
+        del sets
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_probe(args):

@@ -420,23 +420,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             const int nb = n0 + c0;
             if (m < M) {
                 const int64_t row = int64_t(m) * N;
-                if ((N & 3) == 0 && nb + CW <= N) {
+                // Plain f32 stores for split partials and calls without an epilogue; the
+                // epilogue's per-element work only when one is given.
+                float* yf = split ? yp : ((epi.bias || epi.out_bf16) ? nullptr : reinterpret_cast<float*>(y));
+                if (yf) {
+                    if ((N & 3) == 0 && nb + CW <= N) {
 #pragma unroll
-                    for (int j = 0; j < CW; j += 4) {
-                        if (split)
-                            *reinterpret_cast<float4*>(yp + row + nb + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-                        else
-                            epi_store4(y, row + nb + j, nb + j, acc[j], acc[j + 1], acc[j + 2], acc[j + 3], epi);
+                        for (int j = 0; j < CW; j += 4)
+                            *reinterpret_cast<float4*>(yf + row + nb + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < CW; ++j)
+                            if (nb + j < N) yf[row + nb + j] = acc[j];
                     }
+                } else if ((N & 3) == 0 && nb + CW <= N) {
+#pragma unroll
+                    for (int j = 0; j < CW; j += 4)
+                        epi_store4(y, row + nb + j, nb + j, acc[j], acc[j + 1], acc[j + 2], acc[j + 3], epi);
                 } else {
 #pragma unroll
                     for (int j = 0; j < CW; ++j)
-                        if (nb + j < N) {
-                            if (split)
-                                yp[row + nb + j] = acc[j];
-                            else
-                                epi_store(y, row + nb + j, nb + j, acc[j], epi);
-                        }
+                        if (nb + j < N) epi_store(y, row + nb + j, nb + j, acc[j], epi);
                 }
             }
         }
