@@ -10,6 +10,15 @@
 // bound the single-CTA kernel (the expanded operand is 128 B per row and block), while the
 // epilogue is unchanged: each CTA's tensor memory holds its 128 tokens x all 128 rows.
 //
+// Affine weights: the group bias term (b + 8s) * sum(q_x) goes through the tensor core as
+// one more K = 16 MMA per block into the block's accumulator, ahead of the per-block
+// activation scale: the token operand carries the block's two 16-element code sums
+// [S1, S2, S1/2^11, S2/2^11] (exact fp16, written by the quantisation kernel), the weight
+// operand the row's C = b + 8s as [C_hi, C_hi, C_lo, C_lo] with C_hi = fp16(C) and
+// C_lo = fp16((C - C_hi) * 2^11), so that C_hi + C_lo / 2^11 carries 22 bits of C. The
+// second 8-element K chunk of both operands is a zero region of shared memory. The
+// epilogue is then the same single FMA per output and block as for Q4_0.
+//
 // Roles per CTA (448 threads): 8 epilogue warps, 4 producer warps (one thread per (row of
 // the CTA's half, block of the stage), two stages at a time), one MMA warp, one bulk-copy
 // warp. Only the even
@@ -40,14 +49,16 @@ struct PairGeo {
     static constexpr int S = 2;                     // quant blocks per stage (one commit)
     static constexpr int OFF_T = S * W_BLK;
     static constexpr int OFF_DX = OFF_T + S * T_BLK;
-    static constexpr int OFF_C = align_up(OFF_DX + S * DX_BLK, 128);            // affine: b + 8s, all 128 rows
-    static constexpr int OFF_Z = OFF_C + (FMT == 1 ? S * NWT * 4 : 0);          // affine: Z per token
-    static constexpr int OFF_RAW = align_up(OFF_Z + (FMT == 1 ? S * TT * 4 : 0), 128);  // codes, own half
+    static constexpr int OFF_XT = align_up(OFF_DX + S * DX_BLK, 128);           // affine: token code sums
+    static constexpr int OFF_XW = OFF_XT + (FMT == 1 ? S * TT * 16 : 0);        // affine: C parts, own half
+    static constexpr int OFF_RAW = align_up(OFF_XW + (FMT == 1 ? S * NWH * 16 : 0), 128);  // codes, own half
     static constexpr int OFF_RSC = OFF_RAW + S * NWH * 16;                      // scales, all 128 rows
     static constexpr int OFF_RBI = OFF_RSC + NWT * 16;                          // affine biases
     static constexpr int STAGE_BYTES = align_up(OFF_RBI + (FMT == 1 ? NWT * 16 : 0), 1024);
-    static constexpr int NS = cmin(8, (SMEM_LIMIT - CTRL_BYTES - 1024) / STAGE_BYTES);
-    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + CTRL_BYTES + 1024;
+    static constexpr int ZERO_BYTES = (FMT == 1) ? TT * 16 : 0;  // zero K chunk of the bias MMA
+    static constexpr int NS = cmin(8, (SMEM_LIMIT - CTRL_BYTES - ZERO_BYTES - 1024) / STAGE_BYTES);
+    static constexpr int OFF_ZERO = NS * STAGE_BYTES + CTRL_BYTES;
+    static constexpr int SMEM_BYTES = OFF_ZERO + ZERO_BYTES + 1024;
     static constexpr int NBUF = 512 / MN;           // accumulator tiles (one per block)
     static constexpr int NG = NBUF / S;             // TMEM groups: stage st uses group st % NG
     static constexpr int TMEM_COLS = 512;
@@ -63,7 +74,7 @@ struct PairGeo {
     static_assert(NS >= 3 && NS <= 8, "pipeline depth");
     static_assert(NG == 2 && NBUF % S == 0, "TMEM groups");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
-    static_assert(OFF_T % 128 == 0 && OFF_DX % 16 == 0 && OFF_Z % 16 == 0 && OFF_RSC % 16 == 0, "alignment");
+    static_assert(OFF_T % 128 == 0 && OFF_DX % 16 == 0 && OFF_XT % 128 == 0 && OFF_RSC % 16 == 0, "alignment");
 };
 
 struct PairCtrl {
@@ -86,14 +97,14 @@ static_assert(sizeof(PairCtrl) <= CTRL_BYTES, "control block");
 template <int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_THREADS, 1)
     gemm_pair_kernel(int M, int N, int K, int group, const __half* __restrict__ tok, const float* __restrict__ dxs,
-                     const float* __restrict__ zb, void* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
+                     const uint4* __restrict__ xsum, void* __restrict__ y, const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_b, int bsplit,
                      float* __restrict__ ypart, Epilogue epi) {
     using Gm = PairGeo<FMT>;
     constexpr int S = Gm::S, NS = Gm::NS, NG = Gm::NG, TT = Gm::TT, NWT = Gm::NWT, NWH = Gm::NWH;
     constexpr int MN = Gm::MN, CW = Gm::CW, W_PART = Gm::W_PART, W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK;
-    constexpr int DX_BLK = Gm::DX_BLK, OFF_T = Gm::OFF_T, OFF_DX = Gm::OFF_DX, OFF_C = Gm::OFF_C;
-    constexpr int OFF_Z = Gm::OFF_Z, OFF_RAW = Gm::OFF_RAW, OFF_RSC = Gm::OFF_RSC, OFF_RBI = Gm::OFF_RBI;
+    constexpr int DX_BLK = Gm::DX_BLK, OFF_T = Gm::OFF_T, OFF_DX = Gm::OFF_DX, OFF_XT = Gm::OFF_XT;
+    constexpr int OFF_XW = Gm::OFF_XW, OFF_RAW = Gm::OFF_RAW, OFF_RSC = Gm::OFF_RSC, OFF_RBI = Gm::OFF_RBI;
     constexpr int STAGE_BYTES = Gm::STAGE_BYTES, EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0;
     constexpr int PROD_WARPS = Gm::PROD_WARPS, MMA_WARP = Gm::MMA_WARP, COPY_WARP = Gm::COPY_WARP;
     constexpr int LD_COLS = Gm::LD_COLS;
@@ -116,8 +127,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
     // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
     // a run-time divisor cost hundreds of cycles on the copy and producer paths.
     const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;
-    const int bpm = (1 << bsh) - 1;  // block index & bpm == bpm: last block of its group
-    const int G = (FMT == 1) ? K / group : 0;
 
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
     auto bar = [](unsigned long long* p) { return smem_addr(p); };
@@ -136,6 +145,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
         mbar_init(bar(&ctrl->drain), 1);
         ctrl->abort = 0;
         mbar_init_fence();
+    }
+    if (FMT == 1 && threadIdx.x < Gm::ZERO_BYTES / 16) {
+        reinterpret_cast<uint4*>(smem + Gm::OFF_ZERO)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();  // read by the tensor core
     }
     if (warp == MMA_WARP) {
         tmem_alloc_pair(smem_addr(&ctrl->tmem_base), Gm::TMEM_COLS);
@@ -162,9 +175,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
         struct Raw {
             uint4 wv;
             uint32_t sb;
+            uint32_t bb;  // affine: the group's bias
         };
         auto load_raw = [&](int st) {
-            Raw rw{make_uint4(0u, 0u, 0u, 0u), 0u};
+            Raw rw{make_uint4(0u, 0u, 0u, 0u), 0u, 0u};
             const uint8_t* sp = stage_ptr(st % NS);
             const int sb0 = kb0 + st * S;
             const int e0 = (FMT == 0) ? sb0 & ~7 : ((sb0 >> bsh)) & ~7;  // first scale of the TMA box
@@ -173,12 +187,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 const int e = (FMT == 0) ? b : (b >> bsh);
                 rw.wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
                 rw.sb = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + (int(rank) * NWH + p) * 16)[e - e0];
+                if (FMT == 1) rw.bb = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + (int(rank) * NWH + p) * 16)[e - e0];
             }
             return rw;
         };
         auto expand = [&](int st, const Raw& rw) {
             uint8_t* sp = stage_ptr(st % NS);
-            const int sb0 = kb0 + st * S;
             if (st * S + kq < Bl) {
                 const uint32_t sb = rw.sb;
                 const uint32_t w[4] = {rw.wv.x, rw.wv.y, rw.wv.z, rw.wv.w};
@@ -217,24 +231,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                             make_uint4(scaled_codes(r[0], s2, s24), scaled_codes(r[1], s2, s24),
                                        scaled_codes(r[2], s2, s24), scaled_codes(r[3], s2, s24));
                     }
-                }
-            }
-            if (FMT == 1) {
-                // Bias factors b + 8s of all 128 rows of the pair tile (the epilogue of each
-                // CTA covers all of them): thread tid takes row tid for each group ending in
-                // the stage.
-                const int e0 = ((sb0 >> bsh)) & ~7;
-#pragma unroll
-                for (int k = 0; k < S; ++k) {
-                    const int b = sb0 + k;
-                    if (st * S + k < Bl && (b & bpm) == bpm) {
-                        const int e = (b >> bsh);
-                        const uint16_t sv = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + tid * 16)[e - e0];
-                        const uint16_t bv = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + tid * 16)[e - e0];
-                        const float sf = __bfloat162float(__ushort_as_bfloat16(sv));
-                        const float bf = __bfloat162float(__ushort_as_bfloat16(bv));
-                        reinterpret_cast<float*>(sp + OFF_C)[k * NWT + tid] = __fadd_rn(bf, __fmul_rn(8.0f, sf));
-                    }
+                    // The bias MMA's weight column for this row and block: C = b + 8s in two
+                    // fp16 parts (C - C_hi is exact in f32; the scaled low part stays normal
+                    // down to |C| = 2^-14).
+                    const float bf = __bfloat162float(__ushort_as_bfloat16(uint16_t(rw.bb)));
+                    const float cf = __fadd_rn(bf, __fmul_rn(8.0f, sf));
+                    range_bad |= !(fabsf(cf) <= 65504.0f);
+                    const __half ch = __float2half_rn(cf);
+                    const __half cl = __float2half_rn(__fmul_rn(__fsub_rn(cf, __half2float(ch)), 2048.0f));
+                    *reinterpret_cast<uint4*>(sp + OFF_XW + kq * NWH * 16 + p * 16) =
+                        make_uint4(pair_of(ch), pair_of(cl), 0u, 0u);
                 }
             }
         };
@@ -243,7 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             if (!bounded_wait_warp(bar(&ctrl->raw[st % NS]), (st / NS) & 1, abort)) break;
             if (two && !bounded_wait_warp(bar(&ctrl->raw[(st + 1) % NS]), ((st + 1) / NS) & 1, abort)) break;
             const Raw r0 = load_raw(st);
-            const Raw r1 = two ? load_raw(st + 1) : Raw{make_uint4(0u, 0u, 0u, 0u), 0u};
+            const Raw r1 = two ? load_raw(st + 1) : Raw{make_uint4(0u, 0u, 0u, 0u), 0u, 0u};
             expand(st, r0);
             if (two) expand(st + 1, r1);
             fence_proxy_async_smem();
@@ -265,9 +271,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             const int b0 = kb0 + st * S;
             const int nb = min(S, kb0 + Bl - b0);
             if (leader) {
-                int nz = 0;  // affine: groups ending in this stage (each brings its Z row)
-                if (FMT == 1)
-                    for (int k = 0; k < nb; ++k) nz += ((b0 + k) & bpm) == bpm;
                 uint8_t* sp = stage_ptr(slot);
                 const uint32_t rb = bar(&ctrl->raw[slot]);
                 const int e0 = (FMT == 0) ? b0 & ~7 : ((b0 >> bsh)) & ~7;
@@ -277,16 +280,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 tma_load_2d(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
                 if (FMT == 1) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
                 const uint32_t fb = bar(&ctrl->full[slot]);
-                mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK) + nz * TT * 4));
+                mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK + (FMT == 1 ? TT * 16 : 0))));
                 bulk_g2s(smem_addr(sp + OFF_T), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK,
                          uint32_t(nb * T_BLK), fb);
                 bulk_g2s(smem_addr(sp + OFF_DX), dxs + (int64_t(t) * B + b0) * TT, uint32_t(nb * DX_BLK), fb);
-                if (FMT == 1) {
-                    for (int k = 0; k < nb; ++k)
-                        if (((b0 + k) & bpm) == bpm)
-                            bulk_g2s(smem_addr(sp + OFF_Z + k * TT * 4), zb + (int64_t(t) * G + ((b0 + k) >> bsh)) * TT,
-                                     TT * 4, fb);
-                }
+                if (FMT == 1)
+                    bulk_g2s(smem_addr(sp + OFF_XT), xsum + (int64_t(t) * B + b0) * TT, uint32_t(nb * TT * 16), fb);
             }
             __syncwarp();
             issued = st + 1;
@@ -303,6 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
         if (rank == 0) {
             // -------------------------------------------------------- MMA issue (even CTA)
             const uint32_t smem0 = smem_addr(smem);
+            const uint32_t zero_addr = smem0 + uint32_t(Gm::OFF_ZERO);
             for (int st = 0; st < nstages; ++st) {
                 const int slot = st % NS, g = st % NG;
                 if (!bounded_wait_warp(bar(&ctrl->full[slot]), (st / NS) & 1, abort)) break;
@@ -325,6 +325,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                                 const uint64_t td = smem_desc_kmajor(t_addr + h * 256, LBO, SBO);
                                 tc_mma_f16_pair(d, td, wd, Gm::IDESC, (part | h) != 0);
                             }
+                        }
+                        if (FMT == 1) {  // the group bias term; K chunk 1 of both operands is the zero region
+                            const uint32_t xt = smem0 + uint32_t(slot * STAGE_BYTES + OFF_XT + k * TT * 16);
+                            const uint32_t xw = smem0 + uint32_t(slot * STAGE_BYTES + OFF_XW + k * NWH * 16);
+                            tc_mma_f16_pair(d, smem_desc_kmajor(xt, zero_addr - xt, 128),
+                                            smem_desc_kmajor(xw, zero_addr - xw, 128), Gm::IDESC, true);
                         }
                     }
                     tc_commit_pair(bar(&ctrl->tfull[g]), 3);
@@ -362,13 +368,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             if (!bounded_wait_warp(bar(&ctrl->tfull[g]), (st / NG) & 1, abort)) break;
             tc_fence_after();
             const uint8_t* sp = stage_ptr(slot);
-            // Q4_0 needs only d_x from the stage: read it, then hand the stage back to the
-            // copy warp (the stage's MMAs are complete). Affine also reads C and Z at group
-            // ends and releases the stage after the FMAs.
+            // Only d_x is read from the stage: read it, then hand the stage back to the copy
+            // warp (the stage's MMAs are complete).
             float dxv[S];
 #pragma unroll
             for (int k = 0; k < S; ++k) dxv[k] = reinterpret_cast<const float*>(sp + OFF_DX)[k * TT + r];
-            if (FMT == 0) {
+            {
                 const float dep = dxv[0] + dxv[S - 1];  // one warp instruction: waits for the loads
                 __syncwarp();
                 if (lane == 0) mbar_arrive_after(bar(&ctrl->empty[slot]), dep);
@@ -376,10 +381,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
 #pragma unroll
             for (int k = 0; k < S; ++k) {
                 if (k >= nb) break;
-                const int i = kb0 + st * S + k;
                 const bool last = (k == nb - 1);
                 const float dxr = dxv[k];
-                const bool group_end = (FMT == 1) && ((i & bpm) == bpm);
 #pragma unroll
                 for (int h0 = 0; h0 < CW; h0 += LD_COLS) {
                     uint32_t pr[LD_COLS];
@@ -397,22 +400,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
 #pragma unroll
                     for (int j = 0; j < LD_COLS; ++j) acc[h0 + j] = fmaf(__uint_as_float(pr[j]), dxr, acc[h0 + j]);
                 }
-                if (group_end) {  // last block of a group: add (b + 8s) * Z
-                    const float* cs = reinterpret_cast<const float*>(sp + OFF_C) + k * NWT;
-                    const float z = reinterpret_cast<const float*>(sp + OFF_Z)[k * TT + r];
-#pragma unroll
-                    for (int j = 0; j < CW; j += 4) {
-                        const float4 cv = *reinterpret_cast<const float4*>(cs + c0 + j);
-                        acc[j] = fmaf(cv.x, z, acc[j]);
-                        acc[j + 1] = fmaf(cv.y, z, acc[j + 1]);
-                        acc[j + 2] = fmaf(cv.z, z, acc[j + 2]);
-                        acc[j + 3] = fmaf(cv.w, z, acc[j + 3]);
-                    }
-                }
-            }
-            if (FMT == 1) {
-                __syncwarp();  // the values read from the stage were consumed above
-                if (lane == 0) mbar_arrive(bar(&ctrl->empty[slot]));
             }
         }
         if (!*abort) {

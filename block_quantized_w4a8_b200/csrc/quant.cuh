@@ -77,12 +77,14 @@ __global__ void __launch_bounds__(256) quant_act_rowmajor_kernel(const void* __r
 //   FMT 1 (affine): 8c, 8c+4, 8c+2, 8c+6, 8c+1, 8c+5, 8c+3, 8c+7
 // The block scale d goes to `dxs[chunk*tt + r]` (f32). Rows past M are zero (codes and
 // scale). For FMT 1 it also writes, per token and weight group g, Z = the f32 sum over
-// the group's blocks of d*sum(q) (the factor of the bias term), at zb[(t*G + g)*tt + r].
+// the group's blocks of d*sum(q) (the factor of the bias term), at zb[(t*G + g)*tt + r],
+// and, when `sums` is given (128-token tiles), per token and block the 16-byte token
+// column of the CTA-pair GEMM's bias MMA at sums[chunk*tt + r].
 template <bool BF16, int FMT>
 __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restrict__ x, int M, int K, int tt,
                                                            int64_t nblocks, __half* __restrict__ tok,
                                                            float* __restrict__ dxs, float* __restrict__ zb,
-                                                           int group) {
+                                                           int group, uint4* __restrict__ sums) {
     pdl_launch_dependents();
     const int B = K >> 5;
     const int64_t blk = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
@@ -137,6 +139,22 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     if (valid && sub == 0) dxs[chunk * tt + r] = d;
+    if (FMT == 1 && sums) {
+        // The block's two 16-element code sums S1 (lanes 0-3) and S2 (lanes 4-7), |S| <= 2032,
+        // exact in fp16 as are S/2^11: the token column [S1, S2, S1/2^11, S2/2^11, 0, 0, 0, 0]
+        // of the bias MMA of the CTA-pair GEMM (its weight column: b + 8s in two parts).
+        int h = q[0] + q[1] + q[2] + q[3];
+        h += __shfl_xor_sync(0xffffffffu, h, 1);
+        h += __shfl_xor_sync(0xffffffffu, h, 2);
+        const int h2 = __shfl_xor_sync(0xffffffffu, h, 4);
+        if (valid && sub == 0) {
+            const uint32_t p = uint32_t(__half_as_ushort(__int2half_rn(h))) |
+                               (uint32_t(__half_as_ushort(__int2half_rn(h2))) << 16);
+            const uint32_t ps = uint32_t(__half_as_ushort(__float2half_rn(float(h) * 0x1p-11f))) |
+                                (uint32_t(__half_as_ushort(__float2half_rn(float(h2) * 0x1p-11f))) << 16);
+            sums[chunk * tt + r] = make_uint4(p, ps, 0u, 0u);
+        }
+    }
     if (FMT == 1) {
         // Blocks of one weight group are adjacent 8-lane groups of this warp (the warp's
         // four blocks start at a multiple of 4 and B is a multiple of group/32).

@@ -73,6 +73,7 @@ struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
     __half* tok;
     float* dxs;
     float* z;
+    uint4* sums;  // affine, 128-token tiles: per token and block the bias MMA's token column
     int tt;      // tokens per tile
     int tiles;
     size_t bytes;
@@ -89,6 +90,8 @@ TcWs tc_ws(void* ws, int M, int K, int group) {
     w.dxs = reinterpret_cast<float*>(base + off); off = align256(off + size_t(rows) * B * 4);
     w.z = reinterpret_cast<float*>(base + off);
     if (group > 0) off = align256(off + size_t(rows) * (K / group) * 4);
+    w.sums = reinterpret_cast<uint4*>(base + off);
+    if (group > 0 && w.tt == 128) off = align256(off + size_t(rows) * B * 16);
     w.bytes = off;
     return w;
 }
@@ -133,14 +136,16 @@ w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, 
     const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
     if (group == 0) {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0);
+            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0, nullptr);
         else
-            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0);
+            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0, nullptr);
     } else {
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group);
+            quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
+                                                                 w.tt == 128 ? w.sums : nullptr);
         else
-            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group);
+            quant_act_tc_kernel<false, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
+                                                                 w.tt == 128 ? w.sums : nullptr);
     }
     return launch_status();
 }
@@ -394,7 +399,7 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
     const dim3 grid(unsigned(w.tiles), unsigned(cdiv(N, Gm::NWT)), unsigned(sp.ks));
     cudaError_t e = launch_pdl_if(pdl, tc::gemm_pair_kernel<FMT>, grid, dim3(Gm::NUM_THREADS),
                                   size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
-                                  (const float*)w.dxs, (const float*)w.z, y, tq, tsc, tbi, sp.bsplit, part, epi);
+                                  (const float*)w.dxs, (const uint4*)w.sums, y, tq, tsc, tbi, sp.bsplit, part, epi);
     if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
     const int64_t n4 = int64_t(M) * N / 4;
     int64_t rb = cdiv(n4, 256);

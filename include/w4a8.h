@@ -142,7 +142,9 @@ w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int 
  * call. The contraction runs on the original codes: per activation block b inside
  * group g, y += d_x * (s_g * sum q*q_x + b_g * sum q_x). Tolerance as w4a8_gemm.
  * Scale range of the tensor-core path: s = 0 or 2^-17 <= |s| <= 2720 (s * (q - 8) is then
- * exact in fp16); other scales set W4A8_ERR_RANGE as in w4a8_gemm.
+ * exact in fp16), and on its CTA-pair kernel (128-token tiles with K/group a multiple of
+ * 8) also |b + 8s| <= 65504, the bias term's factor being an fp16 operand there; other
+ * values set W4A8_ERR_RANGE as in w4a8_gemm.
  * Arguments and errors as w4a8_gemm, plus `group` (64 or 128).
  */
 w4a8_status w4a8_gemm_affine(int M, int N, int K, int group, const void* x, w4a8_dtype dtype,

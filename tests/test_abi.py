@@ -59,6 +59,8 @@ def test_workspace_bytes(lib, M, N, K, group):
         ntok += ntok % 2
     rows = ntok * tt
     tc = _align(rows * B * 64) + _align(rows * B * 4) + (_align(rows * (K // group) * 4) if group else 0)
+    if group and tt == 128:  # affine on CTA pairs: 16 bytes of code sums per token and block
+        tc += _align(rows * B * 16)
     # split of K when the output tiles do not fill the SMs (148 without a GPU): partial
     # outputs of M*N f32 per split, at least 16 quant blocks per split
     tiles = -(-N // 128) * ntok

@@ -260,6 +260,46 @@ def test_affine_full_size_sampled(wl):
     check_tol(y[ms, ns], yref, T, wl.name)
 
 
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("std,offset", [(1.0, 0.0), (1e-4, 0.0), (0.02, 3000.0), (0.01, -0.05), (1e-3, 2e-5)])
+def test_affine_bias_term_magnitudes(std, offset, group):
+    """The CTA-pair kernel (128-token tiles, K/group a multiple of 8) carries the factor of
+    the group bias term, b + 8s, as two fp16 MMA operands (22 bits of it): weights whose
+    groups put that factor far below or above the codes' term (tiny weights, a large or a
+    small common offset, a factor near zero or in fp16's subnormal range) stay within the
+    tolerance of the oracle, as on the GEMV path."""
+    M, N, K = 300, 256, 1024
+    x = inputs.randn((M, K), seed=31)
+    w = inputs.randn((N, K), seed=32, std=std) + offset
+    rqx, rdx, rsx = oracle.quant_act_q8_0(x.numpy())
+    rq, rs, rb = oracle.pack_affine(w.numpy(), group)
+    yref, T = oracle.gemm_affine(rqx, rdx, rsx, rq, rs, rb, group, nthreads=8)
+    q, s, b = w4a8.pack_affine(dev(w), group)
+    for path in ("gemm", "gemv"):
+        y = as_np(w4a8.gemm_affine(dev(x), q, s, b, group, path=PATHS[path]))
+        assert w4a8.w4a8_last_device_error() == 0
+        check_tol(y, yref, T, f"affine gs{group} std={std} offset={offset} {path}")
+
+
+def test_affine_bias_factor_outside_fp16_is_reported():
+    """A group whose b + 8s exceeds fp16's range cannot be an MMA operand of the CTA-pair
+    kernel: it reports W4A8_ERR_RANGE, while the GEMV path stays within tolerance."""
+    M, N, K, group = 300, 128, 1024, 64
+    x = inputs.randn((M, K), seed=33)
+    w = inputs.randn((N, K), seed=34)
+    w[7, 64:128] += 70000.0  # one group of one row: b + 8s near 7e4
+    rqx, rdx, rsx = oracle.quant_act_q8_0(x.numpy())
+    rq, rs, rb = oracle.pack_affine(w.numpy(), group)
+    yref, T = oracle.gemm_affine(rqx, rdx, rsx, rq, rs, rb, group, nthreads=8)
+    q, s, b = w4a8.pack_affine(dev(w), group)
+    assert w4a8.w4a8_last_device_error() == 0
+    check_tol(as_np(w4a8.gemm_affine(dev(x), q, s, b, group, path=w4a8.PATH_GEMV)), yref, T, "gemv, large bias")
+    assert w4a8.w4a8_last_device_error() == 0
+    w4a8.gemm_affine(dev(x), q, s, b, group, path=w4a8.PATH_GEMM)
+    assert w4a8.w4a8_last_device_error() == 7  # W4A8_ERR_RANGE
+    assert w4a8.w4a8_last_device_error() == 0
+
+
 def test_affine_bias_minus_8s_matches_q4_0_on_gpu():
     """Cross-format invariant on the GPU: affine codes with bias = -8*scale reproduce the
     Q4_0 matmul with d = scale and the same codes."""
