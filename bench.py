@@ -495,8 +495,9 @@ def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
                 tk = entry["tops_kernel"]
                 # The tensor path runs each 32-wide block dot as fp16 MMAs on exact operands:
                 # Q4_0 twice (the weight scale split into two exactly representable parts),
-                # affine once, so the tensor pipe executes `parts` x the useful operations.
-                parts = 1 if affine else 2
+                # affine once plus one K=16 MMA per block for the group bias term (CTA-pair
+                # kernel), so the tensor pipe executes `parts` x the useful operations.
+                parts = 1.5 if affine else 2
                 entry["roofline"] = {"bound": "tensor", "achieved": tk, "unit": "TOP/s",
                                      "peak_int8": int8_peak, "frac_int8": tk / int8_peak,
                                      "mma_f16_tflops_executed": parts * tk, "peak_f16_mma": f16_peak,
