@@ -1,5 +1,5 @@
 """Scalar CPU oracle for the block-quantized W4A8 matmul (Q4_0 x Q8_0) and its affine
-4-bit variant.
+4-, 6- and 8-bit variants.
 
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
 CPU-baseline / reference leg are the only callers. The CUDA library never imports,
@@ -19,8 +19,11 @@ Functions and the definitions they follow (see the header of ``oracle.cpp``):
 * ``gemm_q4_0`` -- y = x . W^T as sum over blocks of d_w * d_x * (exact int block dot),
   in f64 (each term exact), plus T = sum of |terms| (the tolerance scale).
 * ``pack_affine`` / ``gemm_affine`` -- MLX PR #4802 "mx.qqmm ... mode=affine": codes
-  q in [0,15], per-group bf16 scale (max-min)/15 and bias min; the contraction runs on
-  the original codes and applies d_x * (s * sum q q_x + b * sum q_x) per block.
+  q in [0, 2^bits - 1] (bits 4, 6 or 8), per-group (32, 64 or 128) bf16 scale
+  (max-min)/(2^bits - 1) and bias min; the contraction runs on the original codes and
+  applies d_x * (s * sum q q_x + b * sum q_x) per block. Codes of a row are a
+  little-endian bit stream (4 bits: eight codes per 32-bit word, element k at bits
+  4*(k%8) of word k/8).
 * ``epilogue`` -- the output of a linear layer: the optional per-column bias added to
   every row of the f32 product in f32 (C-Kernel-Engine gemm_kernels_q4k.c, "Engine-
   compatible wrapper: GEMM_NT with Q4_K weights"), then f32 or bf16 (nearest even).
@@ -74,10 +77,10 @@ def _load():
         "orc_gemm_q4_0": (None, [I, I, I, P, P, P, P, P, P, I]),
         "orc_gemm_q4_0_sampled": (None, [I, I, P, P, P, P, P, P, P, P]),
         "orc_gemm_q4_0_f32": (None, [I, I, I, P, P, P, P, P]),
-        "orc_pack_affine": (None, [P, I, I, I, P, P, P]),
-        "orc_dequant_affine": (None, [P, P, P, I, I, I, P]),
-        "orc_gemm_affine": (None, [I, I, I, I, P, P, P, P, P, P, P, P, I]),
-        "orc_gemm_affine_sampled": (None, [I, I, I, P, P, P, P, P, P, P, P, P, P]),
+        "orc_pack_affine_bits": (None, [P, I, I, I, I, P, P, P]),
+        "orc_dequant_affine_bits": (None, [P, P, P, I, I, I, I, P]),
+        "orc_gemm_affine_bits": (None, [I, I, I, I, I, P, P, P, P, P, P, P, P, I]),
+        "orc_gemm_affine_bits_sampled": (None, [I, I, I, I, P, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -208,59 +211,73 @@ def gemm_q4_0_f32(qx, dx, qs, d) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------- O5
-def pack_affine(w, group: int) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """W (N, K) f32 -> (q uint32 (N, K/8), scale bf16 bits (N, K/g), bias bf16 bits (N, K/g))."""
+def _codes_bytes(q) -> np.ndarray:
+    """The packed codes as the rows' little-endian byte streams (a 4-bit u32 word array is
+    the same bytes on a little-endian host)."""
+    q = np.ascontiguousarray(q)
+    return q.view(np.uint8).reshape(q.shape[0], -1)
+
+
+def pack_affine(w, group: int, bits: int = 4) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """W (N, K) f32 -> (codes, scale bf16 bits (N, K/g), bias bf16 bits (N, K/g)). The codes
+    are uint32 (N, K/8) words for 4 bits, else uint8 (N, K*bits/8) bytes."""
     w = _f32(w)
     N, K = w.shape
-    assert K % group == 0 and group % 32 == 0
-    q = np.empty((N, K // 8), dtype=np.uint32)
+    assert bits in (4, 6, 8) and K % group == 0 and group % 32 == 0
+    q = np.empty((N, K * bits // 8), dtype=np.uint8)
     s = np.empty((N, K // group), dtype=np.uint16)
     b = np.empty((N, K // group), dtype=np.uint16)
-    _load().orc_pack_affine(_p(w), N, K, int(group), _p(q), _p(s), _p(b))
+    _load().orc_pack_affine_bits(_p(w), N, K, int(group), int(bits), _p(q), _p(s), _p(b))
+    if bits == 4:
+        q = q.view(np.uint32)
     return q, s, b
 
 
-def dequant_affine(q, scale, bias, group: int) -> np.ndarray:
-    q = np.ascontiguousarray(q, dtype=np.uint32)
+def dequant_affine(q, scale, bias, group: int, bits: int = 4) -> np.ndarray:
+    q = _codes_bytes(q)
     N = q.shape[0]
-    K = q.shape[1] * 8
+    K = q.shape[1] * 8 // bits
     out = np.empty((N, K), dtype=np.float64)
-    _load().orc_dequant_affine(_p(q), _p(np.ascontiguousarray(scale, dtype=np.uint16)),
-                               _p(np.ascontiguousarray(bias, dtype=np.uint16)), N, K, int(group), _p(out))
+    _load().orc_dequant_affine_bits(_p(q), _p(np.ascontiguousarray(scale, dtype=np.uint16)),
+                                    _p(np.ascontiguousarray(bias, dtype=np.uint16)), N, K, int(group), int(bits),
+                                    _p(out))
     return out
 
 
 # ----------------------------------------------------------------------------- O6
-def gemm_affine(qx, dx, sx, q, scale, bias, group: int, nthreads: int = 1) -> tuple[np.ndarray, np.ndarray]:
+def gemm_affine(qx, dx, sx, q, scale, bias, group: int, nthreads: int = 1, bits: int = 4
+                ) -> tuple[np.ndarray, np.ndarray]:
     qx = np.ascontiguousarray(qx, dtype=np.int8)
     dx = np.ascontiguousarray(dx, dtype=np.float32)
     sx = np.ascontiguousarray(sx, dtype=np.int32)
-    q = np.ascontiguousarray(q, dtype=np.uint32)
+    q = _codes_bytes(q)
     scale = np.ascontiguousarray(scale, dtype=np.uint16)
     bias = np.ascontiguousarray(bias, dtype=np.uint16)
     M, K = qx.shape
     N = q.shape[0]
-    assert q.shape[1] * 8 == K and scale.shape == (N, K // group) and bias.shape == scale.shape
+    assert q.shape[1] * 8 == K * bits and scale.shape == (N, K // group) and bias.shape == scale.shape
     y = np.empty((M, N), dtype=np.float64)
     T = np.empty((M, N), dtype=np.float64)
-    _load().orc_gemm_affine(M, N, K, int(group), _p(qx), _p(dx), _p(sx), _p(q), _p(scale), _p(bias),
-                            _p(y), _p(T), int(nthreads))
+    _load().orc_gemm_affine_bits(M, N, K, int(group), int(bits), _p(qx), _p(dx), _p(sx), _p(q), _p(scale),
+                                 _p(bias), _p(y), _p(T), int(nthreads))
     return y, T
 
 
-def gemm_affine_sampled(qx, dx, sx, q, scale, bias, group: int, ms, ns) -> tuple[np.ndarray, np.ndarray]:
+def gemm_affine_sampled(qx, dx, sx, q, scale, bias, group: int, ms, ns, bits: int = 4
+                        ) -> tuple[np.ndarray, np.ndarray]:
     qx = np.ascontiguousarray(qx, dtype=np.int8)
     dx = np.ascontiguousarray(dx, dtype=np.float32)
     sx = np.ascontiguousarray(sx, dtype=np.int32)
-    q = np.ascontiguousarray(q, dtype=np.uint32)
+    q = _codes_bytes(q)
     ms = np.ascontiguousarray(ms, dtype=np.int32)
     ns = np.ascontiguousarray(ns, dtype=np.int32)
     K = qx.shape[1]
+    assert q.shape[1] * 8 == K * bits
     y = np.empty(ms.shape, dtype=np.float64)
     T = np.empty(ms.shape, dtype=np.float64)
-    _load().orc_gemm_affine_sampled(K, int(group), ms.size, _p(ms), _p(ns), _p(qx), _p(dx), _p(sx), _p(q),
-                                    _p(np.ascontiguousarray(scale, dtype=np.uint16)),
-                                    _p(np.ascontiguousarray(bias, dtype=np.uint16)), _p(y), _p(T))
+    _load().orc_gemm_affine_bits_sampled(K, int(group), int(bits), ms.size, _p(ms), _p(ns), _p(qx), _p(dx),
+                                         _p(sx), _p(q), _p(np.ascontiguousarray(scale, dtype=np.uint16)),
+                                         _p(np.ascontiguousarray(bias, dtype=np.uint16)), _p(y), _p(T))
     return y, T
 
 

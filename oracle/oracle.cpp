@@ -1,5 +1,5 @@
 // Scalar CPU oracle for block-quantized W4A8 matmul (Q4_0 weights x Q8_0 activations)
-// and its affine 4-bit variant.
+// and its affine 4-, 6- and 8-bit variants.
 //
 // TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call this
 // file; only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
@@ -17,9 +17,9 @@
 //  * The Q4_0 / Q8_0 bit-level encodings (fp16 weight scale d, codes q in [0,15],
 //    w = d*(q-8), low nibbles = elements 0-15 and high nibbles = 16-31 of a block;
 //    activation d = amax/127 in f32, q = round-half-away(x*(1/d)) clamped to +-127).
-//  * MLX PR #4802 "mx.qqmm ... mode=affine": affine 4-bit weights with a per-group scale
-//    and bias; the int8 MMA runs on the original codes and the scale and bias are
-//    applied afterwards (scale = (max-min)/15, bias = min per group of 64 or 128).
+//  * MLX PR #4802 "mx.qqmm ... mode=affine": affine 4-, 6- and 8-bit weights with a
+//    per-group scale and bias; the int8 MMA runs on the original codes and the scale and
+//    bias are applied afterwards (scale = (max-min)/(2^bits - 1), bias = min per group).
 //
 // Readings where the sources leave a step open are marked "Reading:".
 
@@ -304,23 +304,48 @@ void orc_gemm_q4_0_f32(int M, int N, int K, const int8_t* qx, const float* dx, c
 }
 
 // ---------------------------------------------------------------------------------
-// O5. Affine 4-bit weight pack, per row n and group g of `group` (64 or 128)
-//     consecutive elements along K:
+// O5. Affine weight pack with `bits`-bit codes (4, 6 or 8), per row n and group g of
+//     `group` (32, 64 or 128) consecutive elements along K:
 //       mn = min, mx = max (f32)
-//       s  = bf16((mx - mn) / 15),  b = bf16(mn)
-//       q  = s != 0 ? clamp(round_half_away((w - b) / s), 0, 15) : 0   (f32 ops, using
-//            the stored bf16 s and b)
-//     Codes are packed eight per 32-bit word, element i of the row at bits 4*(i%8) of
-//     word i/8. Dequantised weight: s*q + b.
+//       s  = bf16((mx - mn) / (2^bits - 1)),  b = bf16(mn)
+//       q  = s != 0 ? clamp(round_half_away((w - b) / s), 0, 2^bits - 1) : 0   (f32 ops,
+//            using the stored bf16 s and b)
+//     Codes of a row form a little-endian bit stream: element k at bits [bits*k,
+//     bits*k + bits) of the row's K*bits/8 bytes (for 4 bits: eight codes per 32-bit
+//     little-endian word, element k at bits 4*(k%8) of word k/8). Dequantised weight:
+//     s*q + b.
 //     Reading: the codes are computed against the stored (bf16) scale and bias so that
 //     s*q + b is the nearest grid point the kernel can reconstruct; the clamp is needed
-//     because rounding s and b to bf16 can push an end code to -1 or 16.
+//     because rounding s and b to bf16 can push an end code to -1 or 2^bits.
+//     Reading: the pages name 6- and 8-bit codes but not their packing; the bit stream
+//     is the one layout that contains the 4-bit word layout as its special case.
 // ---------------------------------------------------------------------------------
-void orc_pack_affine(const float* w, int N, int K, int group, uint32_t* q_out, uint16_t* scale,
-                     uint16_t* bias) {
+static int64_t affine_row_bytes(int K, int bits) { return int64_t(K) * bits / 8; }
+
+static void put_code(uint8_t* row, int bits, int k, int q) {
+    for (int i = 0; i < bits; ++i) {
+        const int64_t bit = int64_t(k) * bits + i;
+        if ((q >> i) & 1) row[bit / 8] |= uint8_t(1u << (bit % 8));
+    }
+}
+
+static int affine_code(const uint8_t* q, int K, int bits, int n, int k) {
+    const uint8_t* row = q + int64_t(n) * affine_row_bytes(K, bits);
+    int v = 0;
+    for (int i = 0; i < bits; ++i) {
+        const int64_t bit = int64_t(k) * bits + i;
+        v |= ((row[bit / 8] >> (bit % 8)) & 1) << i;
+    }
+    return v;
+}
+
+void orc_pack_affine_bits(const float* w, int N, int K, int group, int bits, uint8_t* q_out, uint16_t* scale,
+                          uint16_t* bias) {
     const int G = K / group;
+    const int qmax = (1 << bits) - 1;
     for (int n = 0; n < N; ++n) {
-        for (int i = 0; i < K / 8; ++i) q_out[int64_t(n) * (K / 8) + i] = 0;
+        uint8_t* row = q_out + int64_t(n) * affine_row_bytes(K, bits);
+        for (int64_t i = 0; i < affine_row_bytes(K, bits); ++i) row[i] = 0;
         for (int g = 0; g < G; ++g) {
             const float* x = w + int64_t(n) * K + int64_t(g) * group;
             float mn = x[0], mx = x[0];
@@ -329,7 +354,7 @@ void orc_pack_affine(const float* w, int N, int K, int group, uint32_t* q_out, u
                 if (x[i] > mx) mx = x[i];
             }
             float range = mx - mn;
-            float sf32 = range / 15.0f;
+            float sf32 = range / float(qmax);
             uint16_t s_bits = orc_f32_to_bf16(sf32);
             uint16_t b_bits = orc_f32_to_bf16(mn);
             float s = orc_bf16_to_f32(s_bits), b = orc_bf16_to_f32(b_bits);
@@ -339,11 +364,10 @@ void orc_pack_affine(const float* w, int N, int K, int group, uint32_t* q_out, u
                     float t = x[i] - b;
                     t = t / s;
                     qi = int(std::round(t));
-                    if (qi > 15) qi = 15;
+                    if (qi > qmax) qi = qmax;
                     if (qi < 0) qi = 0;
                 }
-                const int k = g * group + i;
-                q_out[int64_t(n) * (K / 8) + k / 8] |= uint32_t(qi) << (4 * (k % 8));
+                put_code(row, bits, g * group + i, qi);
             }
             scale[int64_t(n) * G + g] = s_bits;
             bias[int64_t(n) * G + g] = b_bits;
@@ -351,31 +375,27 @@ void orc_pack_affine(const float* w, int N, int K, int group, uint32_t* q_out, u
     }
 }
 
-static int affine_code(const uint32_t* q, int K, int n, int k) {
-    return int((q[int64_t(n) * (K / 8) + k / 8] >> (4 * (k % 8))) & 0xF);
-}
-
-void orc_dequant_affine(const uint32_t* q, const uint16_t* scale, const uint16_t* bias, int N, int K,
-                        int group, double* w_out) {
+void orc_dequant_affine_bits(const uint8_t* q, const uint16_t* scale, const uint16_t* bias, int N, int K,
+                             int group, int bits, double* w_out) {
     const int G = K / group;
     for (int n = 0; n < N; ++n)
         for (int k = 0; k < K; ++k) {
             double s = orc_bf16_to_f32(scale[int64_t(n) * G + k / group]);
             double b = orc_bf16_to_f32(bias[int64_t(n) * G + k / group]);
-            w_out[int64_t(n) * K + k] = s * double(affine_code(q, K, n, k)) + b;
+            w_out[int64_t(n) * K + k] = s * double(affine_code(q, K, bits, n, k)) + b;
         }
 }
 
 // ---------------------------------------------------------------------------------
 // O6. Affine contraction on the original codes. For activation block b (32 wide),
 //     inside weight group g = 32b / group:
-//       D = sum_j q * q_x  (int32),  S = sum_j q_x  (int32, the Q8_0 block sum)
-//       term = d_x*s_g*D + d_x*b_g*S   (each product exact in f64)
+//       D = sum_j q * q_x  (int32, |D| <= 255*127*32),  S = sum_j q_x  (the Q8_0 block sum)
+//       term = d_x*s_g*D + d_x*b_g*S   (each product exact in f64: 8 + 24 + 20 bits)
 //       y = sum of terms (f64), T = sum(|d_x s D| + |d_x b S|)
 //     This is the expansion of sum_k (s q_k + b) (d_x q_x,k) over the block.
 // ---------------------------------------------------------------------------------
-static void gemm_affine_one(int K, int group, int m, int n, const int8_t* qx, const float* dx,
-                            const int32_t* sx, const uint32_t* q, const uint16_t* scale,
+static void gemm_affine_one(int K, int group, int bits, int m, int n, const int8_t* qx, const float* dx,
+                            const int32_t* sx, const uint8_t* q, const uint16_t* scale,
                             const uint16_t* bias, double* y, double* T) {
     const int B = K / 32, G = K / group;
     double acc = 0.0, tabs = 0.0;
@@ -384,7 +404,7 @@ static void gemm_affine_one(int K, int group, int m, int n, const int8_t* qx, co
         int32_t D = 0;
         for (int j = 0; j < 32; ++j) {
             const int k = 32 * b + j;
-            D += affine_code(q, K, n, k) * int32_t(qx[int64_t(m) * K + k]);
+            D += affine_code(q, K, bits, n, k) * int32_t(qx[int64_t(m) * K + k]);
         }
         const int32_t S = sx[int64_t(m) * B + b];
         const double dxv = dx[int64_t(m) * B + b];
@@ -399,21 +419,21 @@ static void gemm_affine_one(int K, int group, int m, int n, const int8_t* qx, co
     if (T) *T = tabs;
 }
 
-void orc_gemm_affine(int M, int N, int K, int group, const int8_t* qx, const float* dx, const int32_t* sx,
-                     const uint32_t* q, const uint16_t* scale, const uint16_t* bias, double* y, double* T,
-                     int nthreads) {
+void orc_gemm_affine_bits(int M, int N, int K, int group, int bits, const int8_t* qx, const float* dx,
+                          const int32_t* sx, const uint8_t* q, const uint16_t* scale, const uint16_t* bias,
+                          double* y, double* T, int nthreads) {
     auto one = [&](int64_t e) {
         const int m = int(e / N), n = int(e % N);
-        gemm_affine_one(K, group, m, n, qx, dx, sx, q, scale, bias, y + e, T ? T + e : nullptr);
+        gemm_affine_one(K, group, bits, m, n, qx, dx, sx, q, scale, bias, y + e, T ? T + e : nullptr);
     };
     parallel_over(int64_t(M) * N, nthreads, one);
 }
 
-void orc_gemm_affine_sampled(int K, int group, int count, const int32_t* ms, const int32_t* ns,
-                             const int8_t* qx, const float* dx, const int32_t* sx, const uint32_t* q,
-                             const uint16_t* scale, const uint16_t* bias, double* y, double* T) {
+void orc_gemm_affine_bits_sampled(int K, int group, int bits, int count, const int32_t* ms, const int32_t* ns,
+                                  const int8_t* qx, const float* dx, const int32_t* sx, const uint8_t* q,
+                                  const uint16_t* scale, const uint16_t* bias, double* y, double* T) {
     for (int i = 0; i < count; ++i)
-        gemm_affine_one(K, group, ms[i], ns[i], qx, dx, sx, q, scale, bias, y + i, T ? T + i : nullptr);
+        gemm_affine_one(K, group, bits, ms[i], ns[i], qx, dx, sx, q, scale, bias, y + i, T ? T + i : nullptr);
 }
 
 }  // extern "C"

@@ -8,6 +8,8 @@ code) so that a layout or indexing mistake in the oracle shows up as a mismatch:
 * Q8_0: x = d * q with one f32 d per 32-block.
 * affine: element k of row n at bits 4*(k%8) of uint32 word k/8; w = s*q + b with bf16
   s and b per group.
+* affine with `bits`-bit codes: the row's bytes read as one little-endian bit stream,
+  element k = bits [bits*k, bits*k + bits).
 """
 import numpy as np
 import torch
@@ -69,3 +71,18 @@ def read_golden(path):
     if rows:
         out["rows"] = rows
     return out
+
+
+def affine_codes_bits(q: np.ndarray, bits: int) -> np.ndarray:
+    qb = np.ascontiguousarray(q).view(np.uint8)
+    N = qb.shape[0]
+    stream = np.unpackbits(qb.reshape(N, -1), axis=1, bitorder="little")  # bit i of byte j at 8j + i
+    K = stream.shape[1] // bits
+    return (stream.reshape(N, K, bits).astype(np.int64) << np.arange(bits)).sum(axis=2)
+
+
+def affine_weights_bits(q: np.ndarray, scale: np.ndarray, bias: np.ndarray, group: int, bits: int) -> np.ndarray:
+    codes = affine_codes_bits(q, bits)
+    s = np.repeat(bf16_bits_to_f64(scale), group, axis=1)
+    b = np.repeat(bf16_bits_to_f64(bias), group, axis=1)
+    return s * codes + b
