@@ -28,7 +28,7 @@ PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 
 EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a8_gemm", "w4a8_gemm_ex",
            "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_gemm_epi", "w4a8_gemm_affine_epi",
-           "w4a8_prepare_act",
+           "w4a8_pack_affine_nbit", "w4a8_gemm_affine_nbit", "w4a8_prepare_act",
            "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_gemm_noalloc", "w4a8_last_device_error",
            "w4a8_last_cuda_error_string", "w4a8_status_string"]
 
@@ -63,6 +63,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_gemm_affine_ex": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, I, P]),
         "w4a8_gemm_epi": (I, [I, I, I, P, I, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
         "w4a8_gemm_affine_epi": (I, [I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
+        "w4a8_pack_affine_nbit": (I, [P, I, I, I, I, I, P, P, P, P]),
+        "w4a8_gemm_affine_nbit": (I, [I, I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
         "w4a8_prepare_act": (I, [I, I, I, P, I, P, Z, I, P]),
         "w4a8_gemm_prepared": (I, [I, I, I, P, P, P, P, Z, I, P]),
         "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
@@ -175,6 +177,26 @@ def w4a8_gemm_affine_epi(x, q, scale, bias_w, y, ws, group: int, bias=None, path
                                                path, _stream(stream)))
 
 
+def w4a8_pack_affine_nbit(w, group: int, bits: int, q, scale, bias, stream=None) -> None:
+    N, K = w.shape
+    _check("w4a8_pack_affine_nbit", load_library().w4a8_pack_affine_nbit(_ptr(w), _dtype(w), N, K, group, bits,
+                                                                         _ptr(q), _ptr(scale), _ptr(bias),
+                                                                         _stream(stream)))
+
+
+def w4a8_gemm_affine_nbit(x, q, scale, bias_w, y, ws, group: int, bits: int, bias=None, path: int = PATH_AUTO,
+                          stream=None) -> None:
+    """Affine weights with 4-, 6- or 8-bit codes (from w4a8_pack_affine_nbit), with the
+    output epilogue (y f32 or bf16; `bias` per column or None)."""
+    M, K = x.shape
+    N = q.shape[0]
+    epi = _epilogue(bias, y.dtype)
+    _check("w4a8_gemm_affine_nbit",
+           load_library().w4a8_gemm_affine_nbit(M, N, K, group, bits, _ptr(x), _dtype(x), _ptr(q), _ptr(scale),
+                                                _ptr(bias_w), ctypes.byref(epi), _ptr(y), _ptr(ws),
+                                                ws.numel() * ws.element_size(), path, _stream(stream)))
+
+
 def w4a8_pack_affine(w, group: int, q, scale, bias, stream=None) -> None:
     N, K = w.shape
     _check("w4a8_pack_affine", load_library().w4a8_pack_affine(_ptr(w), _dtype(w), N, K, group, _ptr(q), _ptr(scale),
@@ -266,6 +288,25 @@ def pack_affine(w: torch.Tensor, group: int, stream=None):
     b = torch.empty(N, K // group, dtype=torch.int16, device=w.device)
     w4a8_pack_affine(w, group, q, s, b, stream)
     return q, s, b
+
+
+def pack_affine_nbit(w: torch.Tensor, group: int, bits: int, stream=None):
+    """Codes as uint8 (N, K*bits/8) little-endian bit streams, scale and bias bf16 bits."""
+    N, K = w.shape
+    q = torch.empty(N, K * bits // 8, dtype=torch.uint8, device=w.device)
+    s = torch.empty(N, K // group, dtype=torch.int16, device=w.device)
+    b = torch.empty(N, K // group, dtype=torch.int16, device=w.device)
+    w4a8_pack_affine_nbit(w, group, bits, q, s, b, stream)
+    return q, s, b
+
+
+def gemm_affine_nbit(x, q, s, b, group: int, bits: int, path: int = PATH_AUTO, ws=None, stream=None):
+    M, K = x.shape
+    N = q.shape[0]
+    y = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    ws = workspace(M, N, K, group, x.device) if ws is None else ws
+    w4a8_gemm_affine_nbit(x, q, s, b, y, ws, group, bits, path=path, stream=stream)
+    return y
 
 
 def workspace(M: int, N: int, K: int, group: int = 0, device="cuda") -> torch.Tensor:

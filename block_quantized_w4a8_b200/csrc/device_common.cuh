@@ -546,6 +546,10 @@ __device__ __forceinline__ float warp_max8(float v) {  // max over aligned group
     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
     return v;
 }
+// log2 of the 32-blocks per affine group (groups of 32, 64 or 128): block index b lies
+// in group b >> group_shift(group), without a run-time division.
+__host__ __device__ __forceinline__ int group_shift(int group) { return group == 128 ? 2 : (group == 64 ? 1 : 0); }
+
 __device__ __forceinline__ int warp_sum8(int v) {
     v += __shfl_xor_sync(0xffffffffu, v, 4);
     v += __shfl_xor_sync(0xffffffffu, v, 2);

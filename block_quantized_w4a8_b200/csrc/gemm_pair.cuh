@@ -126,7 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
     const int nh0 = n0 + int(rank) * NWH;    // the rows this CTA stages
     // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
     // a run-time divisor cost hundreds of cycles on the copy and producer paths.
-    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;
+    const int bsh = (FMT == 1) ? group_shift(group) : 0;
 
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
     auto bar = [](unsigned long long* p) { return smem_addr(p); };

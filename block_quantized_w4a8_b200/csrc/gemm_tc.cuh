@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
     const int t = blockIdx.y;
     // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
     // a run-time divisor cost hundreds of cycles on the copy and producer paths.
-    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;
+    const int bsh = (FMT == 1) ? group_shift(group) : 0;
     const int bpm = (1 << bsh) - 1;  // block index & bpm == bpm: last block of its group
     const int G = (FMT == 1) ? K / group : 0;
 

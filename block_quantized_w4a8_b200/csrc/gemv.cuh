@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(int M, int N, int
     if (n >= N) return;
     const int B = K >> 5;
     const int G = (FMT == 1) ? K / group : 0;
-    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;  // log2(blocks per group): no run-time division
+    const int bsh = (FMT == 1) ? group_shift(group) : 0;  // log2(blocks per group): no run-time division
     const uint4* wrow = reinterpret_cast<const uint4*>(wq + int64_t(n) * (K >> 1));
     float acc[MT];
 #pragma unroll
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kGemv2Threads, 1)
     const int rows_w = (gw < N) ? (N - 1 - gw) / W + 1 : 0;
     const int T = rows_w * C;
     const int G = (FMT == 1) ? K / group : 0;
-    const int bsh = (FMT == 1) ? ((group >> 5) == 4 ? 2 : 1) : 0;  // log2(blocks per group): no run-time division
+    const int bsh = (FMT == 1) ? group_shift(group) : 0;  // log2(blocks per group): no run-time division
 
     struct Item {
         uint4 w[4];
@@ -318,6 +318,123 @@ __global__ void __launch_bounds__(kGemv2Threads, 1)
             process(t + 2, i2);
             if (t + 5 < T) load_item(t + 5, i2);
         }
+    }
+}
+
+}  // namespace w4a8
+
+namespace w4a8 {
+
+// ------------------------------------------------------------------ GEMV, 6- and 8-bit affine codes
+// Same scheme as gemv_kernel (one warp per weight row, lane l takes blocks l, l+32, ...;
+// weights before griddepcontrol.wait, activations after it) for codes of BITS = 6 or 8
+// bits in a little-endian bit stream (24 or 32 bytes per 32-block). The block dot runs
+// on dp4a with the codes widened to one byte each: 8-bit codes as q - 128 (q ^ 0x80 read
+// as a signed byte), so D = dot + 128 * sum(q_x); 6-bit codes (0..63) as they are.
+template <int MT, int BITS>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv_wide_kernel(int M, int N, int K, int group,
+                                                                  const int8_t* __restrict__ qx,
+                                                                  const float* __restrict__ dx,
+                                                                  const int32_t* __restrict__ sx,
+                                                                  const uint8_t* __restrict__ wq,
+                                                                  const uint16_t* __restrict__ wscale,
+                                                                  const uint16_t* __restrict__ wbias,
+                                                                  void* __restrict__ y, Epilogue epi) {
+    static_assert(BITS == 6 || BITS == 8, "code width");
+    constexpr int WORDS = BITS;  // 32-bit words per block (4 * BITS bytes)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = blockIdx.x * kGemvWarps + warp;
+    if (n >= N) return;
+    const int B = K >> 5;
+    const int bsh = group_shift(group);
+    const int G = B >> bsh;
+    const uint8_t* wrow = wq + int64_t(n) * (int64_t(K) * BITS / 8);
+    float acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+    bool waited = false;
+    for (int b0 = 0; b0 < B; b0 += 32 * kGemvUnroll) {
+        uint32_t wv[kGemvUnroll][WORDS];
+        float ws[kGemvUnroll], wb[kGemvUnroll];
+#pragma unroll
+        for (int u = 0; u < kGemvUnroll; ++u) {
+            const int b = b0 + u * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < WORDS; ++i) wv[u][i] = 0u;
+            ws[u] = 0.0f;
+            wb[u] = 0.0f;
+            if (b < B) {
+                if (BITS == 8) {
+                    const uint4* p = reinterpret_cast<const uint4*>(wrow + int64_t(b) * 32);
+                    const uint4 v0 = ld_stream(p), v1 = ld_stream(p + 1);
+                    wv[u][0] = v0.x; wv[u][1] = v0.y; wv[u][2] = v0.z; wv[u][3] = v0.w;
+                    wv[u][4] = v1.x; wv[u][5] = v1.y; wv[u][6] = v1.z; wv[u][7] = v1.w;
+                } else {
+                    const uint2* p = reinterpret_cast<const uint2*>(wrow + int64_t(b) * 24);
+#pragma unroll
+                    for (int i = 0; i < 3; ++i) {
+                        const uint2 v = __ldcs(p + i);
+                        wv[u][2 * i] = v.x;
+                        wv[u][2 * i + 1] = v.y;
+                    }
+                }
+                const int g = b >> bsh;
+                ws[u] = __bfloat162float(__ushort_as_bfloat16(wscale[int64_t(n) * G + g]));
+                wb[u] = __bfloat162float(__ushort_as_bfloat16(wbias[int64_t(n) * G + g]));
+            }
+        }
+        if (!waited) {
+            pdl_wait_primary();
+            waited = true;
+        }
+#pragma unroll
+        for (int u = 0; u < kGemvUnroll; ++u) {
+            const int b = b0 + u * 32 + lane;
+            if (b >= B) continue;
+            uint32_t c[8];  // codes 4i..4i+3 as bytes
+            if (BITS == 8) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) c[i] = wv[u][i] ^ 0x80808080u;
+            } else {
+                // 24-bit groups of four codes at bit 24i of the block's 192-bit stream
+                uint32_t v[8];
+                v[0] = wv[u][0];
+                v[1] = __funnelshift_r(wv[u][0], wv[u][1], 24);
+                v[2] = __funnelshift_r(wv[u][1], wv[u][2], 16);
+                v[3] = wv[u][2] >> 8;
+                v[4] = wv[u][3];
+                v[5] = __funnelshift_r(wv[u][3], wv[u][4], 24);
+                v[6] = __funnelshift_r(wv[u][4], wv[u][5], 16);
+                v[7] = wv[u][5] >> 8;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    c[i] = (v[i] & 0x3Fu) | ((v[i] << 2) & 0x3F00u) | ((v[i] << 4) & 0x3F0000u) |
+                           ((v[i] << 6) & 0x3F000000u);
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m < M) {
+                    const int4* a = reinterpret_cast<const int4*>(qx + int64_t(m) * K + int64_t(b) * 32);
+                    const int4 a0 = a[0], a1 = a[1];
+                    const int aw[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                    int dot = 0;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dot = __dp4a(int(c[i]), aw[i], dot);
+                    const int S = sx[int64_t(m) * B + b];
+                    const float dxv = dx[int64_t(m) * B + b];
+                    const int D = (BITS == 8) ? dot + 128 * S : dot;  // sum q * q_x
+                    const float t = fmaf(ws[u], float(D), __fmul_rn(wb[u], float(S)));
+                    acc[m] = fmaf(dxv, t, acc[m]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        float v = acc[m];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0 && m < M) epi_store(y, int64_t(m) * N + n, n, v, epi);
     }
 }
 

@@ -159,9 +159,9 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         // Blocks of one weight group are adjacent 8-lane groups of this warp (the warp's
         // four blocks start at a multiple of 4 and B is a multiple of group/32).
         float z = __fmul_rn(d, float(s));
-        z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, 8));
+        if (group >= 64) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, 8));
         if (group == 128) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, 16));
-        const int gsh = (group == 128) ? 2 : 1;  // log2(blocks per group)
+        const int gsh = group_shift(group);  // log2(blocks per group)
         if (valid && sub == 0 && (b & ((1 << gsh) - 1)) == 0) {
             const int G = K >> (gsh + 5);
             zb[(t * G + (b >> gsh)) * tt + r] = z;
@@ -209,13 +209,15 @@ __global__ void __launch_bounds__(256) pack_q4_0_kernel(const void* __restrict__
 }
 
 // ------------------------------------------------------------------ affine pack
-// group/4 lanes per group (16 for 64, 32 for 128); groups numbered row-major.
+// group/4 lanes per group (8 for 32, 16 for 64, 32 for 128); groups numbered row-major.
 // min and max keep the first occurrence among equal values (so signed zeros resolve
-// the way a sequential scan does).
-template <bool BF16>
+// the way a sequential scan does). BITS-bit codes (4, 6 or 8) of a row form a
+// little-endian bit stream: element k at bits [BITS*k, BITS*k + BITS) of the row's bytes.
+template <bool BF16, int BITS>
 __global__ void __launch_bounds__(256) pack_affine_kernel(const void* __restrict__ w, int64_t ngroups, int group,
-                                                          uint32_t* __restrict__ q, uint16_t* __restrict__ scale,
+                                                          uint8_t* __restrict__ q, uint16_t* __restrict__ scale,
                                                           uint16_t* __restrict__ bias) {
+    constexpr int QMAX = (1 << BITS) - 1;
     const int L = group >> 2;  // lanes per group (power of two)
     const int64_t gt = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t grp = gt / L;
@@ -239,21 +241,32 @@ __global__ void __launch_bounds__(256) pack_affine_kernel(const void* __restrict
         if (omx > mx || (omx == mx && oimx < imx)) { mx = omx; imx = oimx; }
     }
     const float range = __fsub_rn(mx, mn);
-    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(range, 15.0f));
+    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(range, float(QMAX)));
     const __nv_bfloat16 bb = __float2bfloat16_rn(mn);
     const float sf = __bfloat162float(sb), bf = __bfloat162float(bb);
-    uint32_t mine = 0;
+    uint32_t mine = 0;  // this lane's 4 codes, BITS bits each
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         int qi = 0;
         if (sf != 0.0f) {
             qi = static_cast<int>(roundf(__fdiv_rn(__fsub_rn(v[i], bf), sf)));
-            qi = max(0, min(15, qi));
+            qi = max(0, min(QMAX, qi));
         }
-        mine |= uint32_t(qi) << (4 * i);
+        mine |= uint32_t(qi) << (BITS * i);
     }
-    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-    if (valid && (sub & 1) == 0) q[grp * (group >> 3) + (sub >> 1)] = mine | (other << 16);
+    uint8_t* qg = q + grp * (group * BITS / 8);  // the group's first byte
+    if (BITS == 4) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+        if (valid && (sub & 1) == 0) reinterpret_cast<uint32_t*>(qg)[sub >> 1] = mine | (other << 16);
+    } else if (BITS == 8) {
+        if (valid) reinterpret_cast<uint32_t*>(qg)[sub] = mine;
+    } else {  // 24 bits per lane: 3 bytes
+        if (valid) {
+            qg[sub * 3] = uint8_t(mine);
+            qg[sub * 3 + 1] = uint8_t(mine >> 8);
+            qg[sub * 3 + 2] = uint8_t(mine >> 16);
+        }
+    }
     if (valid && sub == 0) {
         scale[grp] = __bfloat16_as_ushort(sb);
         bias[grp] = __bfloat16_as_ushort(bb);

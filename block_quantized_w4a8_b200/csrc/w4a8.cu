@@ -239,6 +239,35 @@ w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint
     return W4A8_OK;
 }
 
+// GEMV for 6- and 8-bit affine codes from a prepared row-major Q8_0 workspace, in
+// chunks of 8 rows of x.
+template <int BITS>
+w4a8_status run_gemv_wide(int M, int N, int K, int group, const GemvWs& a, const uint8_t* wq, const uint16_t* ws,
+                          const uint16_t* wb, void* y, const Epilogue& epi, cudaStream_t stream) {
+    const int B = K / 32;
+    const dim3 grid(unsigned(cdiv(N, kGemvWarps)));
+    const dim3 block(kGemvWarps * 32);
+    for (int m0 = 0; m0 < M; m0 += 8) {
+        const int mc = (M - m0 < 8) ? (M - m0) : 8;
+        const int mt = gemv_mt(mc);
+        const int8_t* qx = a.qx + int64_t(m0) * K;
+        const float* dx = a.dx + int64_t(m0) * B;
+        const int32_t* sx = a.sx + int64_t(m0) * B;
+        void* yy = static_cast<char*>(y) + int64_t(m0) * N * (epi.out_bf16 ? 2 : 4);
+        cudaError_t e;
+        if (mt == 1)
+            e = launch_pdl(gemv_wide_kernel<1, BITS>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
+        else if (mt == 2)
+            e = launch_pdl(gemv_wide_kernel<2, BITS>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
+        else if (mt == 4)
+            e = launch_pdl(gemv_wide_kernel<4, BITS>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
+        else
+            e = launch_pdl(gemv_wide_kernel<8, BITS>, grid, block, 0, stream, mc, N, K, group, qx, dx, sx, wq, ws, wb, yy, epi);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    return W4A8_OK;
+}
+
 // One-launch GEMV that quantises x itself (requires gemv_fused(M, K)).
 template <int FMT>
 w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
@@ -445,7 +474,7 @@ w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, c
     if (dt != W4A8_F32 && dt != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
     if (path != W4A8_PATH_AUTO && path != W4A8_PATH_GEMV && path != W4A8_PATH_GEMM) return W4A8_ERR_UNSUPPORTED;
     if (affine) {
-        if (group != 64 && group != 128) return W4A8_ERR_UNSUPPORTED;
+        if (group != 32 && group != 64 && group != 128) return W4A8_ERR_UNSUPPORTED;
         if (K % group != 0) return W4A8_ERR_INVALID_ARG;
     }
     if (!aligned16(x) || !aligned16(wq) || !aligned16(ws) || !aligned16(y) || (affine && !aligned16(wb)))
@@ -513,6 +542,48 @@ w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype 
     return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, epi, work, work_bytes, gemv, true, stream);
 }
 
+// Affine 6- and 8-bit codes: the GEMV on a prepared row-major activation for every M
+// (the tensor-core path takes 4-bit codes only; W4A8_PATH_GEMM is refused).
+template <int BITS>
+w4a8_status gemm_wide_impl(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
+                           const uint16_t* ws, const uint16_t* wb, void* y, const Epilogue& epi, void* work,
+                           size_t work_bytes, w4a8_path path, cudaStream_t stream) {
+    w4a8_status st = check_gemm_args(M, N, K, x, dt, wq, ws, wb, true, group, y, work, work_bytes, path);
+    if (st != W4A8_OK) return st;
+    if (path == W4A8_PATH_GEMM) return W4A8_ERR_UNSUPPORTED;
+    st = prepare_impl(M, K, group, x, dt, work, true, stream);
+    if (st != W4A8_OK) return st;
+    return run_gemv_wide<BITS>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, epi, stream);
+}
+
+template <bool BF16>
+void launch_pack_affine(int bits, const void* w, int64_t ngroups, int group, uint8_t* q, uint16_t* scale,
+                        uint16_t* bias, cudaStream_t stream) {
+    const dim3 grid(unsigned(cdiv(ngroups * (group / 4), 256)));
+    if (bits == 4)
+        pack_affine_kernel<BF16, 4><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale, bias);
+    else if (bits == 6)
+        pack_affine_kernel<BF16, 6><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale, bias);
+    else
+        pack_affine_kernel<BF16, 8><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale, bias);
+}
+
+w4a8_status pack_affine_impl(const void* w, w4a8_dtype dtype, int N, int K, int group, int bits, uint8_t* q,
+                             uint16_t* scale_bf16, uint16_t* bias_bf16, cudaStream_t stream) {
+    if (!dims_ok(N, K) || (K % 32) != 0 || !w || !q || !scale_bf16 || !bias_bf16) return W4A8_ERR_INVALID_ARG;
+    if (group != 32 && group != 64 && group != 128) return W4A8_ERR_UNSUPPORTED;
+    if (bits != 4 && bits != 6 && bits != 8) return W4A8_ERR_UNSUPPORTED;
+    if (K % group != 0) return W4A8_ERR_INVALID_ARG;
+    if (dtype != W4A8_F32 && dtype != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
+    if (!aligned16(w) || !aligned16(q) || !aligned16(scale_bf16) || !aligned16(bias_bf16)) return W4A8_ERR_MISALIGNED;
+    const int64_t ngroups = int64_t(N) * (K / group);
+    if (dtype == W4A8_BF16)
+        launch_pack_affine<true>(bits, w, ngroups, group, q, scale_bf16, bias_bf16, stream);
+    else
+        launch_pack_affine<false>(bits, w, ngroups, group, q, scale_bf16, bias_bf16, stream);
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -541,7 +612,7 @@ w4a8_status w4a8_quant_act_q8_0(const void* x, w4a8_dtype dtype, int M, int K, i
 
 size_t w4a8_workspace_bytes(int M, int N, int K, int group) {
     if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 32) != 0) return 0;
-    if (group != 0 && (group != 64 && group != 128)) return 0;
+    if (group != 0 && (group != 32 && group != 64 && group != 128)) return 0;
     if (group != 0 && (K % group) != 0) return 0;
     const size_t a = gemv_ws(nullptr, M, K).bytes;
     const size_t b = tc_ws(nullptr, M, K, group).bytes + partial_bytes(tc_split_pref(M, N, K), M, N);
@@ -561,19 +632,33 @@ w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype, cons
 
 w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int group, uint32_t* q,
                              uint16_t* scale_bf16, uint16_t* bias_bf16, cudaStream_t stream) {
-    if (!dims_ok(N, K) || (K % 32) != 0 || !w || !q || !scale_bf16 || !bias_bf16) return W4A8_ERR_INVALID_ARG;
-    if (group != 64 && group != 128) return W4A8_ERR_UNSUPPORTED;
-    if (K % group != 0) return W4A8_ERR_INVALID_ARG;
-    if (dtype != W4A8_F32 && dtype != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
-    if (!aligned16(w) || !aligned16(q) || !aligned16(scale_bf16) || !aligned16(bias_bf16)) return W4A8_ERR_MISALIGNED;
-    const int64_t ngroups = int64_t(N) * (K / group);
-    const int64_t threads = ngroups * (group / 4);
-    const dim3 grid(unsigned(cdiv(threads, 256)));
-    if (dtype == W4A8_BF16)
-        pack_affine_kernel<true><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale_bf16, bias_bf16);
-    else
-        pack_affine_kernel<false><<<grid, 256, 0, stream>>>(w, ngroups, group, q, scale_bf16, bias_bf16);
-    return launch_status();
+    return pack_affine_impl(w, dtype, N, K, group, 4, reinterpret_cast<uint8_t*>(q), scale_bf16, bias_bf16, stream);
+}
+
+w4a8_status w4a8_pack_affine_nbit(const void* w, w4a8_dtype dtype, int N, int K, int group, int bits, uint8_t* q,
+                                  uint16_t* scale_bf16, uint16_t* bias_bf16, cudaStream_t stream) {
+    return pack_affine_impl(w, dtype, N, K, group, bits, q, scale_bf16, bias_bf16, stream);
+}
+
+w4a8_status w4a8_gemm_affine_nbit(int M, int N, int K, int group, int bits, const void* x, w4a8_dtype dtype,
+                                  const uint8_t* q, const uint16_t* scale_bf16, const uint16_t* bias_bf16,
+                                  const w4a8_epilogue* epi, void* y, void* ws, size_t ws_bytes, w4a8_path path,
+                                  cudaStream_t stream) {
+    Epilogue e;
+    const w4a8_status st = make_epilogue(epi, &e);
+    if (st != W4A8_OK) return st;
+    switch (bits) {
+        case 4:
+            return gemm_impl<1>(M, N, K, group, x, dtype, q, scale_bf16, bias_bf16, y, e, ws, ws_bytes, path, stream);
+        case 6:
+            return gemm_wide_impl<6>(M, N, K, group, x, dtype, q, scale_bf16, bias_bf16, y, e, ws, ws_bytes, path,
+                                     stream);
+        case 8:
+            return gemm_wide_impl<8>(M, N, K, group, x, dtype, q, scale_bf16, bias_bf16, y, e, ws, ws_bytes, path,
+                                     stream);
+        default:
+            return W4A8_ERR_UNSUPPORTED;
+    }
 }
 
 w4a8_status w4a8_gemm_affine_ex(int M, int N, int K, int group, const void* x, w4a8_dtype dtype, const uint32_t* q,

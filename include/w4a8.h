@@ -124,14 +124,14 @@ w4a8_status w4a8_gemm_ex(int M, int N, int K, const void* x, w4a8_dtype dtype,
                          void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream);
 
 /*
- * Affine 4-bit weight pack. Per row n and group g of `group` (64 or 128) elements:
+ * Affine 4-bit weight pack. Per row n and group g of `group` (32, 64 or 128) elements:
  * s = bf16((max - min) / 15), b = bf16(min), q = clamp(round_half_away((w - b) / s), 0, 15)
  * (q = 0 when s == 0), using the stored bf16 s and b. Dequantised weight: s * q + b.
  * w          : N x K row-major, f32 or bf16.
  * q          : out, N x K/8 uint32 words; element k of row n sits at bits 4*(k%8) of
  *              word n*K/8 + k/8.
  * scale_bf16 : out, N x K/group bf16 bit patterns.   bias_bf16 : out, same shape.
- * Errors: INVALID_ARG (also K % group != 0), UNSUPPORTED (group not 64 or 128), MISALIGNED, CUDA.
+ * Errors: INVALID_ARG (also K % group != 0), UNSUPPORTED (group not 32, 64 or 128), MISALIGNED, CUDA.
  */
 w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int group,
                              uint32_t* q, uint16_t* scale_bf16, uint16_t* bias_bf16,
@@ -145,7 +145,7 @@ w4a8_status w4a8_pack_affine(const void* w, w4a8_dtype dtype, int N, int K, int 
  * exact in fp16), and on its CTA-pair kernel (128-token tiles with K/group a multiple of
  * 8) also |b + 8s| <= 65504, the bias term's factor being an fp16 operand there; other
  * values set W4A8_ERR_RANGE as in w4a8_gemm.
- * Arguments and errors as w4a8_gemm, plus `group` (64 or 128).
+ * Arguments and errors as w4a8_gemm, plus `group` (32, 64 or 128).
  */
 w4a8_status w4a8_gemm_affine(int M, int N, int K, int group, const void* x, w4a8_dtype dtype,
                              const uint32_t* q, const uint16_t* scale_bf16,
@@ -197,7 +197,7 @@ w4a8_status w4a8_gemm_affine_epi(int M, int N, int K, int group, const void* x, 
  * ("W4A8MatMul op" measurements) is paid once.
  *  w4a8_prepare_act   quantises x (M x K) into `ws` in the layout of the path that a
  *                     matmul of this M takes (`path` AUTO resolves by M exactly as
- *                     w4a8_gemm does; group = 0 for Q4_0 weights, else 64 or 128).
+ *                     w4a8_gemm does; group = 0 for Q4_0 weights, else 32, 64 or 128).
  *  w4a8_gemm_prepared / w4a8_gemm_affine_prepared
  *                     run only the contraction, reading the quantised activation from
  *                     `ws`. They must be given the same M, K, group and path as the
@@ -213,6 +213,30 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
                                       const uint16_t* scale_bf16, const uint16_t* bias_bf16, float* y,
                                       const void* ws, size_t ws_bytes, w4a8_path path,
                                       cudaStream_t stream);
+
+/*
+ * Affine weights with 4-, 6- or 8-bit codes (MLX PR #4802 "mx.qqmm ... mode=affine": its
+ * int8 kernel takes 4-, 6- and 8-bit affine weights; "Accuracy" gives 6- and 8-bit rows).
+ * Pack, per row n and group g of `group` (32, 64 or 128) elements, with qmax = 2^bits - 1:
+ * s = bf16((max - min) / qmax), b = bf16(min), q = clamp(round_half_away((w - b) / s), 0,
+ * qmax) (q = 0 when s == 0), using the stored bf16 s and b.
+ * q : N x (K*bits/8) bytes; the codes of a row form a little-endian bit stream, element k
+ *     at bits [bits*k, bits*k + bits) of the row's bytes (row n starts at byte
+ *     n*K*bits/8). For bits = 4 this is exactly the layout of w4a8_pack_affine.
+ * scale_bf16, bias_bf16 : out, N x K/group bf16 bit patterns.
+ * w4a8_gemm_affine_nbit computes y = x . W^T exactly as w4a8_gemm_affine does (per
+ * activation block b inside group g: y += d_x * (s_g * sum q*q_x + b_g * sum q_x)), with
+ * the output epilogue of w4a8_gemm_epi (`epi` may be NULL). bits = 4 takes every path of
+ * w4a8_gemm_affine; bits = 6 and 8 run the GEMV kernel for every M (their tensor-core
+ * path is not built: PATH_GEMM returns UNSUPPORTED) and have no scale range limit.
+ * Errors: as w4a8_gemm_affine; UNSUPPORTED also for bits not 4, 6 or 8.
+ */
+w4a8_status w4a8_pack_affine_nbit(const void* w, w4a8_dtype dtype, int N, int K, int group, int bits,
+                                  uint8_t* q, uint16_t* scale_bf16, uint16_t* bias_bf16, cudaStream_t stream);
+w4a8_status w4a8_gemm_affine_nbit(int M, int N, int K, int group, int bits, const void* x, w4a8_dtype dtype,
+                                  const uint8_t* q, const uint16_t* scale_bf16, const uint16_t* bias_bf16,
+                                  const w4a8_epilogue* epi, void* y, void* ws, size_t ws_bytes,
+                                  w4a8_path path, cudaStream_t stream);
 
 /*
  * w4a8_gemm for callers that cannot allocate device memory. Some callers are not allowed

@@ -49,7 +49,8 @@ def _align(v):
 
 
 @pytest.mark.parametrize("M,N,K,group", [(1, 4096, 4096, 0), (64, 1536, 384, 0), (1024, 4096, 4096, 0),
-                                         (1024, 4096, 4096, 64), (1024, 4096, 4096, 128), (300, 333, 800, 0)])
+                                         (1024, 4096, 4096, 64), (1024, 4096, 4096, 128), (300, 333, 800, 0),
+                                         (300, 333, 800, 32), (20, 64, 256, 32)])
 def test_workspace_bytes(lib, M, N, K, group):
     B = K // 32
     gemv = _align(M * K) + _align(M * B * 4) + _align(M * B * 4)
@@ -72,7 +73,7 @@ def test_workspace_bytes(lib, M, N, K, group):
     assert w4a8.w4a8_workspace_bytes(M, N, K, group) == max(gemv, tc)
 
 
-@pytest.mark.parametrize("args", [(0, 16, 32, 0), (16, 16, 33, 0), (16, 16, 64, 32), (16, 16, 96, 64),
+@pytest.mark.parametrize("args", [(0, 16, 32, 0), (16, 16, 33, 0), (16, 16, 64, 16), (16, 16, 96, 64),
                                   (-1, 16, 32, 0), (16, (1 << 20) + 1, 32, 0)])
 def test_workspace_bytes_rejects(lib, args):
     assert w4a8.w4a8_workspace_bytes(*args) == 0
@@ -105,7 +106,7 @@ def test_affine_argument_errors(lib):
     def call(M=8, N=8, K=128, group=64, b=base["b"], dt=0):
         return f(M, N, K, group, base["x"], dt, base["q"], base["s"], b, base["y"], base["ws"], 1 << 40, 0, P(0))
 
-    assert call(group=32) == 2      # only 64 and 128 (the guard of meTile PR #29: bit width / group checked)
+    assert call(group=16) == 2      # only 32, 64 and 128 (the guard of meTile PR #29: bit width / group checked)
     assert call(group=256) == 2
     assert call(K=192, group=128) == 1
     assert call(b=P(0)) == 1
@@ -120,3 +121,23 @@ def test_pack_and_quant_argument_errors(lib):
     assert lib.w4a8_quant_act_q8_0(P(FAKE), 0, 0, 32, P(FAKE), P(FAKE), P(0), P(0)) == 1
     assert lib.w4a8_quant_act_q8_0(P(FAKE), 0, 4, 32, P(FAKE), P(0), P(0), P(0)) == 1
     assert lib.w4a8_quant_act_q8_0(P(FAKE), 0, 4, 32, P(FAKE), P(FAKE), P(FAKE + 4), P(0)) == 6
+
+
+def test_affine_nbit_argument_errors(lib):
+    P = ctypes.c_void_p
+
+    def gemm(bits=6, group=64, path=0, K=128):
+        return lib.w4a8_gemm_affine_nbit(8, 8, K, group, bits, P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), None,
+                                         P(FAKE), P(FAKE), 1 << 40, path, P(0))
+
+    def pack(bits=6, group=64, K=128, q=FAKE):
+        return lib.w4a8_pack_affine_nbit(P(FAKE), 0, 8, K, group, bits, P(q), P(FAKE), P(FAKE), P(0))
+
+    assert gemm(bits=5) == 2 and gemm(bits=16) == 2   # UNSUPPORTED code width
+    assert gemm(group=16) == 2                         # UNSUPPORTED group
+    assert gemm(K=96, group=64) == 1                   # K not a multiple of the group
+    assert gemm(path=2) == 2                           # no tensor-core path for 6/8-bit codes
+    assert gemm(bits=8, path=2) == 2
+    assert pack(bits=7) == 2 and pack(group=256) == 2
+    assert pack(K=96) == 1 and pack(q=0) == 1
+    assert pack(q=FAKE + 8) == 6                       # MISALIGNED
