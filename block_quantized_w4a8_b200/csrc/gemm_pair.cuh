@@ -19,6 +19,15 @@
 // second 8-element K chunk of both operands is a zero region of shared memory. The
 // epilogue is then the same single FMA per output and block as for Q4_0.
 //
+// Affine 6- and 8-bit codes (FMT 3 and 2) read their codes as a little-endian bit stream
+// (one TMA box of both blocks of a stage per row) and widen each code q to the fp16 value
+// 1024 + q with one byte permute per pair. The group scale s is split into two exact
+// parts s_hi + s_lo (its top 4 and low 4 significant bits for 8-bit codes, 5 and 3 for
+// 6-bit) and each part gives (1024 + q) * s_part - (1024 + c) * s_part = (q - c) * s_part
+// (c = 128 or 32) in one fused multiply-add, rounded once to an exactly representable
+// value, so the weight operand has two parts as for Q4_0. The bias column holds
+// C = b + c*s. Exact for s = 0 or 2^-17 <= |s| <= 32.
+//
 // Roles per CTA (448 threads): 8 epilogue warps, 4 producer warps (one thread per (row of
 // the CTA's half, block of the stage), two stages at a time), one MMA warp, one bulk-copy
 // warp. Only the even
@@ -41,7 +50,12 @@ struct PairGeo {
     static constexpr int NWT = 128;                 // weight rows per pair tile (the MMA's N)
     static constexpr int NWH = NWT / 2;             // weight rows each CTA expands and stages
     static constexpr int MN = NWT;                  // TMEM columns per accumulator tile
-    static constexpr int WP = (FMT == 0) ? 2 : 1;   // weight operand parts (hi, lo)
+    static constexpr bool AFF = FMT >= 1;           // affine: group scale and bias, bias MMA
+    static constexpr bool WIDE = FMT >= 2;          // 8-bit (FMT 2) or 6-bit (FMT 3) codes
+    static constexpr int BITS = (FMT == 2) ? 8 : (FMT == 3 ? 6 : 4);
+    static constexpr int BPB = 4 * BITS;            // code bytes per row and block
+    static constexpr int WORDS = BPB / 4;
+    static constexpr int WP = (FMT == 1) ? 1 : 2;   // weight operand parts (hi, lo)
     static constexpr int W_PART = NWH * 64;
     static constexpr int W_BLK = W_PART * WP;
     static constexpr int T_BLK = TT * 64;
@@ -50,12 +64,12 @@ struct PairGeo {
     static constexpr int OFF_T = S * W_BLK;
     static constexpr int OFF_DX = OFF_T + S * T_BLK;
     static constexpr int OFF_XT = align_up(OFF_DX + S * DX_BLK, 128);           // affine: token code sums
-    static constexpr int OFF_XW = OFF_XT + (FMT == 1 ? S * TT * 16 : 0);        // affine: C parts, own half
-    static constexpr int OFF_RAW = align_up(OFF_XW + (FMT == 1 ? S * NWH * 16 : 0), 128);  // codes, own half
-    static constexpr int OFF_RSC = OFF_RAW + S * NWH * 16;                      // scales, all 128 rows
+    static constexpr int OFF_XW = OFF_XT + (AFF ? S * TT * 16 : 0);             // affine: C parts, own half
+    static constexpr int OFF_RAW = align_up(OFF_XW + (AFF ? S * NWH * 16 : 0), 128);  // codes, own half
+    static constexpr int OFF_RSC = OFF_RAW + S * NWH * BPB;                     // scales, all 128 rows
     static constexpr int OFF_RBI = OFF_RSC + NWT * 16;                          // affine biases
-    static constexpr int STAGE_BYTES = align_up(OFF_RBI + (FMT == 1 ? NWT * 16 : 0), 1024);
-    static constexpr int ZERO_BYTES = (FMT == 1) ? TT * 16 : 0;  // zero K chunk of the bias MMA
+    static constexpr int STAGE_BYTES = align_up(OFF_RBI + (AFF ? NWT * 16 : 0), 1024);
+    static constexpr int ZERO_BYTES = AFF ? TT * 16 : 0;  // zero K chunk of the bias MMA
     static constexpr int NS = cmin(8, (SMEM_LIMIT - CTRL_BYTES - ZERO_BYTES - 1024) / STAGE_BYTES);
     static constexpr int OFF_ZERO = NS * STAGE_BYTES + CTRL_BYTES;
     static constexpr int SMEM_BYTES = OFF_ZERO + ZERO_BYTES + 1024;
@@ -126,7 +140,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
     const int nh0 = n0 + int(rank) * NWH;    // the rows this CTA stages
     // Blocks per affine group (2 or 4: group 64 or 128) as a shift: division and modulo by
     // a run-time divisor cost hundreds of cycles on the copy and producer paths.
-    const int bsh = (FMT == 1) ? group_shift(group) : 0;
+    const int bsh = Gm::AFF ? group_shift(group) : 0;
 
     auto stage_ptr = [&](int slot) { return smem + slot * STAGE_BYTES; };
     auto bar = [](unsigned long long* p) { return smem_addr(p); };
@@ -146,7 +160,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
         ctrl->abort = 0;
         mbar_init_fence();
     }
-    if (FMT == 1 && threadIdx.x < Gm::ZERO_BYTES / 16) {
+    if (Gm::AFF && threadIdx.x < Gm::ZERO_BYTES / 16) {
         reinterpret_cast<uint4*>(smem + Gm::OFF_ZERO)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();  // read by the tensor core
     }
@@ -173,21 +187,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
         // before any expanded value is stored (the stores of one stage could alias the next
         // stage's loads, so the loads of both stages are issued first).
         struct Raw {
-            uint4 wv;
+            uint32_t w[Gm::WORDS];  // the codes of this row and block
             uint32_t sb;
             uint32_t bb;  // affine: the group's bias
         };
         auto load_raw = [&](int st) {
-            Raw rw{make_uint4(0u, 0u, 0u, 0u), 0u, 0u};
+            Raw rw;
+#pragma unroll
+            for (int i = 0; i < Gm::WORDS; ++i) rw.w[i] = 0u;
+            rw.sb = 0u;
+            rw.bb = 0u;
             const uint8_t* sp = stage_ptr(st % NS);
             const int sb0 = kb0 + st * S;
             const int e0 = (FMT == 0) ? sb0 & ~7 : ((sb0 >> bsh)) & ~7;  // first scale of the TMA box
             if (st * S + kq < Bl) {
                 const int b = sb0 + kq;
                 const int e = (FMT == 0) ? b : (b >> bsh);
-                rw.wv = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
+                if (Gm::BITS == 4) {  // one 16-byte box row per block
+                    const uint4 v = *reinterpret_cast<const uint4*>(sp + OFF_RAW + kq * NWH * 16 + p * 16);
+                    rw.w[0] = v.x; rw.w[1] = v.y; rw.w[2] = v.z; rw.w[3] = v.w;
+                } else if (Gm::BITS == 8) {  // one box of both blocks: row p at p * 64
+                    const uint4* v = reinterpret_cast<const uint4*>(sp + OFF_RAW + p * (S * 32) + kq * 32);
+                    const uint4 a = v[0], c = v[1];
+                    rw.w[0] = a.x; rw.w[1] = a.y; rw.w[2] = a.z; rw.w[3] = a.w;
+                    rw.w[4] = c.x; rw.w[5] = c.y; rw.w[6] = c.z; rw.w[7] = c.w;
+                } else {  // 6-bit: row p at p * 48, 24 bytes per block
+                    const uint2* v = reinterpret_cast<const uint2*>(sp + OFF_RAW + p * (S * 24) + kq * 24);
+#pragma unroll
+                    for (int i = 0; i < 3; ++i) {
+                        const uint2 a = v[i];
+                        rw.w[2 * i] = a.x;
+                        rw.w[2 * i + 1] = a.y;
+                    }
+                }
                 rw.sb = reinterpret_cast<const uint16_t*>(sp + OFF_RSC + (int(rank) * NWH + p) * 16)[e - e0];
-                if (FMT == 1) rw.bb = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + (int(rank) * NWH + p) * 16)[e - e0];
+                if (Gm::AFF) rw.bb = reinterpret_cast<const uint16_t*>(sp + OFF_RBI + (int(rank) * NWH + p) * 16)[e - e0];
             }
             return rw;
         };
@@ -195,7 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             uint8_t* sp = stage_ptr(st % NS);
             if (st * S + kq < Bl) {
                 const uint32_t sb = rw.sb;
-                const uint32_t w[4] = {rw.wv.x, rw.wv.y, rw.wv.z, rw.wv.w};
+                const uint32_t* w = rw.w;
                 uint8_t* dst = sp + kq * W_BLK + (p >> 3) * 512 + (p & 7) * 16;
                 if (FMT == 0) {
                     range_bad |= (sb & 0x7FF8u) > 0x6950u;  // d_hi > 2720 (24 d_hi > 65504), inf or nan
@@ -216,6 +250,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                             make_uint4(scaled_codes(r[0], l2, l24), scaled_codes(r[1], l2, l24),
                                        scaled_codes(r[2], l2, l24), scaled_codes(r[3], l2, l24));
                     }
+                } else if (Gm::WIDE) {
+                    const float sf = __bfloat162float(__ushort_as_bfloat16(uint16_t(sb)));
+                    const float af = fabsf(sf);
+                    range_bad |= !(af <= 32.0f) || (af != 0.0f && af < 7.62939453125e-06f);  // 2^-17
+                    // s = s_hi + s_lo: the top 4 (8-bit) or 5 (6-bit) significant bits of the
+                    // bf16 scale, and the rest (exact in f32 and in fp16 within the range)
+                    const uint16_t hib = uint16_t(sb) & uint16_t(Gm::BITS == 8 ? 0xFFF0u : 0xFFF8u);
+                    const float shf = __bfloat162float(__ushort_as_bfloat16(hib));
+                    const __half sh = __float2half_rn(shf);
+                    const __half sl = __float2half_rn(__fsub_rn(sf, shf));
+                    const __half off = __float2half(Gm::BITS == 8 ? -1152.0f : -1056.0f);  // -(1024 + c)
+                    const uint32_t h1 = pair_of(sh), hA = pair_of(__hmul(sh, off));
+                    const uint32_t l1 = pair_of(sl), lA = pair_of(__hmul(sl, off));
+                    uint32_t cb[8];  // codes 4i..4i+3 as bytes
+                    if (Gm::BITS == 8) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) cb[i] = w[i];
+                    } else {
+                        uint32_t v[8];  // 24-bit groups of four codes at bit 24i
+                        v[0] = w[0];
+                        v[1] = __funnelshift_r(w[0], w[1], 24);
+                        v[2] = __funnelshift_r(w[1], w[2], 16);
+                        v[3] = w[2] >> 8;
+                        v[4] = w[3];
+                        v[5] = __funnelshift_r(w[3], w[4], 24);
+                        v[6] = __funnelshift_r(w[4], w[5], 16);
+                        v[7] = w[5] >> 8;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            cb[i] = (v[i] & 0x3Fu) | ((v[i] << 2) & 0x3F00u) | ((v[i] << 4) & 0x3F0000u) |
+                                    ((v[i] << 6) & 0x3F000000u);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {  // segment c: codes 8c..8c+7 as fp16 1024 + q
+                        const uint32_t r[4] = {__byte_perm(cb[2 * c], 0x64646464u, 0x4140),
+                                               __byte_perm(cb[2 * c], 0x64646464u, 0x4342),
+                                               __byte_perm(cb[2 * c + 1], 0x64646464u, 0x4140),
+                                               __byte_perm(cb[2 * c + 1], 0x64646464u, 0x4342)};
+                        *reinterpret_cast<uint4*>(dst + c * 128) =
+                            make_uint4(scaled_codes(r[0], h1, hA), scaled_codes(r[1], h1, hA),
+                                       scaled_codes(r[2], h1, hA), scaled_codes(r[3], h1, hA));
+                        *reinterpret_cast<uint4*>(dst + W_PART + c * 128) =
+                            make_uint4(scaled_codes(r[0], l1, lA), scaled_codes(r[1], l1, lA),
+                                       scaled_codes(r[2], l1, lA), scaled_codes(r[3], l1, lA));
+                    }
+                    const float bf = __bfloat162float(__ushort_as_bfloat16(uint16_t(rw.bb)));
+                    const float cf = __fadd_rn(bf, __fmul_rn(Gm::BITS == 8 ? 128.0f : 32.0f, sf));  // b + c*s
+                    range_bad |= !(fabsf(cf) <= 65504.0f);
+                    const __half ch = __float2half_rn(cf);
+                    const __half cl = __float2half_rn(__fmul_rn(__fsub_rn(cf, __half2float(ch)), 2048.0f));
+                    *reinterpret_cast<uint4*>(sp + OFF_XW + kq * NWH * 16 + p * 16) =
+                        make_uint4(pair_of(ch), pair_of(cl), 0u, 0u);
                 } else {
                     const float sf = __bfloat162float(__ushort_as_bfloat16(uint16_t(sb)));
                     const float af = fabsf(sf);
@@ -249,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
             if (!bounded_wait_warp(bar(&ctrl->raw[st % NS]), (st / NS) & 1, abort)) break;
             if (two && !bounded_wait_warp(bar(&ctrl->raw[(st + 1) % NS]), ((st + 1) / NS) & 1, abort)) break;
             const Raw r0 = load_raw(st);
-            const Raw r1 = two ? load_raw(st + 1) : Raw{make_uint4(0u, 0u, 0u, 0u), 0u, 0u};
+            const Raw r1 = load_raw(two ? st + 1 : nstages);  // past the end: zeros
             expand(st, r0);
             if (two) expand(st + 1, r1);
             fence_proxy_async_smem();
@@ -274,17 +360,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 uint8_t* sp = stage_ptr(slot);
                 const uint32_t rb = bar(&ctrl->raw[slot]);
                 const int e0 = (FMT == 0) ? b0 & ~7 : ((b0 >> bsh)) & ~7;
-                mbar_arrive_expect_tx(rb, uint32_t(nb * NWH * 16 + NWT * 16 * (FMT == 1 ? 2 : 1)));
-                for (int k = 0; k < nb; ++k)
-                    tma_load_2d(smem_addr(sp + OFF_RAW + k * NWH * 16), &tm_q, (b0 + k) * 16, nh0, rb);
+                if (Gm::BITS == 4) {  // a box of 16 bytes x 64 rows per block
+                    mbar_arrive_expect_tx(rb, uint32_t(nb * NWH * 16 + NWT * 16 * (Gm::AFF ? 2 : 1)));
+                    for (int k = 0; k < nb; ++k)
+                        tma_load_2d(smem_addr(sp + OFF_RAW + k * NWH * 16), &tm_q, (b0 + k) * 16, nh0, rb);
+                } else {  // one box of both blocks (b0 is even: its byte offset is a multiple of 16)
+                    mbar_arrive_expect_tx(rb, uint32_t(S * Gm::BPB * NWH + NWT * 16 * 2));
+                    tma_load_2d(smem_addr(sp + OFF_RAW), &tm_q, b0 * Gm::BPB, nh0, rb);
+                }
                 tma_load_2d(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
-                if (FMT == 1) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
+                if (Gm::AFF) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
                 const uint32_t fb = bar(&ctrl->full[slot]);
-                mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK + (FMT == 1 ? TT * 16 : 0))));
+                mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK + (Gm::AFF ? TT * 16 : 0))));
                 bulk_g2s(smem_addr(sp + OFF_T), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK,
                          uint32_t(nb * T_BLK), fb);
                 bulk_g2s(smem_addr(sp + OFF_DX), dxs + (int64_t(t) * B + b0) * TT, uint32_t(nb * DX_BLK), fb);
-                if (FMT == 1)
+                if (Gm::AFF)
                     bulk_g2s(smem_addr(sp + OFF_XT), xsum + (int64_t(t) * B + b0) * TT, uint32_t(nb * TT * 16), fb);
             }
             __syncwarp();
@@ -326,7 +417,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                                 tc_mma_f16_pair(d, td, wd, Gm::IDESC, (part | h) != 0);
                             }
                         }
-                        if (FMT == 1) {  // the group bias term; K chunk 1 of both operands is the zero region
+                        if (Gm::AFF) {  // the group bias term; K chunk 1 of both operands is the zero region
                             const uint32_t xt = smem0 + uint32_t(slot * STAGE_BYTES + OFF_XT + k * TT * 16);
                             const uint32_t xw = smem0 + uint32_t(slot * STAGE_BYTES + OFF_XW + k * NWH * 16);
                             tc_mma_f16_pair(d, smem_desc_kmajor(xt, zero_addr - xt, 128),

@@ -75,8 +75,9 @@ __global__ void __launch_bounds__(256) quant_act_rowmajor_kernel(const void* __r
 // the block, applied identically to both operands, so every block dot is unchanged):
 //   FMT 0 (Q4_0):   4c, 4c+2, 4c+1, 4c+3, 16+4c, 16+4c+2, 16+4c+1, 16+4c+3
 //   FMT 1 (affine): 8c, 8c+4, 8c+2, 8c+6, 8c+1, 8c+5, 8c+3, 8c+7
+//   FMT 2 (affine 6- and 8-bit codes): 8c, 8c+1, ..., 8c+7
 // The block scale d goes to `dxs[chunk*tt + r]` (f32). Rows past M are zero (codes and
-// scale). For FMT 1 it also writes, per token and weight group g, Z = the f32 sum over
+// scale). For FMT 1 and 2 it also writes, per token and weight group g, Z = the f32 sum over
 // the group's blocks of d*sum(q) (the factor of the bias term), at zb[(t*G + g)*tt + r],
 // and, when `sums` is given (128-token tiles), per token and block the 16-byte token
 // column of the CTA-pair GEMM's bias MMA at sums[chunk*tt + r].
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
     const uint32_t mine = (uint32_t(q[0]) & 0xFFu) | ((uint32_t(q[1]) & 0xFFu) << 8) |
                           ((uint32_t(q[2]) & 0xFFu) << 16) | ((uint32_t(q[3]) & 0xFFu) << 24);
     const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, FMT == 0 ? 4 : 1);
+    static_assert(FMT >= 0 && FMT <= 2, "token operand order");
     auto code = [](uint32_t w, int i) { return int(int8_t((w >> (8 * i)) & 0xFFu)); };
     const int64_t t = m / tt;
     const int r = int(m - t * tt);
@@ -123,9 +125,12 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         if (FMT == 0) {  // own = elements 4c..4c+3, other = 16+4c..16+4c+3
             e[0] = code(mine, 0); e[1] = code(mine, 2); e[2] = code(mine, 1); e[3] = code(mine, 3);
             e[4] = code(other, 0); e[5] = code(other, 2); e[6] = code(other, 1); e[7] = code(other, 3);
-        } else {         // own = elements 8c..8c+3, other = 8c+4..8c+7
+        } else if (FMT == 1) {  // own = elements 8c..8c+3, other = 8c+4..8c+7
             e[0] = code(mine, 0); e[1] = code(other, 0); e[2] = code(mine, 2); e[3] = code(other, 2);
             e[4] = code(mine, 1); e[5] = code(other, 1); e[6] = code(mine, 3); e[7] = code(other, 3);
+        } else {                // element order
+            e[0] = code(mine, 0); e[1] = code(mine, 1); e[2] = code(mine, 2); e[3] = code(mine, 3);
+            e[4] = code(other, 0); e[5] = code(other, 1); e[6] = code(other, 2); e[7] = code(other, 3);
         }
         uint32_t h[4];
 #pragma unroll
@@ -139,7 +144,7 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
         *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     if (valid && sub == 0) dxs[chunk * tt + r] = d;
-    if (FMT == 1 && sums) {
+    if (FMT >= 1 && sums) {
         // The block's two 16-element code sums S1 (lanes 0-3) and S2 (lanes 4-7), |S| <= 2032,
         // exact in fp16 as are S/2^11: the token column [S1, S2, S1/2^11, S2/2^11, 0, 0, 0, 0]
         // of the bias MMA of the CTA-pair GEMM (its weight column: b + 8s in two parts).
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
             sums[chunk * tt + r] = make_uint4(p, ps, 0u, 0u);
         }
     }
-    if (FMT == 1) {
+    if (FMT >= 1) {
         // Blocks of one weight group are adjacent 8-lane groups of this warp (the warp's
         // four blocks start at a multiple of 4 and B is a multiple of group/32).
         float z = __fmul_rn(d, float(s));

@@ -131,10 +131,19 @@ w4a8_status run_quant_rowmajor(const void* x, w4a8_dtype dt, int M, int K, int8_
     return launch_status();
 }
 
-w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, const TcWs& w, cudaStream_t stream) {
+// `wide`: the token order of the 6- and 8-bit affine weight expansion (element order).
+w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, const TcWs& w, cudaStream_t stream,
+                         bool wide = false) {
     const int64_t nblocks = int64_t(w.tiles) * w.tt * (K / 32);
     const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
-    if (group == 0) {
+    if (wide) {
+        if (dt == W4A8_BF16)
+            quant_act_tc_kernel<true, 2><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
+                                                                 w.sums);
+        else
+            quant_act_tc_kernel<false, 2><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
+                                                                  w.sums);
+    } else if (group == 0) {
         if (dt == W4A8_BF16)
             quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0, nullptr);
         else
@@ -415,12 +424,14 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
     CUtensorMap tq, tsc, tbi;
     memset(&tbi, 0, sizeof(tbi));
     const int E = (FMT == 0) ? K / 32 : K / group;  // scales per row (a multiple of 8 here)
-    if (!encode_2d(&tq, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 16,
-                   Gm::NWH) ||
+    // codes: rows of K*BITS/8 bytes; 4-bit boxes of one block, wider codes one box per stage
+    const uint64_t row_bytes = uint64_t(K) * Gm::BITS / 8;
+    if (!encode_2d(&tq, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, row_bytes, uint64_t(N), row_bytes,
+                   Gm::BITS == 4 ? 16 : Gm::S * Gm::BPB, Gm::NWH) ||
         !encode_2d(&tsc, ws, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N), uint64_t(E) * 2, 8,
                    Gm::NWT))
         return W4A8_ERR_CUDA;
-    if (FMT == 1 && !encode_2d(&tbi, wb, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N),
+    if (FMT >= 1 && !encode_2d(&tbi, wb, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(E), uint64_t(N),
                                uint64_t(E) * 2, 8, Gm::NWT))
         return W4A8_ERR_CUDA;
     const KSplit sp = tc_split(M, N, K, w.bytes, work_bytes);
@@ -542,15 +553,29 @@ w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype 
     return contract_impl<FMT>(M, N, K, group, wq, ws, wb, y, epi, work, work_bytes, gemv, true, stream);
 }
 
-// Affine 6- and 8-bit codes: the GEMV on a prepared row-major activation for every M
-// (the tensor-core path takes 4-bit codes only; W4A8_PATH_GEMM is refused).
+// True when the CTA-pair kernel takes 6- or 8-bit codes of this shape: 128-token tiles
+// (M > 64), scale rows and code rows whose pitch is a multiple of 16 bytes (TMA).
+inline bool wide_pair_ok(int M, int K, int group, int bits) {
+    return tc_token_tile(M) == 128 && ((K / group) * 2) % 16 == 0 && (int64_t(K) * bits / 8) % 16 == 0;
+}
+
+// Affine 6- and 8-bit codes: CTA pairs for M > 64 (AUTO or PATH_GEMM, shapes of
+// wide_pair_ok), the GEMV on a prepared row-major activation otherwise (PATH_GEMM on
+// other shapes is refused: there is no small-M tensor kernel for these codes).
 template <int BITS>
 w4a8_status gemm_wide_impl(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
                            const uint16_t* ws, const uint16_t* wb, void* y, const Epilogue& epi, void* work,
                            size_t work_bytes, w4a8_path path, cudaStream_t stream) {
     w4a8_status st = check_gemm_args(M, N, K, x, dt, wq, ws, wb, true, group, y, work, work_bytes, path);
     if (st != W4A8_OK) return st;
-    if (path == W4A8_PATH_GEMM) return W4A8_ERR_UNSUPPORTED;
+    const bool pair_ok = wide_pair_ok(M, K, group, BITS);
+    if (path == W4A8_PATH_GEMM && !pair_ok) return W4A8_ERR_UNSUPPORTED;
+    if (pair_ok && path != W4A8_PATH_GEMV && M > kGemvMaxM) {
+        const TcWs w = tc_ws(work, M, K, group);
+        st = run_quant_tc(x, dt, M, K, group, w, stream, true);
+        if (st != W4A8_OK) return st;
+        return launch_gemm_pair<BITS == 8 ? 2 : 3>(M, N, K, group, w, wq, ws, wb, y, epi, true, work_bytes, stream);
+    }
     st = prepare_impl(M, K, group, x, dt, work, true, stream);
     if (st != W4A8_OK) return st;
     return run_gemv_wide<BITS>(M, N, K, group, gemv_ws(work, M, K), wq, ws, wb, y, epi, stream);

@@ -227,8 +227,11 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
  * w4a8_gemm_affine_nbit computes y = x . W^T exactly as w4a8_gemm_affine does (per
  * activation block b inside group g: y += d_x * (s_g * sum q*q_x + b_g * sum q_x)), with
  * the output epilogue of w4a8_gemm_epi (`epi` may be NULL). bits = 4 takes every path of
- * w4a8_gemm_affine; bits = 6 and 8 run the GEMV kernel for every M (their tensor-core
- * path is not built: PATH_GEMM returns UNSUPPORTED) and have no scale range limit.
+ * w4a8_gemm_affine. bits = 6 and 8: M > 64 with K/group a multiple of 8 and K*bits/8 a
+ * multiple of 16 runs the CTA-pair tensor-core kernel (AUTO or PATH_GEMM), which holds
+ * the weights exactly for s = 0 or 2^-17 <= |s| <= 32 and |b + c*s| <= 65504 (c =
+ * 2^(bits-1)); other values set W4A8_ERR_RANGE in the device status word. Every other
+ * shape runs the GEMV (no range limit); PATH_GEMM there returns UNSUPPORTED.
  * Errors: as w4a8_gemm_affine; UNSUPPORTED also for bits not 4, 6 or 8.
  */
 w4a8_status w4a8_pack_affine_nbit(const void* w, w4a8_dtype dtype, int N, int K, int group, int bits,

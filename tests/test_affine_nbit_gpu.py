@@ -1,7 +1,9 @@
 """Affine weights with 6- and 8-bit codes and with groups of 32 on the GPU, against the
 oracle: the pack bit for bit (codes, scales, biases), the contraction element by element
-within the tolerance of the 4-bit paths (|y - y_ref| <= 1e-5 * T), with and without the
-output epilogue, on ragged shapes; 4-bit codes in groups of 32 on every kernel path."""
+within the tolerance of the 4-bit paths (|y - y_ref| <= 1e-5 * T) on the GEMV and on the
+CTA-pair tensor-core kernel (with and without a split of K), with and without the output
+epilogue, on ragged shapes; the scale range of the tensor path; 4-bit codes in groups of
+32 on every kernel path."""
 import numpy as np
 import pytest
 import torch
@@ -42,8 +44,15 @@ def test_pack_nbit_bitwise(bits, group, dtype):
 
 
 # (M, N, K): single token, a few tokens, ragged N, K with a tail of 32-blocks that does not
-# fill a lane's last unrolled step, more rows than one GEMV chunk (8), larger M
-SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (13, 129, 384), (40, 200, 1280), (130, 96, 4096)]
+# fill a lane's last unrolled step, more rows than one GEMV chunk (8); M > 64 takes CTA
+# pairs (a padded pair for 130 rows, ragged N tiles, a split of K for 200 x 512 x 4096)
+# where K/group is a multiple of 8, and the GEMV otherwise
+SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (13, 129, 384), (40, 200, 1280), (130, 96, 4096),
+          (300, 333, 1024), (200, 512, 4096), (256, 160, 2048), (100, 64, 640)]
+
+
+def _pair_ok(M, K, group, bits):
+    return M > 64 and (K // group) % 8 == 0 and (K * bits // 8) % 16 == 0
 
 
 @pytest.mark.parametrize("group", [32, 64, 128])
@@ -58,14 +67,17 @@ def test_gemm_affine_nbit_vs_oracle(M, N, K, bits, group):
     rq, rs, rb = oracle.pack_affine(w.numpy(), group, bits=bits)
     yref, T = oracle.gemm_affine(rqx, rdx, rsx, rq, rs, rb, group, nthreads=8, bits=bits)
     q, s, b = w4a8.pack_affine_nbit(w.cuda(), group, bits)
-    y = as_np(w4a8.gemm_affine_nbit(x.cuda(), q, s, b, group, bits))
-    assert w4a8.w4a8_last_device_error() == 0
-    check_tol(y, yref, T, f"affine {bits}-bit gs{group} M={M} N={N} K={K}")
+    paths = ["auto", "gemv"] + (["gemm"] if _pair_ok(M, K, group, bits) else [])
+    for path in paths:
+        y = as_np(w4a8.gemm_affine_nbit(x.cuda(), q, s, b, group, bits, path=PATHS[path]))
+        assert w4a8.w4a8_last_device_error() == 0
+        check_tol(y, yref, T, f"affine {bits}-bit gs{group} M={M} N={N} K={K} {path}")
 
 
 @pytest.mark.parametrize("bits", [6, 8])
-def test_gemm_affine_nbit_epilogue(bits):
-    M, N, K, group = 5, 300, 1024, 64
+@pytest.mark.parametrize("M", [5, 300])
+def test_gemm_affine_nbit_epilogue(bits, M):
+    N, K, group = 300, 1024, 64
     wl = inputs.Workload("nbit_epi", M=M, K=K, N=N, seed=5 + bits)
     x, w = inputs.make(wl)
     rqx, rdx, rsx = oracle.quant_act_q8_0(x.float().numpy())
@@ -83,12 +95,52 @@ def test_gemm_affine_nbit_epilogue(bits):
     assert np.all(np.abs(yv - rv) <= TOL * T + np.abs(rv) * 2.0 ** -7)
 
 
-def test_gemm_affine_nbit_tensor_path_is_refused():
-    x = torch.randn(200, 256, device="cuda")
-    q, s, b = w4a8.pack_affine_nbit(torch.randn(64, 256, device="cuda"), 64, 8)
+@pytest.mark.parametrize("M,K", [(40, 1024), (200, 256)])
+def test_gemm_affine_nbit_tensor_path_is_refused(M, K):
+    """No tensor kernel for 6/8-bit codes at M <= 64, nor when K/group is not a multiple of
+    8 (the scale rows' pitch): PATH_GEMM is refused there (AUTO takes the GEMV)."""
+    x = torch.randn(M, K, device="cuda")
+    q, s, b = w4a8.pack_affine_nbit(torch.randn(64, K, device="cuda"), 64, 8)
     with pytest.raises(w4a8.W4A8Error) as e:
         w4a8.gemm_affine_nbit(x, q, s, b, 64, 8, path=w4a8.PATH_GEMM)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_wide_scale_outside_tensor_range_is_reported(bits):
+    """A group scale above 32 cannot be split into the CTA-pair kernel's exact fp16 parts
+    for 6/8-bit codes: W4A8_ERR_RANGE, while the GEMV path stays within tolerance."""
+    M, N, K, group = 200, 128, 1024, 64
+    x = inputs.randn((M, K), seed=51)
+    w = inputs.randn((N, K), seed=52)
+    w[9, :64] *= 4000.0  # scale near 4000 * 6 / 2^bits
+    rqx, rdx, rsx = oracle.quant_act_q8_0(x.numpy())
+    rq, rs, rb = oracle.pack_affine(w.numpy(), group, bits=bits)
+    yref, T = oracle.gemm_affine(rqx, rdx, rsx, rq, rs, rb, group, nthreads=8, bits=bits)
+    q, s, b = w4a8.pack_affine_nbit(w.cuda(), group, bits)
+    assert w4a8.w4a8_last_device_error() == 0
+    check_tol(as_np(w4a8.gemm_affine_nbit(x.cuda(), q, s, b, group, bits, path=w4a8.PATH_GEMV)), yref, T, "gemv")
+    assert w4a8.w4a8_last_device_error() == 0
+    w4a8.gemm_affine_nbit(x.cuda(), q, s, b, group, bits, path=w4a8.PATH_GEMM)
+    assert w4a8.w4a8_last_device_error() == 7  # W4A8_ERR_RANGE
+    assert w4a8.w4a8_last_device_error() == 0
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+@pytest.mark.parametrize("std,offset", [(1e-3, 0.0), (0.02, 500.0), (1.0, -3.0)])
+def test_wide_bias_term_magnitudes(bits, std, offset):
+    """Bias factors b + c*s near zero, in fp16's subnormal range and at large offsets on
+    the CTA-pair kernel for 6/8-bit codes."""
+    M, N, K, group = 300, 256, 1024, 64
+    x = inputs.randn((M, K), seed=61)
+    w = inputs.randn((N, K), seed=62, std=std) + offset
+    rqx, rdx, rsx = oracle.quant_act_q8_0(x.numpy())
+    rq, rs, rb = oracle.pack_affine(w.numpy(), group, bits=bits)
+    yref, T = oracle.gemm_affine(rqx, rdx, rsx, rq, rs, rb, group, nthreads=8, bits=bits)
+    q, s, b = w4a8.pack_affine_nbit(w.cuda(), group, bits)
+    y = as_np(w4a8.gemm_affine_nbit(x.cuda(), q, s, b, group, bits, path=w4a8.PATH_GEMM))
+    assert w4a8.w4a8_last_device_error() == 0
+    check_tol(y, yref, T, f"{bits}-bit std={std} offset={offset}")
 
 
 def test_nbit_4bit_equals_affine_entry():
