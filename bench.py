@@ -51,7 +51,8 @@ def parse_args():
     ap.add_argument("--sweep", choices=["some", "all", "none"], default="some")
     ap.add_argument("--probe", default=None,
                     help="profiling probe: run `--steps` calls of one workload (decode, minilm, prefill, affine64, "
-                         "affine128, or MxKxN) through w4a8_gemm[_affine], then exit without timing")
+                         "affine128, affine6_64, affine8_64, or MxKxN) through w4a8_gemm[_affine[_nbit]], then exit "
+                         "without timing")
     return ap.parse_args()
 
 
@@ -507,6 +508,7 @@ def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
         del sets
         torch.cuda.empty_cache()
     results += run_epilogue(args, torch, w4a8, oracle, inputs, steps, dev)
+    results += run_wide(args, torch, w4a8, oracle, inputs, steps, dev, int8_peak)
     return results
 
 
@@ -561,6 +563,52 @@ def run_epilogue(args, torch, w4a8, oracle, inputs, steps, dev):
     return out
 
 
+def run_wide(args, torch, w4a8, oracle, inputs, steps, dev, int8_peak):
+    """Affine weights with 6- and 8-bit codes (w4a8_gemm_affine_nbit) on the MLX page's
+    setup (M=1024, K=N=4096, bf16 x, normal weights; groups of 64 and 128) and a decode
+    GEMV line, each parity-checked on sampled outputs before it is timed. Per call,
+    including the activation quantisation."""
+    import numpy as np
+    out = []
+    cases = [(1024, 6, 64), (1024, 8, 64), (1024, 8, 128), (1, 8, 64)]
+    for M, bits, group in cases:
+        N = K = 4096
+        wl = inputs.Workload(f"affine{bits}_m{M}_{K}x{N}_gs{group}", M=M, K=K, N=N, x_dtype="bf16", w_std=1.0,
+                             kind="affine", group=group)
+        x, w = inputs.make(wl)
+        xd = x.to(dev)
+        q, s, b = w4a8.pack_affine_nbit(w.to(dev), group, bits)
+        wbytes = N * K * bits // 8 + 2 * N * (K // group) * 2
+        R = copies_for(wbytes)
+        sets = [(q.clone(), s.clone(), b.clone()) for _ in range(R)]
+        ws = w4a8.workspace(M, N, K, group, dev)
+        y = torch.empty(M, N, device=dev)
+        w4a8.w4a8_gemm_affine_nbit(xd, q, s, b, y, ws, group, bits)
+        torch.cuda.synchronize()
+        rqx, rdx, rsx = oracle.quant_act_q8_0(x.float().numpy())
+        rq, rs, rb = oracle.pack_affine(w.numpy(), group, bits=bits)
+        ok = check_parity_sampled(y, lambda ms, ns: oracle.gemm_affine_sampled(
+            rqx, rdx, rsx, rq, rs, rb, group, np.asarray(ms), np.asarray(ns), bits=bits), M, N)
+        entry = {"workload": wl.name, "M": M, "N": N, "K": K, "bits": bits, "group": group,
+                 "path": "gemv" if M <= 8 else "gemm_pair", "parity": "pass" if ok else "FAIL"}
+        if ok:
+            def step(i):
+                qq, ss, bb = sets[i % R]
+                w4a8.w4a8_gemm_affine_nbit(xd, qq, ss, bb, y, ws, group, bits)
+            for i in range(3):
+                step(i)
+            us = timed(step, steps, torch, graph=True) / steps * 1e3
+            tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            entry.update({"us_per_call": us, "tops_call": tops, "weight_gbs_call": wbytes / (us * 1e-6) / 1e9,
+                          "l2": f"{R} rotating weight copies"})
+            if M > 8:
+                entry["frac_int8_call"] = tops / int8_peak
+        out.append(entry)
+        del sets
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_probe(args):
     """A short, fixed sequence of launches for ncu: `--steps` calls of w4a8_gemm (or
     w4a8_gemm_affine) through the C ABI on the workload named by --probe."""
@@ -569,7 +617,13 @@ def run_probe(args):
     from block_quantized_w4a8_b200 import inputs
     named = {"decode": inputs.DECODE, "minilm": inputs.MINILM, "prefill": inputs.PREFILL,
              "affine64": inputs.AFFINE_GS64, "affine128": inputs.AFFINE_GS128}
-    if args.probe in named:
+    wide = {"affine6_64": (6, 64), "affine8_64": (8, 64)}  # 6/8-bit codes, M=1024, K=N=4096
+    bits = 4
+    if args.probe in wide:
+        bits, group = wide[args.probe]
+        wl = inputs.Workload(f"affine{bits}_m1024_4096x4096_gs{group}", M=1024, K=4096, N=4096, x_dtype="bf16",
+                             w_std=1.0, kind="affine", group=group)
+    elif args.probe in named:
         wl = named[args.probe]
     else:
         M, K, N = (int(v) for v in args.probe.split("x"))
@@ -581,13 +635,17 @@ def run_probe(args):
     g = wl.group if wl.kind == "affine" else 0
     ws = w4a8.workspace(wl.M, wl.N, wl.K, g)
     y = torch.empty(wl.M, wl.N, device="cuda")
-    if g:
+    if bits != 4:
+        q, s, b = w4a8.pack_affine_nbit(wd, g, bits)
+    elif g:
         q, s, b = w4a8.pack_affine(wd, g)
     else:
         qs, d = w4a8.pack_q4_0(wd)
     torch.cuda.synchronize()
     for _ in range(args.steps):  # the public call one benchmark step makes
-        if g:
+        if bits != 4:
+            w4a8.w4a8_gemm_affine_nbit(xd, q, s, b, y, ws, g, bits)
+        elif g:
             w4a8.w4a8_gemm_affine(xd, q, s, b, y, ws, g)
         else:
             w4a8.w4a8_gemm(xd, qs, d, y, ws)
