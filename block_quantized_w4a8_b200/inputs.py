@@ -84,3 +84,19 @@ def sample_indices(M: int, N: int, count: int, seed: int = 1234):
     corners_m = torch.tensor([0, 0, M - 1, M - 1], dtype=torch.int32)
     corners_n = torch.tensor([0, N - 1, 0, N - 1], dtype=torch.int32)
     return torch.cat([corners_m, ms]).numpy(), torch.cat([corners_n, ns]).numpy()
+
+
+def make_q4_k(N: int, K: int, seed: int, d_scale: float = 2.0 ** -10) -> torch.Tensor:
+    """Random Q4_K weights: N rows of K/256 super-blocks of 144 bytes (uint8, (N, K/256*144)).
+    Every byte pattern of the 12 scale bytes and of the 128 code bytes is a valid block, so
+    they are drawn uniformly; d and dmin are fp16 draws of U(0.5, 1) * d_scale and
+    U(0, 1) * d_scale (bytes 0-1 and 2-3, little-endian)."""
+    assert K % 256 == 0
+    g = torch.Generator().manual_seed(seed)
+    nb = K // 256
+    blocks = torch.randint(0, 256, (N, nb, 144), generator=g, dtype=torch.int32).to(torch.uint8)
+    d = ((torch.rand((N, nb), generator=g) * 0.5 + 0.5) * d_scale).to(torch.float16)
+    dmin = (torch.rand((N, nb), generator=g) * d_scale).to(torch.float16)
+    blocks[:, :, 0:2] = d.view(torch.uint8).reshape(N, nb, 2)
+    blocks[:, :, 2:4] = dmin.view(torch.uint8).reshape(N, nb, 2)
+    return blocks.reshape(N, nb * 144)

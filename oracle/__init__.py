@@ -24,6 +24,10 @@ Functions and the definitions they follow (see the header of ``oracle.cpp``):
   applies d_x * (s * sum q q_x + b * sum q_x) per block. Codes of a row are a
   little-endian bit stream (4 bits: eight codes per 32-bit word, element k at bits
   4*(k%8) of word k/8).
+* ``q4_k_unpack_scales`` / ``dequant_q4_k`` / ``gemv_q4_k`` / ``gemv_q4_k_backward`` --
+  C-Kernel-Engine gemm_kernels_q4k.c ("GEMV: y = W @ x", "Backward Pass: Gradient w.r.t.
+  Input"): Q4_K super-blocks of 256 (w = d*sc*q - dmin*m per 32-element sub-block) with
+  FP32 activations, y = x W^T and dX = dY W, in f64 with T = sum of |terms|.
 * ``epilogue`` -- the output of a linear layer: the optional per-column bias added to
   every row of the f32 product in f32 (C-Kernel-Engine gemm_kernels_q4k.c, "Engine-
   compatible wrapper: GEMM_NT with Q4_K weights"), then f32 or bf16 (nearest even).
@@ -78,6 +82,10 @@ def _load():
         "orc_gemm_q4_0_sampled": (None, [I, I, P, P, P, P, P, P, P, P]),
         "orc_gemm_q4_0_f32": (None, [I, I, I, P, P, P, P, P]),
         "orc_pack_affine_bits": (None, [P, I, I, I, I, P, P, P]),
+        "orc_q4_k_unpack_scales": (None, [P, P, P]),
+        "orc_dequant_q4_k": (None, [P, I, I, P]),
+        "orc_gemv_q4_k": (None, [I, I, I, P, P, P, P, I]),
+        "orc_gemv_q4_k_backward": (None, [I, I, I, P, P, P, P, I]),
         "orc_dequant_affine_bits": (None, [P, P, P, I, I, I, I, P]),
         "orc_gemm_affine_bits": (None, [I, I, I, I, I, P, P, P, P, P, P, P, P, I]),
         "orc_gemm_affine_bits_sampled": (None, [I, I, I, I, P, P, P, P, P, P, P, P, P, P]),
@@ -279,6 +287,50 @@ def gemm_affine_sampled(qx, dx, sx, q, scale, bias, group: int, ms, ns, bits: in
                                          _p(sx), _p(q), _p(np.ascontiguousarray(scale, dtype=np.uint16)),
                                          _p(np.ascontiguousarray(bias, dtype=np.uint16)), _p(y), _p(T))
     return y, T
+
+
+# ----------------------------------------------------------------------------- O7 Q4_K
+def q4_k_unpack_scales(s) -> tuple[np.ndarray, np.ndarray]:
+    """The 12 packed scale bytes of a Q4_K super-block -> (sc[8], m[8]), 6 bits each."""
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    assert s.shape == (12,)
+    sc = np.empty(8, dtype=np.uint8)
+    m = np.empty(8, dtype=np.uint8)
+    _load().orc_q4_k_unpack_scales(_p(s), _p(sc), _p(m))
+    return sc, m
+
+
+def dequant_q4_k(W, N: int, K: int) -> np.ndarray:
+    """Q4_K weights (N rows x K/256 super-blocks of 144 bytes) -> f64 (N, K)."""
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    assert W.size == N * (K // 256) * 144
+    out = np.empty((N, K), dtype=np.float64)
+    _load().orc_dequant_q4_k(_p(W), N, K, _p(out))
+    return out
+
+
+def gemv_q4_k(x, W, N: int, nthreads: int = 1) -> tuple[np.ndarray, np.ndarray]:
+    """y = x . W^T for FP32 x (M, K) and Q4_K W (N rows); f64 y (M, N) and T."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    M, K = x.shape
+    assert K % 256 == 0 and W.size == N * (K // 256) * 144
+    y = np.empty((M, N), dtype=np.float64)
+    T = np.empty((M, N), dtype=np.float64)
+    _load().orc_gemv_q4_k(M, N, K, _p(x), _p(W), _p(y), _p(T), int(nthreads))
+    return y, T
+
+
+def gemv_q4_k_backward(dy, W, K: int, nthreads: int = 1) -> tuple[np.ndarray, np.ndarray]:
+    """dX = dY . W for FP32 dY (M, N) and Q4_K W (N rows, K columns); f64 dX (M, K) and T."""
+    dy = np.ascontiguousarray(dy, dtype=np.float32)
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    M, N = dy.shape
+    assert K % 256 == 0 and W.size == N * (K // 256) * 144
+    dx = np.empty((M, K), dtype=np.float64)
+    T = np.empty((M, K), dtype=np.float64)
+    _load().orc_gemv_q4_k_backward(M, N, K, _p(dy), _p(W), _p(dx), _p(T), int(nthreads))
+    return dx, T
 
 
 def epilogue(p, bias=None, bias_bf16: bool = False, out_bf16: bool = False) -> np.ndarray:

@@ -17,6 +17,10 @@
 //  * The Q4_0 / Q8_0 bit-level encodings (fp16 weight scale d, codes q in [0,15],
 //    w = d*(q-8), low nibbles = elements 0-15 and high nibbles = 16-31 of a block;
 //    activation d = amax/127 in f32, q = round-half-away(x*(1/d)) clamped to +-127).
+//  * C-Kernel-Engine gemm_kernels_q4k.c, "GEMV: y = W @ x" and "Backward Pass: Gradient
+//    w.r.t. Input": Q4_K weights (super-blocks of 256 with fp16 d and dmin and eight
+//    6-bit sub-block scales and mins, w = d*sc*q - dmin*m per 32-element sub-block) times
+//    FP32 activations, and the input gradient dX = W^T dY with the weights frozen.
 //  * MLX PR #4802 "mx.qqmm ... mode=affine": affine 4-, 6- and 8-bit weights with a
 //    per-group scale and bias; the int8 MMA runs on the original codes and the scale and
 //    bias are applied afterwards (scale = (max-min)/(2^bits - 1), bias = min per group).
@@ -434,6 +438,94 @@ void orc_gemm_affine_bits_sampled(int K, int group, int bits, int count, const i
                                   const uint16_t* scale, const uint16_t* bias, double* y, double* T) {
     for (int i = 0; i < count; ++i)
         gemm_affine_one(K, group, bits, ms[i], ns[i], qx, dx, sx, q, scale, bias, y + i, T ? T + i : nullptr);
+}
+
+// ---------------------------------------------------------------------------------
+// O7. Q4_K weights (C-Kernel-Engine gemm_kernels_q4k.c, "GEMV: y = W @ x"; the page
+//     follows the llama.cpp Q4_K layout). W is N rows x K/256 super-blocks of 144 bytes:
+//       bytes 0-1  d (fp16), bytes 2-3 dmin (fp16), bytes 4-15 the packed 6-bit scales
+//       sc[0..7] and mins m[0..7], bytes 16-143 qs[0..127] (codes 0..15).
+//     Within a super-block, the 64 elements 64i..64i+63 (i = 0..3) use qs[32i..32i+31]:
+//     element 64i + l (l < 32) is the low nibble of qs[32i + l] with sub-block 2i, element
+//     64i + 32 + l the high nibble with sub-block 2i + 1. Weight: w = d*sc[j]*q - dmin*m[j]
+//     for sub-block j.
+//     Reading (the page calls unpack_q4_k_scales without printing it; it names the llama.cpp
+//     layout): for j < 4, sc[j] = s[j] & 63 and m[j] = s[j+4] & 63; for j >= 4,
+//     sc[j] = (s[j+4] & 15) | ((s[j-4] >> 6) << 4) and m[j] = (s[j+4] >> 4) | ((s[j] >> 6) << 4),
+//     s being the 12 scale bytes.
+// ---------------------------------------------------------------------------------
+void orc_q4_k_unpack_scales(const uint8_t* s, uint8_t* sc, uint8_t* m) {
+    for (int j = 0; j < 8; ++j) {
+        if (j < 4) {
+            sc[j] = uint8_t(s[j] & 63);
+            m[j] = uint8_t(s[j + 4] & 63);
+        } else {
+            sc[j] = uint8_t((s[j + 4] & 15) | ((s[j - 4] >> 6) << 4));
+            m[j] = uint8_t((s[j + 4] >> 4) | ((s[j] >> 6) << 4));
+        }
+    }
+}
+
+// Weight of element k of row n, exact in f64 (d*sc*q: 11 + 6 + 4 bits; dmin*m: 11 + 6).
+static double q4_k_weight(const uint8_t* W, int K, int n, int k) {
+    const int64_t row_bytes = int64_t(K / 256) * 144;
+    const uint8_t* blk = W + int64_t(n) * row_bytes + int64_t(k / 256) * 144;
+    uint16_t d_bits, dmin_bits;
+    std::memcpy(&d_bits, blk, 2);
+    std::memcpy(&dmin_bits, blk + 2, 2);
+    uint8_t sc[8], m[8];
+    orc_q4_k_unpack_scales(blk + 4, sc, m);
+    const int e = k % 256;
+    const int i = e / 64, r = e % 64;
+    int q, j;
+    if (r < 32) {
+        q = blk[16 + 32 * i + r] & 15;
+        j = 2 * i;
+    } else {
+        q = blk[16 + 32 * i + (r - 32)] >> 4;
+        j = 2 * i + 1;
+    }
+    return double(orc_f16_to_f32(d_bits)) * double(sc[j]) * double(q) -
+           double(orc_f16_to_f32(dmin_bits)) * double(m[j]);
+}
+
+void orc_dequant_q4_k(const uint8_t* W, int N, int K, double* w_out) {
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) w_out[int64_t(n) * K + k] = q4_k_weight(W, K, n, k);
+}
+
+// y[m][n] = sum_k w[n][k] * x[m][k] (x is M x K, FP32), summed in f64; T = sum |w * x|.
+void orc_gemv_q4_k(int M, int N, int K, const float* x, const uint8_t* W, double* y, double* T, int nthreads) {
+    auto one = [&](int64_t e) {
+        const int m = int(e / N), n = int(e % N);
+        double acc = 0.0, tabs = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const double t = q4_k_weight(W, K, n, k) * double(x[int64_t(m) * K + k]);
+            acc += t;
+            tabs += std::fabs(t);
+        }
+        y[e] = acc;
+        if (T) T[e] = tabs;
+    };
+    parallel_over(int64_t(M) * N, nthreads, one);
+}
+
+// Input gradient, "Backward Pass: Gradient w.r.t. Input": dX[m][k] = sum_n w[n][k] *
+// dY[m][n] (dY is M x N), summed in f64; T = sum |w * dY|. The weights get no gradient.
+void orc_gemv_q4_k_backward(int M, int N, int K, const float* dY, const uint8_t* W, double* dX, double* T,
+                            int nthreads) {
+    auto one = [&](int64_t e) {
+        const int m = int(e / K), k = int(e % K);
+        double acc = 0.0, tabs = 0.0;
+        for (int n = 0; n < N; ++n) {
+            const double t = q4_k_weight(W, K, n, k) * double(dY[int64_t(m) * N + n]);
+            acc += t;
+            tabs += std::fabs(t);
+        }
+        dX[e] = acc;
+        if (T) T[e] = tabs;
+    };
+    parallel_over(int64_t(M) * K, nthreads, one);
 }
 
 }  // extern "C"

@@ -86,3 +86,27 @@ def affine_weights_bits(q: np.ndarray, scale: np.ndarray, bias: np.ndarray, grou
     s = np.repeat(bf16_bits_to_f64(scale), group, axis=1)
     b = np.repeat(bf16_bits_to_f64(bias), group, axis=1)
     return s * codes + b
+
+
+def q4_k_scales(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """(..., 12) scale bytes -> (..., 8) sub-block scales and mins of 6 bits (llama.cpp
+    Q4_K packing: the low 6 bits of bytes 0-3 / 4-7 are sc / m of sub-blocks 0-3; sub-blocks
+    4-7 take their low 4 bits from the nibbles of bytes 8-11 and their top 2 bits from the
+    top 2 bits of bytes 0-3 (sc) and 4-7 (m))."""
+    s = s.astype(np.int64)
+    sc = np.concatenate([s[..., 0:4] & 63, (s[..., 8:12] & 15) | ((s[..., 0:4] >> 6) << 4)], axis=-1)
+    m = np.concatenate([s[..., 4:8] & 63, (s[..., 8:12] >> 4) | ((s[..., 4:8] >> 6) << 4)], axis=-1)
+    return sc, m
+
+
+def q4_k_weights(W: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Q4_K rows (N, K/256*144 bytes) -> f64 weights (N, K)."""
+    b = np.ascontiguousarray(W, dtype=np.uint8).reshape(N, K // 256, 144)
+    d = b[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+    dmin = b[..., 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+    sc, m = q4_k_scales(b[..., 4:16])
+    qs = b[..., 16:].reshape(N, K // 256, 4, 32).astype(np.int64)
+    codes = np.concatenate([qs & 15, qs >> 4], axis=-1).reshape(N, K // 256, 256)  # per 64: low 32, high 32
+    sub = np.arange(256) // 32                                                      # sub-block of each element
+    w = d[..., None] * sc[..., sub] * codes - dmin[..., None] * m[..., sub]
+    return w.reshape(N, K)
