@@ -509,6 +509,7 @@ def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
         torch.cuda.empty_cache()
     results += run_epilogue(args, torch, w4a8, oracle, inputs, steps, dev)
     results += run_wide(args, torch, w4a8, oracle, inputs, steps, dev, int8_peak)
+    results += run_q4k(args, torch, w4a8, oracle, inputs, steps, dev, peaks)
     return results
 
 
@@ -606,6 +607,50 @@ def run_wide(args, torch, w4a8, oracle, inputs, steps, dev, int8_peak):
         out.append(entry)
         del sets
         torch.cuda.empty_cache()
+    return out
+
+
+def run_q4k(args, torch, w4a8, oracle, inputs, steps, dev, peaks):
+    """Q4_K GEMV (y = x W^T) and its input gradient (dX = dY W) with FP32 activations at
+    decode size (M=1, K=N=4096), each checked against the oracle on sampled outputs before
+    it is timed; weight GB/s against the measured HBM copy bandwidth."""
+    import numpy as np
+    out = []
+    M, N, K = 1, 4096, 4096
+    W = inputs.make_q4_k(N, K, seed=21)
+    wbytes = N * K // 256 * 144
+    R = copies_for(wbytes)
+    sets = [W.to(dev) for _ in range(R)]
+    x = inputs.randn((M, K), seed=22)
+    dy = inputs.randn((M, N), seed=23)
+    xd, dyd = x.to(dev), dy.to(dev)
+    y = torch.empty(M, N, device=dev)
+    dx = torch.empty(M, K, device=dev)
+    ws = torch.empty(max(16, w4a8.w4a8_q4_k_backward_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+    w4a8.w4a8_gemv_q4_k(xd, sets[0], y)
+    w4a8.w4a8_gemv_q4_k_backward(dyd, sets[0], dx, ws)
+    torch.cuda.synchronize()
+    yref, Ty = oracle.gemv_q4_k(x.numpy(), W.numpy(), N, nthreads=8)
+    dxref, Tx = oracle.gemv_q4_k_backward(dy.numpy(), W.numpy(), K, nthreads=8)
+    tol = 2.0 ** -24 * (K // 8 + 32)
+    ok_f = bool(np.all(np.abs(y.cpu().numpy().astype(np.float64) - yref) <= tol * Ty))
+    ok_b = bool(np.all(np.abs(dx.cpu().numpy().astype(np.float64) - dxref) <= 2.0 ** -24 * (N // 32 + 33) * Tx))
+    for name, ok, fn in [("q4_k_gemv_m1_4096x4096", ok_f, lambda i: w4a8.w4a8_gemv_q4_k(xd, sets[i % R], y)),
+                         ("q4_k_backward_m1_4096x4096", ok_b,
+                          lambda i: w4a8.w4a8_gemv_q4_k_backward(dyd, sets[i % R], dx, ws))]:
+        entry = {"workload": name, "M": M, "N": N, "K": K, "parity": "pass" if ok else "FAIL"}
+        if ok:
+            for i in range(3):
+                fn(i)
+            us = timed(fn, steps, torch, graph=True) / steps * 1e3
+            gbs = wbytes / (us * 1e-6) / 1e9
+            entry.update({"us_per_call": us, "weight_gbs_call": gbs,
+                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                       "frac": gbs / peaks["hbm_gbs"]},
+                          "l2": f"{R} rotating weight copies"})
+        out.append(entry)
+    del sets
+    torch.cuda.empty_cache()
     return out
 
 

@@ -28,7 +28,8 @@ PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 
 EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a8_gemm", "w4a8_gemm_ex",
            "w4a8_pack_affine", "w4a8_gemm_affine", "w4a8_gemm_affine_ex", "w4a8_gemm_epi", "w4a8_gemm_affine_epi",
-           "w4a8_pack_affine_nbit", "w4a8_gemm_affine_nbit", "w4a8_prepare_act",
+           "w4a8_pack_affine_nbit", "w4a8_gemm_affine_nbit", "w4a8_gemv_q4_k", "w4a8_gemv_q4_k_backward",
+           "w4a8_q4_k_backward_workspace_bytes", "w4a8_prepare_act",
            "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_gemm_noalloc", "w4a8_last_device_error",
            "w4a8_last_cuda_error_string", "w4a8_status_string"]
 
@@ -65,6 +66,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_gemm_affine_epi": (I, [I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
         "w4a8_pack_affine_nbit": (I, [P, I, I, I, I, I, P, P, P, P]),
         "w4a8_gemm_affine_nbit": (I, [I, I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
+        "w4a8_gemv_q4_k": (I, [I, I, I, P, P, P, P]),
+        "w4a8_gemv_q4_k_backward": (I, [I, I, I, P, P, P, P, Z, P]),
+        "w4a8_q4_k_backward_workspace_bytes": (Z, [I, I, I]),
         "w4a8_prepare_act": (I, [I, I, I, P, I, P, Z, I, P]),
         "w4a8_gemm_prepared": (I, [I, I, I, P, P, P, P, Z, I, P]),
         "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
@@ -195,6 +199,42 @@ def w4a8_gemm_affine_nbit(x, q, scale, bias_w, y, ws, group: int, bits: int, bia
            load_library().w4a8_gemm_affine_nbit(M, N, K, group, bits, _ptr(x), _dtype(x), _ptr(q), _ptr(scale),
                                                 _ptr(bias_w), ctypes.byref(epi), _ptr(y), _ptr(ws),
                                                 ws.numel() * ws.element_size(), path, _stream(stream)))
+
+
+def w4a8_gemv_q4_k(x, w_q4k, y, stream=None) -> None:
+    """y (M, N) f32 = x (M, K) f32 . W^T, W in Q4_K (uint8 (N, K/256*144))."""
+    M, K = x.shape
+    N = w_q4k.shape[0]
+    _check("w4a8_gemv_q4_k", load_library().w4a8_gemv_q4_k(M, N, K, _ptr(x), _ptr(w_q4k), _ptr(y), _stream(stream)))
+
+
+def w4a8_gemv_q4_k_backward(dy, w_q4k, dx, ws, stream=None) -> None:
+    """dx (M, K) f32 = dy (M, N) f32 . W (the input gradient), W in Q4_K."""
+    M, N = dy.shape
+    K = dx.shape[1]
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("w4a8_gemv_q4_k_backward",
+           load_library().w4a8_gemv_q4_k_backward(M, N, K, _ptr(dy), _ptr(w_q4k), _ptr(dx),
+                                                  _ptr(ws) if ws is not None else None, nbytes, _stream(stream)))
+
+
+def w4a8_q4_k_backward_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load_library().w4a8_q4_k_backward_workspace_bytes(M, N, K))
+
+
+def gemv_q4_k(x, w_q4k, stream=None):
+    y = torch.empty(x.shape[0], w_q4k.shape[0], dtype=torch.float32, device=x.device)
+    w4a8_gemv_q4_k(x, w_q4k, y, stream)
+    return y
+
+
+def gemv_q4_k_backward(dy, w_q4k, K: int, ws=None, stream=None):
+    M, N = dy.shape
+    dx = torch.empty(M, K, dtype=torch.float32, device=dy.device)
+    if ws is None:
+        ws = torch.empty(max(16, w4a8_q4_k_backward_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dy.device)
+    w4a8_gemv_q4_k_backward(dy, w_q4k, dx, ws, stream)
+    return dx
 
 
 def w4a8_pack_affine(w, group: int, q, scale, bias, stream=None) -> None:

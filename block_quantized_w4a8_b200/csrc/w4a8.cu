@@ -11,6 +11,7 @@
 #include "device_common.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_pair.cuh"
+#include "q4k.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
 
@@ -609,9 +610,92 @@ w4a8_status pack_affine_impl(const void* w, w4a8_dtype dtype, int N, int K, int 
     return launch_status();
 }
 
+// ------------------------------------------------------------------ Q4_K
+// Row ranges of the backward: enough CTAs (super-block columns x ranges) for four per
+// SM, at least 32 rows per range.
+inline int q4k_row_ranges(int N, int K) {
+    const int nb = K / 256;
+    int64_t R = cdiv(4 * int64_t(sm_count()), nb);
+    const int64_t rmax = cdiv(N, 32);
+    if (R > rmax) R = rmax;
+    if (R < 1) R = 1;
+    const int rows = int(cdiv(N, R));
+    return int(cdiv(N, rows));
+}
+inline size_t q4k_bwd_bytes(int M, int N, int K) {
+    const int R = q4k_row_ranges(N, K);
+    return R > 1 ? size_t(R) * (M < 2 ? M : 2) * K * 4 : 0;
+}
+w4a8_status check_q4k(int M, int N, int K, const void* a, const void* w, const void* out) {
+    if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 256) != 0 || !a || !w || !out) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return W4A8_ERR_MISALIGNED;
+    return W4A8_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+w4a8_status w4a8_gemv_q4_k(int M, int N, int K, const float* x, const uint8_t* w_q4k, float* y,
+                           cudaStream_t stream) {
+    const w4a8_status st = check_q4k(M, N, K, x, w_q4k, y);
+    if (st != W4A8_OK) return st;
+    const dim3 grid(unsigned(cdiv(N, 4)));
+    for (int m0 = 0; m0 < M; m0 += 2) {
+        const int mt = (M - m0 < 2) ? (M - m0) : 2;
+        if (mt == 1)
+            q4k::gemv_kernel<1><<<grid, q4k::kThreads, 0, stream>>>(1, N, K, x + int64_t(m0) * K, w_q4k,
+                                                                   y + int64_t(m0) * N);
+        else
+            q4k::gemv_kernel<2><<<grid, q4k::kThreads, 0, stream>>>(2, N, K, x + int64_t(m0) * K, w_q4k,
+                                                                   y + int64_t(m0) * N);
+        const w4a8_status ls = launch_status();
+        if (ls != W4A8_OK) return ls;
+    }
+    return W4A8_OK;
+}
+
+size_t w4a8_q4_k_backward_workspace_bytes(int M, int N, int K) {
+    if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 256) != 0) return 0;
+    const size_t b = q4k_bwd_bytes(M, N, K);
+    return b ? b : 16;
+}
+
+w4a8_status w4a8_gemv_q4_k_backward(int M, int N, int K, const float* dy, const uint8_t* w_q4k, float* dx,
+                                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+    w4a8_status st = check_q4k(M, N, K, dy, w_q4k, dx);
+    if (st != W4A8_OK) return st;
+    const int R = q4k_row_ranges(N, K);
+    const size_t need = q4k_bwd_bytes(M, N, K);
+    if (need > 0) {
+        if (!ws || ws_bytes < need) return W4A8_ERR_WORKSPACE;
+        if (!aligned16(ws)) return W4A8_ERR_MISALIGNED;
+    }
+    const int rows = int(cdiv(N, R));
+    float* part = static_cast<float*>(ws);
+    const dim3 grid(unsigned(K / 256), unsigned(R));
+    for (int m0 = 0; m0 < M; m0 += 2) {
+        const int mt = (M - m0 < 2) ? (M - m0) : 2;
+        const float* dyc = dy + int64_t(m0) * N;
+        float* dxc = dx + int64_t(m0) * K;
+        float* out = R > 1 ? part : dxc;
+        if (mt == 1)
+            q4k::bwd_kernel<1><<<grid, q4k::kThreads, 0, stream>>>(1, N, K, rows, dyc, w_q4k, out);
+        else
+            q4k::bwd_kernel<2><<<grid, q4k::kThreads, 0, stream>>>(2, N, K, rows, dyc, w_q4k, out);
+        st = launch_status();
+        if (st != W4A8_OK) return st;
+        if (R > 1) {
+            const int64_t count = int64_t(mt) * K;
+            int64_t nblk = cdiv(count, 256);
+            if (nblk > 4 * int64_t(sm_count())) nblk = 4 * int64_t(sm_count());
+            q4k::bwd_reduce_kernel<<<unsigned(nblk), 256, 0, stream>>>(part, R, count, dxc);
+            st = launch_status();
+            if (st != W4A8_OK) return st;
+        }
+    }
+    return W4A8_OK;
+}
 
 w4a8_status w4a8_pack_q4_0(const void* w, w4a8_dtype dtype, int N, int K, uint8_t* qs, uint16_t* d_fp16,
                            cudaStream_t stream) {

@@ -242,6 +242,32 @@ w4a8_status w4a8_gemm_affine_nbit(int M, int N, int K, int group, int bits, cons
                                   w4a8_path path, cudaStream_t stream);
 
 /*
+ * Q4_K weights with FP32 activations (C-Kernel-Engine gemm_kernels_q4k.c, "GEMV: y = W @ x"
+ * and "Backward Pass: Gradient w.r.t. Input"; the page follows the llama.cpp Q4_K layout).
+ * w_q4k : N rows, each K/256 super-blocks of 144 bytes: d (fp16), dmin (fp16), 12 bytes of
+ *         packed 6-bit sub-block scales sc[8] and mins m[8] (j < 4: sc = s[j] & 63,
+ *         m = s[j+4] & 63; j >= 4: sc = (s[j+4] & 15) | (s[j-4] >> 6) << 4,
+ *         m = (s[j+4] >> 4) | (s[j] >> 6) << 4), 128 code bytes (byte 32i + l: element
+ *         64i + l in the low nibble, sub-block 2i; element 64i + 32 + l in the high nibble,
+ *         sub-block 2i + 1). Weight: w = d*sc*q - dmin*m. K must be a multiple of 256.
+ * w4a8_gemv_q4_k          : y[m][n] = sum_k w[n][k] * x[m][k]; x M x K f32, y M x N f32.
+ * w4a8_gemv_q4_k_backward : dx[m][k] = sum_n w[n][k] * dy[m][n] (the input gradient of
+ *                           y = x W^T; the weights get none); dy M x N f32, dx M x K f32.
+ *                           `ws` of w4a8_q4_k_backward_workspace_bytes(M, N, K) bytes holds
+ *                           partial sums over row ranges, added in a fixed order (the
+ *                           result does not depend on scheduling).
+ * Sums are taken in f32 with fused multiply-adds; each output is within a few units of
+ * 2^-24 * (terms per chain) of the exact value relative to sum |terms|.
+ * All pointers device memory, 16-byte aligned, caller-owned; async on `stream`.
+ * Errors: INVALID_ARG (sizes, K % 256, null), MISALIGNED, WORKSPACE, CUDA.
+ */
+w4a8_status w4a8_gemv_q4_k(int M, int N, int K, const float* x, const uint8_t* w_q4k, float* y,
+                           cudaStream_t stream);
+size_t w4a8_q4_k_backward_workspace_bytes(int M, int N, int K);
+w4a8_status w4a8_gemv_q4_k_backward(int M, int N, int K, const float* dy, const uint8_t* w_q4k, float* dx,
+                                    void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * w4a8_gemm for callers that cannot allocate device memory. Some callers are not allowed
  * to call cudaMalloc at all: a host application that reserves every byte of device memory
  * up front and owns its allocator, or a plug-in interface whose call signature carries

@@ -141,3 +141,16 @@ def test_affine_nbit_argument_errors(lib):
     assert pack(bits=7) == 2 and pack(group=256) == 2
     assert pack(K=96) == 1 and pack(q=0) == 1
     assert pack(q=FAKE + 8) == 6                       # MISALIGNED
+
+
+def test_q4_k_argument_errors(lib):
+    P = ctypes.c_void_p
+    f, b = lib.w4a8_gemv_q4_k, lib.w4a8_gemv_q4_k_backward
+    assert f(1, 8, 300, P(FAKE), P(FAKE), P(FAKE), P(0)) == 1      # K not a multiple of 256
+    assert f(0, 8, 256, P(FAKE), P(FAKE), P(FAKE), P(0)) == 1
+    assert f(1, 8, 256, P(0), P(FAKE), P(FAKE), P(0)) == 1
+    assert f(1, 8, 256, P(FAKE + 4), P(FAKE), P(FAKE), P(0)) == 6  # MISALIGNED
+    assert b(1, 8, 256, P(FAKE), P(FAKE), P(FAKE + 8), P(FAKE), 1 << 20, P(0)) == 6
+    assert b(1, 4096, 4096, P(FAKE), P(FAKE), P(FAKE), P(0), 0, P(0)) == 3  # WORKSPACE missing
+    assert lib.w4a8_q4_k_backward_workspace_bytes(1, 4096, 4000) == 0
+    assert lib.w4a8_q4_k_backward_workspace_bytes(1, 8, 256) == 16      # one row range: no partials
