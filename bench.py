@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--sweep", choices=["some", "all", "none"], default="some")
     ap.add_argument("--probe", default=None,
                     help="profiling probe: run `--steps` calls of one workload (decode, minilm, prefill, affine64, "
-                         "affine128, affine6_64, affine8_64, or MxKxN) through w4a8_gemm[_affine[_nbit]], then exit "
+                         "affine128, affine6_64, affine8_64, q4k, q4k_bwd, or MxKxN) through w4a8_gemm[_affine[_nbit]], then exit "
                          "without timing")
     return ap.parse_args()
 
@@ -664,6 +664,22 @@ def run_probe(args):
              "affine64": inputs.AFFINE_GS64, "affine128": inputs.AFFINE_GS128}
     wide = {"affine6_64": (6, 64), "affine8_64": (8, 64)}  # 6/8-bit codes, M=1024, K=N=4096
     bits = 4
+    if args.probe in ("q4k", "q4k_bwd"):  # Q4_K forward / input gradient, M=1, K=N=4096
+        torch.cuda.set_device(0)
+        w4a8.load_library()
+        W = inputs.make_q4_k(4096, 4096, seed=21).cuda()
+        x = inputs.randn((1, 4096), seed=22).cuda()
+        out = torch.empty(1, 4096, device="cuda")
+        ws = torch.empty(max(16, w4a8.w4a8_q4_k_backward_workspace_bytes(1, 4096, 4096)), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(args.steps):
+            if args.probe == "q4k":
+                w4a8.w4a8_gemv_q4_k(x, W, out)
+            else:
+                w4a8.w4a8_gemv_q4_k_backward(x, W, out, ws)
+        torch.cuda.synchronize()
+        print(f"probe {args.probe}: {args.steps} steps ok")
+        return 0
     if args.probe in wide:
         bits, group = wide[args.probe]
         wl = inputs.Workload(f"affine{bits}_m1024_4096x4096_gs{group}", M=1024, K=4096, N=4096, x_dtype="bf16",
