@@ -62,73 +62,86 @@ __device__ __forceinline__ ChunkScales chunk_scales(const uint4& h, int c) {
 
 // ------------------------------------------------------------------ forward
 // y[m][n] = sum_k w[n][k] x[m][k] for MT tokens (x: MT x K f32, row-major). CTA b owns
-// rows 4b..4b+3; warp w takes super-blocks w, w + 8, w + 16, ... of those rows, two per
-// step with all their loads issued first. The 8 lanes of a row then add their partial
-// sums by shuffles, and the 8 warps' sums are added in warp order through shared memory.
-template <int MT>
-__device__ __forceinline__ void fwd_accumulate(const uint4& h, const uint4& q, int c, const float* xp, float& a) {
-    const ChunkScales cs = chunk_scales(h, c);
-    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {  // code bytes 4v..4v+3 of the chunk
-        const float4 xl = __ldg(reinterpret_cast<const float4*>(xp) + v);
-        const float4 xh = __ldg(reinterpret_cast<const float4*>(xp + 32) + v);
-        a = fmaf(fmaf(cs.d_lo, code_f(qw[v], 0), -cs.m_lo), xl.x, a);
-        a = fmaf(fmaf(cs.d_lo, code_f(qw[v], 8), -cs.m_lo), xl.y, a);
-        a = fmaf(fmaf(cs.d_lo, code_f(qw[v], 16), -cs.m_lo), xl.z, a);
-        a = fmaf(fmaf(cs.d_lo, code_f(qw[v], 24), -cs.m_lo), xl.w, a);
-        a = fmaf(fmaf(cs.d_hi, code_f(qw[v], 4), -cs.m_hi), xh.x, a);
-        a = fmaf(fmaf(cs.d_hi, code_f(qw[v], 12), -cs.m_hi), xh.y, a);
-        a = fmaf(fmaf(cs.d_hi, code_f(qw[v], 20), -cs.m_hi), xh.z, a);
-        a = fmaf(fmaf(cs.d_hi, code_f(qw[v], 28), -cs.m_hi), xh.w, a);
-    }
-}
-
+// rows 16b..16b+15 (four row groups of four); warp w takes super-blocks w, w + 8, ...
+// For each of them the warp reads its lanes' slice of x once into registers (the same
+// 32 elements serve all four row groups) and issues the loads of the four groups' code
+// chunks together, so x costs the L1 one read per CTA rather than one per row group.
+// The 8 lanes of a row add their partial sums by shuffles, the 8 warps' sums are added
+// in warp order through shared memory.
 template <int MT>
 __global__ void __launch_bounds__(kThreads) gemv_kernel(int M, int N, int K, const float* __restrict__ x,
                                                       const uint8_t* __restrict__ W, float* __restrict__ y) {
-    __shared__ float red[kWarps][4][MT];
+    constexpr int RG = 4;  // row groups of four rows per CTA
+    __shared__ float red[kWarps][4 * RG][MT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rr = lane >> 3, c = lane & 7;
-    const int n = blockIdx.x * 4 + rr;
     const int nb = K >> 8;
-    const bool row_ok = n < N;
-    const uint8_t* row = W + int64_t(row_ok ? n : 0) * nb * kBlockBytes;
+    const int n0 = blockIdx.x * 4 * RG;
     const int e0 = 64 * (c >> 1) + 16 * (c & 1);  // first element of the chunk's low nibbles
-    float acc[MT];
+    float acc[RG][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-    for (int sb = warp; sb < nb; sb += 2 * kWarps) {
-        const int sb2 = sb + kWarps;
-        const bool two = sb2 < nb;
-        uint4 h0 = make_uint4(0u, 0u, 0u, 0u), q0 = h0, h1 = h0, q1 = h0;
-        if (row_ok) {
-            h0 = __ldcs(reinterpret_cast<const uint4*>(row + sb * kBlockBytes));
-            q0 = __ldcs(reinterpret_cast<const uint4*>(row + sb * kBlockBytes + 16 + 16 * c));
-            if (two) {
-                h1 = __ldcs(reinterpret_cast<const uint4*>(row + sb2 * kBlockBytes));
-                q1 = __ldcs(reinterpret_cast<const uint4*>(row + sb2 * kBlockBytes + 16 + 16 * c));
+    for (int g = 0; g < RG; ++g)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[g][m] = 0.0f;
+    for (int sb = warp; sb < nb; sb += kWarps) {
+        float xs[MT][32];  // x[m][sb*256 + e0 + t] (t < 16) and x[m][sb*256 + e0 + 32 + t]
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const float* xp = x + int64_t(m < M ? m : 0) * K + sb * 256 + e0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(xp) + v);
+                const float4 b = __ldg(reinterpret_cast<const float4*>(xp + 32) + v);
+                xs[m][4 * v] = a.x; xs[m][4 * v + 1] = a.y; xs[m][4 * v + 2] = a.z; xs[m][4 * v + 3] = a.w;
+                xs[m][16 + 4 * v] = b.x; xs[m][16 + 4 * v + 1] = b.y;
+                xs[m][16 + 4 * v + 2] = b.z; xs[m][16 + 4 * v + 3] = b.w;
+            }
+        }
+        uint4 h[RG], q[RG];
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {
+            const int n = n0 + 4 * g + rr;
+            h[g] = make_uint4(0u, 0u, 0u, 0u);
+            q[g] = h[g];
+            if (n < N) {
+                const uint8_t* blk = W + (int64_t(n) * nb + sb) * kBlockBytes;
+                h[g] = __ldcs(reinterpret_cast<const uint4*>(blk));
+                q[g] = __ldcs(reinterpret_cast<const uint4*>(blk + 16 + 16 * c));
             }
         }
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if (m >= M) break;
-            fwd_accumulate<MT>(h0, q0, c, x + int64_t(m) * K + sb * 256 + e0, acc[m]);
-            if (two) fwd_accumulate<MT>(h1, q1, c, x + int64_t(m) * K + sb2 * 256 + e0, acc[m]);
+        for (int g = 0; g < RG; ++g) {
+            const ChunkScales cs = chunk_scales(h[g], c);
+            const uint32_t qw[4] = {q[g].x, q[g].y, q[g].z, q[g].w};
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const float wl = fmaf(cs.d_lo, code_f(qw[v], 8 * b), -cs.m_lo);
+                    const float wh = fmaf(cs.d_hi, code_f(qw[v], 8 * b + 4), -cs.m_hi);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        acc[g][m] = fmaf(wl, xs[m][4 * v + b], acc[g][m]);
+                        acc[g][m] = fmaf(wh, xs[m][16 + 4 * v + b], acc[g][m]);
+                    }
+                }
+            }
         }
     }
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        float v = acc[m];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        if (c == 0) red[warp][rr][m] = v;
-    }
+    for (int g = 0; g < RG; ++g)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float v = acc[g][m];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            if (c == 0) red[warp][4 * g + rr][m] = v;
+        }
     __syncthreads();
-    if (threadIdx.x < 4 * MT) {
-        const int r2 = threadIdx.x / MT, m = threadIdx.x % MT;
-        const int n2 = blockIdx.x * 4 + r2;
+    for (int i = threadIdx.x; i < 4 * RG * MT; i += kThreads) {
+        const int r2 = i / MT, m = i % MT;
+        const int n2 = n0 + r2;
         if (n2 < N && m < M) {
             float v = 0.0f;
 #pragma unroll

@@ -640,7 +640,7 @@ w4a8_status w4a8_gemv_q4_k(int M, int N, int K, const float* x, const uint8_t* w
                            cudaStream_t stream) {
     const w4a8_status st = check_q4k(M, N, K, x, w_q4k, y);
     if (st != W4A8_OK) return st;
-    const dim3 grid(unsigned(cdiv(N, 4)));
+    const dim3 grid(unsigned(cdiv(N, 16)));  // 16 rows per CTA
     for (int m0 = 0; m0 < M; m0 += 2) {
         const int mt = (M - m0 < 2) ? (M - m0) : 2;
         if (mt == 1)
