@@ -138,6 +138,9 @@ def test_affine_nbit_argument_errors(lib):
     assert gemm(K=96, group=64) == 1                   # K not a multiple of the group
     assert gemm(path=2) == 2                           # no tensor-core path for 6/8-bit codes
     assert gemm(bits=8, path=2) == 2
+    # M > 64 but K/group = 4 (scale rows not a multiple of 16 bytes): no pair kernel
+    assert lib.w4a8_gemm_affine_nbit(200, 8, 256, 64, 8, P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), None,
+                                     P(FAKE), P(FAKE), 1 << 40, 2, P(0)) == 2
     assert pack(bits=7) == 2 and pack(group=256) == 2
     assert pack(K=96) == 1 and pack(q=0) == 1
     assert pack(q=FAKE + 8) == 6                       # MISALIGNED
