@@ -255,7 +255,10 @@ w4a8_status w4a8_gemm_affine_nbit(int M, int N, int K, int group, int bits, cons
  *                           y = x W^T; the weights get none); dy M x N f32, dx M x K f32.
  *                           `ws` of w4a8_q4_k_backward_workspace_bytes(M, N, K) bytes holds
  *                           partial sums over row ranges, added in a fixed order (the
- *                           result does not depend on scheduling).
+ *                           result does not depend on scheduling). The size depends on the
+ *                           current device's SM count (query it with that device current);
+ *                           it is 16 when the shape needs a single row range, and then
+ *                           `ws` may also be NULL. Returns 0 for invalid sizes.
  * Sums are taken in f32 with fused multiply-adds; each output is within a few units of
  * 2^-24 * (terms per chain) of the exact value relative to sum |terms|.
  * All pointers device memory, 16-byte aligned, caller-owned; async on `stream`.
