@@ -378,6 +378,8 @@ def run_ours(args):
         "ms_per_step_eager": ms_eager / args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic.get(tkey),
+                     "traffic_note": None if traffic.get(tkey) is not None else
+                     "no ncu capture of the current kernel build (profiles/ holds an earlier build's counters)",
                      "kernel": "gemv2_kernel<1,0,1> (Q4_0, M=1, x quantised in-kernel; the whole step)",
                      "kernel_us": k_us, "prepared_contraction_us": prepared_us,
                      "algorithmic_bytes_per_launch": alg, "peak_source": peaks.get("source", "measured") +
