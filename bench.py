@@ -399,6 +399,11 @@ def run_ours(args):
                                 "sample": f"{reps} full decode steps (Q8_0 quantisation of x + all 4096 outputs "
                                           f"of the 1x4096x4096 contraction), ~{args.cpu_seconds:.0f} s, "
                                           f"threads over output elements"}
+        # the same oracle on one host thread (the scalar figure), a shorter bounded sample
+        sec1, reps1 = oracle_decode_seconds(max(1.0, args.cpu_seconds / 4), 1)
+        line["cpu_baseline"]["single_thread"] = {"value": weight_bytes(N, K) / sec1 / 1e9, "unit": "GB/s",
+                                                 "cores": 1, "ms_per_step": sec1 * 1e3,
+                                                 "sample": f"{reps1} full decode steps on one thread"}
 
     # ---------------- other workloads (rank 0 only, after the collective steps)
     if rank == 0 and not args.no_extra:
