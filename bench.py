@@ -149,6 +149,34 @@ def rank_info():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+# Cross-rank steps of the benchmark. Every rank calls each of these at the same point (in
+# the error paths too), so the collectives match; with dist None (one process) they are
+# plain values. `device` is where the collective's tensor lives ("cuda" under NCCL).
+def max_over_ranks(value: float, dist=None, device="cuda") -> float:
+    """The largest `value` over all ranks (the job's time is its slowest rank's)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_ranks_ok(ok: bool, dist=None, device="cuda") -> bool:
+    """True when `ok` holds on every rank."""
+    if dist is None:
+        return bool(ok)
+    import torch
+    t = torch.tensor([1 if ok else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, over the max-over-ranks time `ms`."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def check_parity_sampled(y_dev, ref_fn, M, N, count=400, seed=7):
     import numpy as np
     from block_quantized_w4a8_b200 import inputs
@@ -192,12 +220,7 @@ def timed(step, steps, torch, dist=None, graph=False):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
 
 
 def copies_for(bytes_per_copy: int) -> int:
@@ -308,10 +331,12 @@ def run_ours(args):
     yref, T = oracle.gemm_q4_0(rqx, rdx, rqs, rd, nthreads=os.cpu_count() or 1)
     parity = bool(np.array_equal(qs0.cpu().numpy(), rqs)) and bool(
         np.all(np.abs(y.cpu().numpy().astype(np.float64) - yref) <= 1e-5 * T))
-    if not parity:
+    if not all_ranks_ok(parity, dist, "cuda"):  # every rank stops together
         if rank == 0:
             print(json.dumps({"metric": "W4A8 decode GEMV weight GB/s (M=1, K=N=4096)", "value": None,
                               "error": "parity check against the oracle failed; not timed"}), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
         return 1
 
     def step(i):
@@ -333,7 +358,7 @@ def run_ours(args):
     # M*K = 4096 is small enough for the GEMV to quantise x itself: one launch per step
     launches += args.steps
     ms_step = ms / args.steps
-    value = weight_bytes(N, K) * args.steps * world / (ms * 1e-3) / 1e9
+    value = whole_job_rate(weight_bytes(N, K) * args.steps, world, ms) / 1e9
     k_us = ms_step * 1e3
     alg = weight_bytes(N, K) + M * K * 4 + M * N * 4   # packed weights + scales, f32 x, f32 y
     achieved = alg / (k_us * 1e-6) / 1e9
@@ -359,7 +384,7 @@ def run_ours(args):
     for i in range(args.warmup):
         step_e2e(i)
     ems = timed(step_e2e, args.steps, torch, dist)
-    e2e_value = weight_bytes(N, K) * args.steps * world / (ems * 1e-3) / 1e9
+    e2e_value = whole_job_rate(weight_bytes(N, K) * args.steps, world, ems) / 1e9
     sampler.stop()
     clocks = sampler.summary(t0, t1)
 
