@@ -124,3 +124,19 @@ def test_bias_column_split_carries_22_bits():
         for scale in (1.0, 2.0 ** -11):
             prod = part[:, None] * (S[None, :] * scale)
             assert np.all(prod.astype(np.float32).astype(np.float64) == prod)
+
+
+def test_q4_k_weight_product_is_exact_in_f32():
+    """Q4_K on the GPU forms each weight as fma(d*sc, q, -dmin*m): d*sc (fp16 times a 6-bit
+    scale) and d*sc*q (times a 4-bit code) are exact in f32 for every finite fp16 d, so the
+    single rounding of the fused form is the page's d1*q - m1 with d1 = d*sc (whose product
+    is exact), and dmin*m is exact likewise."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    d = bits.view(np.float16).astype(np.float64)
+    d = d[np.isfinite(d)]
+    sc = np.arange(64, dtype=np.float64)
+    d1 = d[:, None] * sc[None, :]
+    assert np.all(d1.astype(np.float32).astype(np.float64) == d1)
+    for q in (13.0, 15.0):  # the codes with the most significant bits
+        p = d1 * q
+        assert np.all(p.astype(np.float32).astype(np.float64) == p)
