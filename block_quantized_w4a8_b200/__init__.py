@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libw4a8.so")
 
 W4A8_OK = 0
 STATUS_NAMES = {0: "W4A8_OK", 1: "W4A8_ERR_INVALID_ARG", 2: "W4A8_ERR_UNSUPPORTED", 3: "W4A8_ERR_WORKSPACE",
-                4: "W4A8_ERR_CUDA", 5: "W4A8_ERR_DEVICE_TIMEOUT", 6: "W4A8_ERR_MISALIGNED", 7: "W4A8_ERR_RANGE"}
+                4: "W4A8_ERR_CUDA", 5: "W4A8_ERR_DEVICE_TIMEOUT", 6: "W4A8_ERR_MISALIGNED", 7: "W4A8_ERR_RANGE",
+                8: "W4A8_ERR_CHECK"}
 W4A8_F32, W4A8_BF16 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 

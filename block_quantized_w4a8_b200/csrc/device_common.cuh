@@ -12,11 +12,31 @@ namespace w4a8 {
 
 // Bit set in the device status word when a bounded wait ran out.
 constexpr unsigned kDevErrTimeout = 1u;
+// Bit set by a device-side check of the checked build (W4A8_CHECKED) that failed.
+constexpr unsigned kDevErrChecked = 4u;
 // Upper bound on any single wait inside a kernel (ns of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 1500000000ull;
 
 // Device status word, read and cleared by w4a8_last_device_error().
 __device__ unsigned int g_device_status = 0;
+
+// Checked build (compiled with -DW4A8_CHECKED): device-side checks of the conditions a
+// copy needs to be legal (alignment of TMA coordinates and bulk-copy addresses and sizes).
+// A failed check records kDevErrChecked and the copy is skipped, so the waiting barrier
+// runs out into the bounded-wait error path instead of the copy faulting the GPU. In the
+// default build `checked` is the constant true and the checks compile away.
+#ifdef W4A8_CHECKED
+constexpr bool kCheckedBuild = true;
+#else
+constexpr bool kCheckedBuild = false;
+#endif
+__device__ __forceinline__ bool checked(bool ok) {
+    if (kCheckedBuild && !ok) {
+        atomicOr(&g_device_status, kDevErrChecked);
+        return false;
+    }
+    return true;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -204,6 +224,7 @@ __device__ __forceinline__ bool elect_one() {
 // Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
 // that completes `bytes` transactions on mbarrier `bar`. Plain (no multicast).
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    if (!checked((dst & 15u) == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (bytes & 15u) == 0)) return;
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
@@ -213,8 +234,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // 2-D tiled tensor copy (TMA) global -> shared of one box of the tensor map at `tmap`
 // (a __grid_constant__ kernel parameter), box origin (c0 = innermost, c1), completing its
 // bytes on mbarrier `bar`. Plain (no multicast). c0 times the element size must be a
-// multiple of 16 bytes; parts of the box outside the tensor are filled with zeros.
+// multiple of 16 bytes (ESIZE = the element size in bytes, checked in the checked
+// build); parts of the box outside the tensor are filled with zeros.
+template <int ESIZE>
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
+    if (!checked(((c0 * ESIZE) & 15) == 0 && (dst & 15u) == 0)) return;
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
             "r"(dst),

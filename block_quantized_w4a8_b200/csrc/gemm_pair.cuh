@@ -363,13 +363,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairGeo<FMT>::NUM_TH
                 if (Gm::BITS == 4) {  // a box of 16 bytes x 64 rows per block
                     mbar_arrive_expect_tx(rb, uint32_t(nb * NWH * 16 + NWT * 16 * (Gm::AFF ? 2 : 1)));
                     for (int k = 0; k < nb; ++k)
-                        tma_load_2d(smem_addr(sp + OFF_RAW + k * NWH * 16), &tm_q, (b0 + k) * 16, nh0, rb);
+                        tma_load_2d<1>(smem_addr(sp + OFF_RAW + k * NWH * 16), &tm_q, (b0 + k) * 16, nh0, rb);
                 } else {  // one box of both blocks (b0 is even: its byte offset is a multiple of 16)
                     mbar_arrive_expect_tx(rb, uint32_t(S * Gm::BPB * NWH + NWT * 16 * 2));
-                    tma_load_2d(smem_addr(sp + OFF_RAW), &tm_q, b0 * Gm::BPB, nh0, rb);
+                    tma_load_2d<1>(smem_addr(sp + OFF_RAW), &tm_q, b0 * Gm::BPB, nh0, rb);
                 }
-                tma_load_2d(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
-                if (Gm::AFF) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
+                tma_load_2d<2>(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
+                if (Gm::AFF) tma_load_2d<2>(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
                 const uint32_t fb = bar(&ctrl->full[slot]);
                 mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK + (Gm::AFF ? TT * 16 : 0))));
                 bulk_g2s(smem_addr(sp + OFF_T), reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK,

@@ -376,10 +376,10 @@ __global__ void __launch_bounds__(Geo<FMT, TOKL, MN>::NUM_THREADS, 1)
                 const int e0 = (FMT == 0) ? b0 & ~7 : (b0 >> bsh) & ~7;
                 mbar_arrive_expect_tx(rb, uint32_t(nb * NW * 16 + (sc_tma ? NW * 16 * (FMT == 1 ? 2 : 1) : 0)));
                 for (int k = 0; k < nb; ++k)
-                    tma_load_2d(smem_addr(sp + OFF_RAW + k * NW * 16), &tm_q, (b0 + k) * 16, n0, rb);
+                    tma_load_2d<1>(smem_addr(sp + OFF_RAW + k * NW * 16), &tm_q, (b0 + k) * 16, n0, rb);
                 if (sc_tma) {
-                    tma_load_2d(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
-                    if (FMT == 1) tma_load_2d(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
+                    tma_load_2d<2>(smem_addr(sp + OFF_RSC), &tm_s, e0, n0, rb);
+                    if (FMT == 1) tma_load_2d<2>(smem_addr(sp + OFF_RBI), &tm_b, e0, n0, rb);
                 }
                 const uint32_t fb = bar(&ctrl->full[slot]);
                 mbar_arrive_expect_tx(fb, uint32_t(nb * (T_BLK + DX_BLK) + nz * TT * 4));

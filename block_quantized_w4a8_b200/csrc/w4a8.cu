@@ -862,6 +862,7 @@ w4a8_status w4a8_last_device_error(void) {
     if (cudaMemcpyFromSymbol(&v, w4a8::g_device_status, sizeof(v)) != cudaSuccess) return W4A8_ERR_CUDA;
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(w4a8::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (v & w4a8::kDevErrChecked) return W4A8_ERR_CHECK;  // the cause of any timeout that follows
     if (v & w4a8::kDevErrTimeout) return W4A8_ERR_DEVICE_TIMEOUT;
     return v ? W4A8_ERR_RANGE : W4A8_OK;
 }
@@ -878,6 +879,7 @@ const char* w4a8_status_string(w4a8_status s) {
         case W4A8_ERR_DEVICE_TIMEOUT: return "W4A8_ERR_DEVICE_TIMEOUT";
         case W4A8_ERR_MISALIGNED: return "W4A8_ERR_MISALIGNED";
         case W4A8_ERR_RANGE: return "W4A8_ERR_RANGE";
+        case W4A8_ERR_CHECK: return "W4A8_ERR_CHECK";
     }
     return "W4A8_UNKNOWN_STATUS";
 }

@@ -43,8 +43,11 @@ typedef enum {
     W4A8_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed */
     W4A8_ERR_DEVICE_TIMEOUT = 5, /* a bounded wait inside a kernel ran out (see w4a8_last_device_error) */
     W4A8_ERR_MISALIGNED = 6,     /* a pointer is not 16-byte aligned */
-    W4A8_ERR_RANGE = 7           /* a weight scale outside the tensor-core path's exact range
+    W4A8_ERR_RANGE = 7,          /* a weight scale outside the tensor-core path's exact range
                                     (see w4a8_gemm); reported by w4a8_last_device_error */
+    W4A8_ERR_CHECK = 8           /* checked build only (libw4a8_checked.so, -DW4A8_CHECKED): a
+                                    device-side check of a copy's alignment failed and the
+                                    copy was skipped; reported by w4a8_last_device_error */
 } w4a8_status;
 
 /* Element type of the unquantised input (x or W). bf16 is widened exactly to f32. */
@@ -300,9 +303,10 @@ w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dty
  * Reads and clears the device status word that kernels set when a bounded wait runs
  * out or a weight scale is outside the tensor-core path's range. Synchronises the
  * current device. Returns W4A8_OK when no kernel has reported a problem since the last
- * call, W4A8_ERR_DEVICE_TIMEOUT if a wait ran out (this takes precedence),
- * W4A8_ERR_RANGE if only a scale was out of range, W4A8_ERR_CUDA if the read itself
- * failed.
+ * call; else, in order of precedence: W4A8_ERR_CHECK (checked build only) if a device-side
+ * check failed (the timeout that the skipped copy causes is then reported as this),
+ * W4A8_ERR_DEVICE_TIMEOUT if a wait ran out, W4A8_ERR_RANGE if only a scale was out of
+ * range; W4A8_ERR_CUDA if the read itself failed.
  */
 w4a8_status w4a8_last_device_error(void);
 

@@ -157,3 +157,19 @@ def test_q4_k_argument_errors(lib):
     assert b(1, 4096, 4096, P(FAKE), P(FAKE), P(FAKE), P(0), 0, P(0)) == 3  # WORKSPACE missing
     assert lib.w4a8_q4_k_backward_workspace_bytes(1, 4096, 4000) == 0
     assert lib.w4a8_q4_k_backward_workspace_bytes(1, 8, 256) == 16      # one row range: no partials
+
+
+def test_checked_build_exports_the_same_boundary():
+    """The checked variant (-DW4A8_CHECKED: device-side checks of each copy's alignment,
+    reported as W4A8_ERR_CHECK) builds and exports every declared entry point."""
+    from block_quantized_w4a8_b200 import build
+    path = build.build(checked=True)
+    chk = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(chk, name), name
+    chk.w4a8_status_string.restype = ctypes.c_char_p
+    assert chk.w4a8_status_string(8) == b"W4A8_ERR_CHECK"
+
+
+def test_status_string_of_check(lib):
+    assert w4a8.w4a8_status_string(8) == "W4A8_ERR_CHECK"
