@@ -114,3 +114,26 @@ def test_q4_k_unit_scales_is_integer_matmul():
     x = np.random.default_rng(3).integers(-50, 50, size=(2, K))
     y, _ = oracle.gemv_q4_k(x.astype(np.float32), W, N)
     assert np.array_equal(y, (x @ codes.T).astype(np.float64))
+
+
+def test_oracle_agrees_with_the_pages_f32_sequence():
+    """The page's scalar GEMV in f32 (d1 = d*sc, m1 = dmin*m, w = d1*q - m1, then
+    sum += w * x element after element), written here with numpy float32 and a sequential
+    accumulation, is within the f32 bound (K + 2) * 2^-24 * T of the oracle's f64 result."""
+    N, K = 9, 1024
+    W = inputs.make_q4_k(N, K, seed=31).numpy()
+    x = inputs.randn((1, K), seed=32).numpy().astype(np.float32)
+    b = W.reshape(N, K // 256, 144)
+    d = b[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float32)
+    dmin = b[..., 2:4].copy().view(np.float16)[..., 0].astype(np.float32)
+    sc, m = ref.q4_k_scales(b[..., 4:16])
+    qs = b[..., 16:].reshape(N, K // 256, 4, 32).astype(np.int64)
+    codes = np.concatenate([qs & 15, qs >> 4], axis=-1).reshape(N, K // 256, 256).astype(np.float32)
+    sub = np.arange(256) // 32
+    d1 = (d[..., None] * sc[..., sub].astype(np.float32)).astype(np.float32)
+    m1 = (dmin[..., None] * m[..., sub].astype(np.float32)).astype(np.float32)
+    w = (d1 * codes).astype(np.float32) - m1                      # f32 subtraction, rounded
+    terms = (w.reshape(N, K) * x[0][None, :]).astype(np.float32)  # f32 products, rounded
+    y32 = np.add.accumulate(terms, axis=1, dtype=np.float32)[:, -1].astype(np.float64)
+    y, T = oracle.gemv_q4_k(x, W, N)
+    assert np.all(np.abs(y32 - y[0]) <= (K + 2) * 2.0 ** -24 * T[0])
