@@ -222,7 +222,7 @@ __device__ __forceinline__ bool elect_one() {
 
 // ------------------------------------------------------------------ bulk async copy
 // Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
-// that completes `bytes` transactions on mbarrier `bar`. Plain (no multicast).
+// that completes `bytes` transactions on mbarrier `bar`, into this CTA's shared memory only.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     if (!checked((dst & 15u) == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (bytes & 15u) == 0)) return;
     asm volatile(
@@ -233,7 +233,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 
 // 2-D tiled tensor copy (TMA) global -> shared of one box of the tensor map at `tmap`
 // (a __grid_constant__ kernel parameter), box origin (c0 = innermost, c1), completing its
-// bytes on mbarrier `bar`. Plain (no multicast). c0 times the element size must be a
+// bytes on mbarrier `bar`, into this CTA's shared memory only. c0 times the element size must be a
 // multiple of 16 bytes (ESIZE = the element size in bytes, checked in the checked
 // build); parts of the box outside the tensor are filled with zeros.
 template <int ESIZE>

@@ -37,7 +37,7 @@
 // row per thread: reads the stage's packed codes and scales, nibble -> scaled fp16
 // expansion, store in the core-matrix layout); one MMA-issue warp (also allocates TMEM);
 // one copy warp (2-D TMA boxes of the packed weights; token operand, d_x and Z via plain
-// cp.async.bulk; no multicast). The
+// cp.async.bulk, each CTA fetching its own data). The
 // MMA and copy warps run their loops warp-uniformly with one elected lane issuing. Every
 // wait is bounded and taken by each warp on its own (all lanes probe, a vote keeps the
 // warp converged), so no role is held in lockstep by its slowest warp; the epilogue
