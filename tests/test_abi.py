@@ -144,6 +144,15 @@ def test_affine_nbit_argument_errors(lib):
     assert pack(bits=7) == 2 and pack(group=256) == 2
     assert pack(K=96) == 1 and pack(q=0) == 1
     assert pack(q=FAKE + 8) == 6                       # MISALIGNED
+    e = w4a8.Epilogue()
+    e.bias, e.bias_dtype, e.out_dtype = FAKE, 0, 5     # unknown output type
+    assert lib.w4a8_gemm_affine_nbit(8, 8, 128, 64, 8, P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), ctypes.byref(e),
+                                     P(FAKE), P(FAKE), 1 << 40, 0, P(0)) == 2
+    e.out_dtype, e.bias = 0, FAKE + 2                   # f32 bias not 4-byte aligned
+    assert lib.w4a8_gemm_affine_nbit(8, 8, 128, 64, 6, P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), ctypes.byref(e),
+                                     P(FAKE), P(FAKE), 1 << 40, 0, P(0)) == 6
+    assert lib.w4a8_gemm_affine_nbit(8, 8, 128, 64, 8, P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), None,
+                                     P(FAKE), P(FAKE), 16, 0, P(0)) == 3   # workspace too small
 
 
 def test_q4_k_argument_errors(lib):
