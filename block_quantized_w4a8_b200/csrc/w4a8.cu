@@ -4,6 +4,8 @@
 
 #include <string.h>
 
+#include <mutex>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -833,12 +835,69 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
 }
 
 // Scratch of w4a8_gemm_noalloc. In host code this name is only a stand-in for the
-// device array; its device address comes from cudaGetSymbolAddress (once per device).
+// device array; its device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_BYTES];
+
+}  // extern "C"
+
+namespace {
+
+// Unique ID of the calling thread's current CUDA context (false when there is none, or
+// when the driver does not offer the query).
+bool current_context_id(unsigned long long* id) {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_noalloc_scratch in the current context of device `dev`. The address
+// belongs to a context, not to a device: after cudaDeviceReset the next context loads the
+// library's device code again and the array may sit elsewhere. So the looked-up address is
+// kept per device together with the ID of the context it was looked up in, and looked up
+// again whenever the current context differs (or cannot be identified). The cache is read
+// and filled under a lock, so first calls from several host threads do not race.
+cudaError_t noalloc_scratch_address(int dev, void** out) {
+    static std::mutex mu;
+    static bool valid[64] = {false};
+    static unsigned long long ctx_of[64] = {0};
+    static void* addr_of[64] = {nullptr};
+    std::lock_guard<std::mutex> lock(mu);
+    unsigned long long id = 0;
+    if (valid[dev] && current_context_id(&id) && id == ctx_of[dev]) {
+        *out = addr_of[dev];
+        return cudaSuccess;
+    }
+    void* p = nullptr;  // this lookup also creates the device's primary context if needed
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    valid[dev] = current_context_id(&id);
+    ctx_of[dev] = id;
+    addr_of[dev] = p;
+    *out = p;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
 
 w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
                               const uint16_t* d_fp16, float* y, cudaStream_t stream) {
-    static void* scratch_ptr[64] = {nullptr};
     const size_t need = (dims_ok(M, N) && dims_ok(K, 1) && K % 32 == 0) ? min_workspace_bytes(M, K, 0) : 0;
     if (need == 0) return W4A8_ERR_INVALID_ARG;
     if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
@@ -846,13 +905,10 @@ w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dty
     const cudaError_t ed = cudaGetDevice(&dev);
     if (ed != cudaSuccess) return cuda_status(ed);
     if (dev < 0 || dev >= 64) return W4A8_ERR_UNSUPPORTED;
-    if (scratch_ptr[dev] == nullptr) {  // set-up, once per device, with that device current
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_status(e);
-        scratch_ptr[dev] = p;
-    }
-    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, kPlain, scratch_ptr[dev], W4A8_NOALLOC_SCRATCH_BYTES,
+    void* scratch = nullptr;
+    const cudaError_t es = noalloc_scratch_address(dev, &scratch);
+    if (es != cudaSuccess) return cuda_status(es);
+    return gemm_impl<0>(M, N, K, 0, x, dtype, qs, d_fp16, nullptr, y, kPlain, scratch, W4A8_NOALLOC_SCRATCH_BYTES,
                         W4A8_PATH_AUTO, stream);
 }
 

@@ -283,7 +283,12 @@ w4a8_status w4a8_gemv_q4_k_backward(int M, int N, int K, const float* dy, const 
  * W4A8_NOALLOC_SCRATCH_BYTES (every GPU that loads the library holds it until the process
  * exits). The library itself never calls cudaMalloc or cudaFree here.
  *  - The first call on each device looks up that array's device address (with that device
- *    current), so that first call should come before any stream capture.
+ *    current), so that first call should come before any stream capture. The address
+ *    belongs to the device's CUDA context: after a context reset (cudaDeviceReset) the
+ *    library's device code is loaded again and the array may move, so the first call in
+ *    the new context looks it up again (same rule on stream capture). The looked-up
+ *    address is cached under a lock; concurrent first calls from several host threads
+ *    are safe.
  *  - Shapes whose minimum workspace (see w4a8_workspace_bytes) exceeds the array are
  *    rejected with W4A8_ERR_WORKSPACE; nothing is launched. Within the array the
  *    tensor-core path splits K only as far as its partial sums fit.
