@@ -362,7 +362,7 @@ def run_ours(args):
     k_us = ms_step * 1e3
     alg = weight_bytes(N, K) + M * K * 4 + M * N * 4   # packed weights + scales, f32 x, f32 y
     achieved = alg / (k_us * 1e-6) / 1e9
-    tkey = "gemv2_fused_m1_q4_0:decode_m1_4096x4096"
+    tkey = "gemv_resident_m1_q4_0:decode_m1_4096x4096"
 
     # the split form (quantise once, then the contraction kernel alone), for reference
     w4a8.w4a8_prepare_act(xd, ws)
@@ -405,7 +405,8 @@ def run_ours(args):
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic.get(tkey),
                      "traffic_note": None if traffic.get(tkey) is not None else
                      "no ncu capture of the current kernel build (profiles/ holds an earlier build's counters)",
-                     "kernel": "gemv2_kernel<1,0,1> (Q4_0, M=1, x quantised in-kernel; the whole step)",
+                     "kernel": "gemv_resident_kernel<1,0,true,XS> (Q4_0, M=1, weights resident in shared "
+                               "memory, x quantised in-kernel; the whole step)",
                      "kernel_us": k_us, "prepared_contraction_us": prepared_us,
                      "algorithmic_bytes_per_launch": alg, "peak_source": peaks.get("source", "measured") +
                      " (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"},

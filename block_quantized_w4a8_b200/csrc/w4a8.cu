@@ -15,6 +15,7 @@
 #include "gemm_pair.cuh"
 #include "q4k.cuh"
 #include "gemv.cuh"
+#include "gemv_resident.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -214,6 +215,96 @@ cudaError_t launch_gemv2_mt(int mt, int M, int N, int K, int group, const void* 
     }
 }
 
+// ------------------------------------------------------------------ resident GEMV
+// Geometry of one gemv_resident_kernel launch (see gemv_resident.cuh); ok = false when the
+// shape does not suit it: scale rows not a whole number of 16-byte pieces, K too long for
+// the lanes' registers, or a CTA's weights (beside the activation) beyond its share of
+// shared memory -- those shapes take gemv2_kernel.
+struct GvPlan {
+    bool ok = false;
+    int xs = 1, lnsw = 0, grid = 1;
+    size_t smem = 0;
+};
+// Shared memory per CTA such that two CTAs (of consecutive calls) fit on one SM.
+constexpr size_t kGvSmemMax = 112 * 1024;
+
+GvPlan gv_plan(int mt, int N, int K, int group, bool affine, bool quantise) {
+    GvPlan p;
+    const int B = K / 32;
+    const int E = affine ? K / group : B;
+    if (E % 8 != 0) return p;
+    const int NS = (B + 31) / 32;
+    const int G = N < sm_count() ? N : sm_count();
+    const int rc = int(cdiv(N, G));  // rows of the largest CTA
+    const size_t smem = gv::kHeaderBytes + gv::xregion_bytes(mt, K, quantise) +
+                        gv::resident_weight_bytes(rc, K, E, affine);
+    if (smem > kGvSmemMax) return p;
+    // Blocks per lane and row (xs): registers hold 8 words of x per block and token. The
+    // slice warps of a row group are the power of two covering the row's slices.
+    int64_t best = -1;
+    for (int c : {1, 2, 4}) {
+        if (c * mt > 8) continue;
+        int lnsw = 0;
+        while ((1 << lnsw) * c < NS) ++lnsw;
+        if (lnsw > 3) continue;
+        const int H = gv::warps_for(mt) >> lnsw;
+        const int64_t T = cdiv(rc, H);  // rows per group
+        // issue-slot estimate per warp: row-block dots, one reduce-scatter per pass (and a
+        // block barrier when a row's slices are on several warps), x codes per owned block
+        const int64_t cost =
+            T * c * (10 + 14 * mt) + cdiv(T, gv::rows_per_pass(mt, c)) * (40 + (lnsw ? 60 : 0)) + c * mt * 24;
+        if (best < 0 || cost < best) {
+            best = cost;
+            p.xs = c;
+            p.lnsw = lnsw;
+        }
+    }
+    if (best < 0) return p;
+    p.grid = G;
+    p.smem = smem;
+    p.ok = true;
+    return p;
+}
+
+template <int MT, int FMT, bool QX, int XS>
+cudaError_t launch_gv(const GvPlan& p, int M, int N, int K, int group, const void* x, int xbf16, const int8_t* qx,
+                      const float* dx, const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb,
+                      void* y, const Epilogue& epi, cudaStream_t stream) {
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gv::gemv_resident_kernel<MT, FMT, QX, XS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGvSmemMax));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    return launch_pdl(gv::gemv_resident_kernel<MT, FMT, QX, XS>, dim3(unsigned(p.grid)),
+                      dim3(gv::warps_for(MT) * 32), p.smem, stream, M, N, K, group, x, xbf16, qx, dx, sx, wq, ws, wb,
+                      y, epi, p.lnsw);
+}
+
+template <int FMT, bool QX>
+cudaError_t launch_gv_mt(const GvPlan& p, int mt, int M, int N, int K, int group, const void* x, int xbf16,
+                         const int8_t* qx, const float* dx, const int32_t* sx, const uint8_t* wq, const uint16_t* ws,
+                         const uint16_t* wb, void* y, const Epilogue& epi, cudaStream_t stream) {
+#define W4A8_GV(MT_, XS_) \
+    launch_gv<MT_, FMT, QX, XS_>(p, M, N, K, group, x, xbf16, qx, dx, sx, wq, ws, wb, y, epi, stream)
+    switch (mt * 8 + p.xs) {
+        case 1 * 8 + 1: return W4A8_GV(1, 1);
+        case 1 * 8 + 2: return W4A8_GV(1, 2);
+        case 1 * 8 + 4: return W4A8_GV(1, 4);
+        case 2 * 8 + 1: return W4A8_GV(2, 1);
+        case 2 * 8 + 2: return W4A8_GV(2, 2);
+        case 2 * 8 + 4: return W4A8_GV(2, 4);
+        case 4 * 8 + 1: return W4A8_GV(4, 1);
+        case 4 * 8 + 2: return W4A8_GV(4, 2);
+        case 8 * 8 + 1: return W4A8_GV(8, 1);
+        default: return cudaErrorInvalidConfiguration;
+    }
+#undef W4A8_GV
+}
+
 // True when one call can quantise x inside the GEMV (no separate act-quant launch).
 inline bool gemv_fused(int M, int K) {
     return int64_t(M) * K <= kFuseMaxElems && gemv2_smem_bytes(gemv_mt(M < 8 ? M : 8), K) <= kGemv2MaxSmem && M <= 8;
@@ -232,7 +323,10 @@ w4a8_status run_gemv(int M, int N, int K, int group, const GemvWs& a, const uint
         const int32_t* sx = a.sx + int64_t(m0) * B;
         void* yy = static_cast<char*>(y) + int64_t(m0) * N * (epi.out_bf16 ? 2 : 4);
         cudaError_t e;
-        if (gemv2_smem_bytes(mt, K) <= kGemv2MaxSmem) {
+        const GvPlan p = gv_plan(mt, N, K, group, FMT == 1, false);
+        if (p.ok) {
+            e = launch_gv_mt<FMT, false>(p, mt, mc, N, K, group, nullptr, 0, qx, dx, sx, wq, ws, wb, yy, epi, stream);
+        } else if (gemv2_smem_bytes(mt, K) <= kGemv2MaxSmem) {
             e = launch_gemv2_mt<FMT, 0>(mt, mc, N, K, group, nullptr, qx, dx, sx, wq, ws, wb, yy, epi, stream);
         } else {  // activation too large for shared memory: stream it from L1/L2
             const dim3 grid(unsigned(cdiv(N, kGemvWarps)));
@@ -285,6 +379,10 @@ template <int FMT>
 w4a8_status run_gemv_fused(int M, int N, int K, int group, const void* x, w4a8_dtype dt, const uint8_t* wq,
                            const uint16_t* ws, const uint16_t* wb, void* y, const Epilogue& epi, cudaStream_t stream) {
     const int mt = gemv_mt(M);
+    const GvPlan p = gv_plan(mt, N, K, group, FMT == 1, true);
+    if (p.ok)
+        return cuda_status(launch_gv_mt<FMT, true>(p, mt, M, N, K, group, x, dt == W4A8_BF16 ? 1 : 0, nullptr, nullptr,
+                                                   nullptr, wq, ws, wb, y, epi, stream));
     cudaError_t e = (dt == W4A8_BF16)
                         ? launch_gemv2_mt<FMT, 2>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, epi, stream)
                         : launch_gemv2_mt<FMT, 1>(mt, M, N, K, group, x, nullptr, nullptr, nullptr, wq, ws, wb, y, epi, stream);

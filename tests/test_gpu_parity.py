@@ -117,7 +117,10 @@ def test_pack_affine_bit_exact(group, N, K, dtype):
 # pairs; the other M > 64 shapes take the single-CTA kernel (scale rows not 16-B aligned).
 SHAPES = [(1, 1, 32), (1, 4096, 4096), (2, 333, 800), (5, 1536, 384), (8, 200, 256), (17, 96, 640),
           (32, 520, 1056), (64, 1536, 384), (300, 333, 800), (129, 128, 128), (130, 257, 4128), (3, 64, 32768),
-          (300, 333, 1024), (200, 512, 4096)]
+          (300, 333, 1024), (200, 512, 4096),
+          # bulk-copy GEMV: fewer rows than SMs, rows not a multiple of the SM count, long K,
+          # several stage refills per CTA, eight tokens at the sweep's K
+          (1, 100, 2048), (6, 1000, 2048), (1, 1000, 14336), (4, 2000, 4096), (8, 300, 8192)]
 
 
 def _q4_0_case(M, N, K, x_dtype="f32", w_std=0.02, seed=0):
