@@ -591,13 +591,26 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __rest
                                                              int N, void* __restrict__ y, Epilogue epi) {
     pdl_wait_primary();  // the partials are written by the preceding GEMM
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
-        float4 a = part[i];
-        for (int z = 1; z < ks; ++z) {
-            const float4 b = part[int64_t(z) * n4 + i];
-            a.x = __fadd_rn(a.x, b.x);
-            a.y = __fadd_rn(a.y, b.y);
-            a.z = __fadd_rn(a.z, b.z);
-            a.w = __fadd_rn(a.w, b.w);
+        // splits in order, in groups of 16 whose sums are added in order (at most 15 + ks/16
+        // roundings in any output's chain)
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int z0 = 0; z0 < ks; z0 += 16) {
+            float4 g = part[int64_t(z0) * n4 + i];
+            for (int z = z0 + 1; z < ks && z < z0 + 16; ++z) {
+                const float4 b = part[int64_t(z) * n4 + i];
+                g.x = __fadd_rn(g.x, b.x);
+                g.y = __fadd_rn(g.y, b.y);
+                g.z = __fadd_rn(g.z, b.z);
+                g.w = __fadd_rn(g.w, b.w);
+            }
+            if (z0 == 0) {
+                a = g;
+            } else {
+                a.x = __fadd_rn(a.x, g.x);
+                a.y = __fadd_rn(a.y, g.y);
+                a.z = __fadd_rn(a.z, g.z);
+                a.w = __fadd_rn(a.w, g.w);
+            }
         }
         if (!epi.bias && !epi.out_bf16) {
             reinterpret_cast<float4*>(y)[i] = a;
@@ -608,6 +621,22 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __rest
 #pragma unroll
             for (int j = 0; j < 4; ++j) epi_store(y, 4 * i + j, int((4 * i + j) % N), v[j], epi);
         }
+    }
+}
+
+// The same reduction element by element, for M * N not a multiple of 4 (partial z of
+// output i at part[z * n + i]).
+__global__ void __launch_bounds__(256) splitk_reduce_scalar_kernel(const float* __restrict__ part, int ks, int64_t n,
+                                                                    int N, void* __restrict__ y, Epilogue epi) {
+    pdl_wait_primary();  // the partials are written by the preceding GEMM
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+        float a = 0.0f;
+        for (int z0 = 0; z0 < ks; z0 += 16) {  // in groups of 16, as splitk_reduce_kernel
+            float g = part[int64_t(z0) * n + i];
+            for (int z = z0 + 1; z < ks && z < z0 + 16; ++z) g = __fadd_rn(g, part[int64_t(z) * n + i]);
+            a = (z0 == 0) ? g : __fadd_rn(a, g);
+        }
+        epi_store(y, i, int(i % N), a, epi);
     }
 }
 

@@ -78,12 +78,15 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(int M, int N, int K, con
     const int nb = K >> 8;
     const int n0 = blockIdx.x * 4 * RG;
     const int e0 = 64 * (c >> 1) + 16 * (c & 1);  // first element of the chunk's low nibbles
-    float acc[RG][MT];
+    // Three levels of f32 sums keep every output's rounding chain short at any K: a
+    // super-block's 32 products (sb_acc), 16 super-blocks of a warp (mid), the rest (acc).
+    float acc[RG][MT], mid[RG][MT];
 #pragma unroll
     for (int g = 0; g < RG; ++g)
 #pragma unroll
-        for (int m = 0; m < MT; ++m) acc[g][m] = 0.0f;
-    for (int sb = warp; sb < nb; sb += kWarps) {
+        for (int m = 0; m < MT; ++m) acc[g][m] = mid[g][m] = 0.0f;
+    int step = 0;
+    for (int sb = warp; sb < nb; sb += kWarps, ++step) {
         float xs[MT][32];  // x[m][sb*256 + e0 + t] (t < 16) and x[m][sb*256 + e0 + 32 + t]
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
@@ -113,6 +116,9 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(int M, int N, int K, con
         for (int g = 0; g < RG; ++g) {
             const ChunkScales cs = chunk_scales(h[g], c);
             const uint32_t qw[4] = {q[g].x, q[g].y, q[g].z, q[g].w};
+            float sb_acc[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) sb_acc[m] = 0.0f;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
 #pragma unroll
@@ -121,13 +127,28 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(int M, int N, int K, con
                     const float wh = fmaf(cs.d_hi, code_f(qw[v], 8 * b + 4), -cs.m_hi);
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
-                        acc[g][m] = fmaf(wl, xs[m][4 * v + b], acc[g][m]);
-                        acc[g][m] = fmaf(wh, xs[m][16 + 4 * v + b], acc[g][m]);
+                        sb_acc[m] = fmaf(wl, xs[m][4 * v + b], sb_acc[m]);
+                        sb_acc[m] = fmaf(wh, xs[m][16 + 4 * v + b], sb_acc[m]);
                     }
                 }
             }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) mid[g][m] += sb_acc[m];
+        }
+        if ((step & 15) == 15) {
+#pragma unroll
+            for (int g = 0; g < RG; ++g)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    acc[g][m] += mid[g][m];
+                    mid[g][m] = 0.0f;
+                }
         }
     }
+#pragma unroll
+    for (int g = 0; g < RG; ++g)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[g][m] += mid[g][m];
 #pragma unroll
     for (int g = 0; g < RG; ++g)
 #pragma unroll
@@ -158,7 +179,8 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(int M, int N, int K, con
 // chunk's 32 elements over the rows it visits; the four lanes that hold the same chunk
 // (one per row of a group) and then the 8 warps are added in a fixed order, and the CTA
 // writes its partial sums to part[r][m][k] (or dX directly when there is one row range),
-// so the result does not depend on scheduling.
+// so the result does not depend on scheduling. A row range holds at most 2048 rows, so a
+// lane's chain of products is at most 64 long.
 template <int MT>
 __global__ void __launch_bounds__(kThreads) bwd_kernel(int M, int N, int K, int rows, const float* __restrict__ dy,
                                                      const uint8_t* __restrict__ W, float* __restrict__ out) {
@@ -246,12 +268,17 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(int M, int N, int K, int 
     }
 }
 
-// dX[i] = sum over row ranges r = 0..R-1 (in order) of part[r][i], i < M*K.
+// dX[i] = sum over row ranges r = 0..R-1 of part[r][i], i < M*K: in order, in groups of 16
+// whose sums are added in order (at most 15 + R/16 roundings in a chain).
 __global__ void __launch_bounds__(256) bwd_reduce_kernel(const float* __restrict__ part, int R, int64_t count,
                                                          float* __restrict__ dx) {
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += int64_t(gridDim.x) * blockDim.x) {
         float v = 0.0f;
-        for (int r = 0; r < R; ++r) v += part[int64_t(r) * count + i];
+        for (int r0 = 0; r0 < R; r0 += 16) {
+            float g = part[int64_t(r0) * count + i];
+            for (int r = r0 + 1; r < R && r < r0 + 16; ++r) g += part[int64_t(r) * count + i];
+            v = (r0 == 0) ? g : v + g;
+        }
         dx[i] = v;
     }
 }

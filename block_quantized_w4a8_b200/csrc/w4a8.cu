@@ -399,21 +399,32 @@ struct KSplit {
 };
 inline int64_t tc_tiles(int M, int N) { return cdiv(N, 128) * tc_token_tiles(M); }
 inline size_t partial_bytes(int ks, int M, int N) { return ks > 1 ? align256(size_t(ks) * M * N * 4) : 0; }
+// Longest chain of per-block f32 additions the tensor-core epilogue makes for one output.
+// Summing n terms one rounding at a time errs by at most n * 2^-24 * sum|terms|. With at
+// most 128 blocks per split, the splits added in groups of 16 (at most 15 + 15 roundings
+// for ks <= 256, i.e. K <= 2^20) and the two roundings of the weight operand's hi/lo parts,
+// every output stays within (128 + 30 + 2) * 2^-24 < 9.6e-6 of the exact sum relative to
+// sum|terms|: inside the API's 1e-5 tolerance at every K.
+constexpr int kMaxChainBlocks = 128;
+inline int tc_split_min(int K) { return int(cdiv(K / 32, kMaxChainBlocks)); }
 int tc_split_pref(int M, int N, int K) {
-    if ((int64_t(M) * N) % 4 != 0) return 1;  // the reduction works on float4
+    const int kmin = tc_split_min(K);
+    if ((int64_t(M) * N) % 4 != 0) return kmin;  // the fast reduction works on float4
     const int64_t tiles = tc_tiles(M, N);
     const int sms = sm_count();
-    if (tiles >= sms) return 1;
+    if (tiles >= sms) return kmin;
     int ks = int(sms / tiles);
     const int by_k = (K / 32) / 16;
     if (ks > by_k) ks = by_k;
-    return ks < 1 ? 1 : ks;
+    return ks < kmin ? kmin : ks;
 }
-// The split for this call: the preferred one, reduced until its partials fit `work_bytes`.
+// The split for this call: the preferred one, reduced until its partials fit `work_bytes`,
+// but never below the split that bounds the accumulation chain.
 KSplit tc_split(int M, int N, int K, size_t base_bytes, size_t work_bytes) {
     const int B = K / 32;
+    const int kmin = tc_split_min(K);
     int ks = tc_split_pref(M, N, K);
-    while (ks > 1 && base_bytes + partial_bytes(ks, M, N) > work_bytes) --ks;
+    while (ks > kmin && base_bytes + partial_bytes(ks, M, N) > work_bytes) --ks;
     KSplit sp{1, B};
     if (ks > 1) {
         sp.bsplit = int((cdiv(B, ks) + 7) / 8 * 8);
@@ -421,6 +432,23 @@ KSplit tc_split(int M, int N, int K, size_t base_bytes, size_t work_bytes) {
         if (sp.ks < 2) sp = KSplit{1, B};
     }
     return sp;
+}
+
+// Sum of the ks partial outputs in split order (+ epilogue) into y.
+w4a8_status run_splitk_reduce(const float* part, int ks, int M, int N, void* y, const Epilogue& epi,
+                              cudaStream_t stream) {
+    const int64_t n = int64_t(M) * N;
+    const int64_t units = (n % 4 == 0) ? n / 4 : n;
+    int64_t rb = cdiv(units, 256);
+    if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
+    cudaError_t e;
+    if (n % 4 == 0)
+        e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream,
+                       reinterpret_cast<const float4*>(part), ks, units, N, y, epi);
+    else
+        e = launch_pdl(tc::splitk_reduce_scalar_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, part, ks, n, N, y,
+                       epi);
+    return cuda_status(e);
 }
 
 // cuTensorMapEncodeTiled, resolved once through the runtime (no link against the driver
@@ -497,12 +525,7 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
                                   (const float*)w.dxs, (const float*)w.z, wq, ws, wb, y, tq, tsc, tbi, sc_tma,
                                   sp.bsplit, part, epi);
     if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
-    const int64_t n4 = int64_t(M) * N / 4;
-    int64_t rb = cdiv(n4, 256);
-    if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
-    e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, (const float4*)part, sp.ks, n4,
-                   N, y, epi);
-    return cuda_status(e);
+    return run_splitk_reduce(part, sp.ks, M, N, y, epi, stream);
 }
 
 // CTA-pair kernel for 128-token tiles: two consecutive token tiles share one 128-row
@@ -542,12 +565,7 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
                                   size_t(Gm::SMEM_BYTES), stream, M, N, K, group, (const __half*)w.tok,
                                   (const float*)w.dxs, (const uint4*)w.sums, y, tq, tsc, tbi, sp.bsplit, part, epi);
     if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
-    const int64_t n4 = int64_t(M) * N / 4;
-    int64_t rb = cdiv(n4, 256);
-    if (rb > 4 * int64_t(sm_count())) rb = 4 * int64_t(sm_count());
-    e = launch_pdl(tc::splitk_reduce_kernel, dim3(unsigned(rb)), dim3(256), 0, stream, (const float4*)part, sp.ks, n4,
-                   N, y, epi);
-    return cuda_status(e);
+    return run_splitk_reduce(part, sp.ks, M, N, y, epi, stream);
 }
 
 // Orientation by token tile: tiles of 16..64 tokens put the tokens on the MMA's N; tiles
@@ -570,12 +588,15 @@ w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uin
     }
 }
 
-// Smallest workspace any call of this shape accepts (no split of K); a larger one, up to
-// w4a8_workspace_bytes, lets the tensor-core path split K.
-size_t min_workspace_bytes(int M, int K, int group) {
-    const size_t a = gemv_ws(nullptr, M, K).bytes;
-    const size_t b = tc_ws(nullptr, M, K, group).bytes;
-    return a > b ? a : b;
+inline bool use_gemv(int M, w4a8_path path);
+
+// Smallest workspace a call of this shape accepts on `path`: the GEMV's activation, or the
+// tensor-core operand plus the partial outputs of the split of K that bounds the
+// accumulation chain (K > 4096); a larger one, up to w4a8_workspace_bytes, lets the
+// tensor-core path split K further to fill the SMs.
+size_t min_workspace_bytes(int M, int N, int K, int group, w4a8_path path) {
+    if (use_gemv(M, path)) return gemv_ws(nullptr, M, K).bytes;
+    return tc_ws(nullptr, M, K, group).bytes + partial_bytes(tc_split_min(K), M, N);
 }
 
 w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
@@ -593,7 +614,7 @@ w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, c
         return W4A8_ERR_MISALIGNED;
     if (!work) return W4A8_ERR_WORKSPACE;
     if (!aligned16(work)) return W4A8_ERR_MISALIGNED;
-    if (work_bytes < min_workspace_bytes(M, K, affine ? group : 0)) return W4A8_ERR_WORKSPACE;
+    if (work_bytes < min_workspace_bytes(M, N, K, affine ? group : 0, path)) return W4A8_ERR_WORKSPACE;
     return W4A8_OK;
 }
 
@@ -712,12 +733,14 @@ w4a8_status pack_affine_impl(const void* w, w4a8_dtype dtype, int N, int K, int 
 
 // ------------------------------------------------------------------ Q4_K
 // Row ranges of the backward: enough CTAs (super-block columns x ranges) for four per
-// SM, at least 32 rows per range.
+// SM, at least 32 rows per range, at most 2048 (a lane's f32 chain of products is then at
+// most 64 long).
 inline int q4k_row_ranges(int N, int K) {
     const int nb = K / 256;
     int64_t R = cdiv(4 * int64_t(sm_count()), nb);
     const int64_t rmax = cdiv(N, 32);
     if (R > rmax) R = rmax;
+    if (R < cdiv(N, 2048)) R = cdiv(N, 2048);
     if (R < 1) R = 1;
     const int rows = int(cdiv(N, R));
     return int(cdiv(N, rows));
@@ -996,7 +1019,8 @@ extern "C" {
 
 w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
                               const uint16_t* d_fp16, float* y, cudaStream_t stream) {
-    const size_t need = (dims_ok(M, N) && dims_ok(K, 1) && K % 32 == 0) ? min_workspace_bytes(M, K, 0) : 0;
+    const size_t need =
+        (dims_ok(M, N) && dims_ok(K, 1) && K % 32 == 0) ? min_workspace_bytes(M, N, K, 0, W4A8_PATH_AUTO) : 0;
     if (need == 0) return W4A8_ERR_INVALID_ARG;
     if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
     int dev = 0;

@@ -93,10 +93,13 @@ w4a8_status w4a8_quant_act_q8_0(const void* x, w4a8_dtype dtype, int M, int K,
  * Size in bytes of the workspace w4a8_gemm / w4a8_gemm_affine use for this shape
  * (group = 0 for Q4_0, else the affine group size) on the current device. Covers every
  * path, so one allocation serves AUTO and both forced paths. It includes room for the
- * tensor-core path to split K when the output tiles do not fill the SMs (partial sums,
- * reduced in a fixed order). A smaller workspace is accepted down to the unsplit minimum
- * (the split then shrinks to what fits, which can change the last bits of the result);
- * below that minimum the calls return W4A8_ERR_WORKSPACE. Returns 0 for invalid sizes.
+ * tensor-core path's split of K (partial sums, reduced in a fixed order): at least one
+ * split per 128 quant blocks (K > 4096), which bounds each output's f32 accumulation
+ * chain, and more when the output tiles do not fill the SMs. A smaller workspace is
+ * accepted down to the minimum of the path the call takes (GEMV: the quantised
+ * activation; tensor cores: the operand plus the partial sums of the bounding split); the
+ * extra split then shrinks to what fits, which can change the last bits of the result.
+ * Below that minimum the calls return W4A8_ERR_WORKSPACE. Returns 0 for invalid sizes.
  */
 size_t w4a8_workspace_bytes(int M, int N, int K, int group);
 
@@ -104,10 +107,12 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group);
  * y = x . W^T with W in Q4_0 (from w4a8_pack_q4_0) and x quantised to Q8_0 inside the
  * call: y[m][n] = sum_b f32(d_w[n][b]) * d_x[m][b] * D[m][n][b], with
  * D = sum_{j<32} (q_w - 8) * q_x computed exactly. The sum over blocks is taken in f32;
- * each output is within 1e-5 * sum_b |term_b| of the exact value.
+ * each output is within 1e-5 * sum_b |term_b| of the exact value at every K: the GEMV
+ * paths add at most a few dozen terms in any chain, and the tensor-core path splits K so
+ * that no chain is longer than 128 blocks (error <= 160 * 2^-24 * sum_b |term_b|).
  * x        : M x K, f32 or bf16.       qs, d_fp16 : as produced by w4a8_pack_q4_0.
  * y        : out, M x N f32.           ws, ws_bytes : scratch of w4a8_workspace_bytes(M, N,
- *            K, 0) bytes (or at least the unsplit minimum, see there), owned by the
+ *            K, 0) bytes (or at least the path's minimum, see there), owned by the
  *            caller; contents on entry are ignored and are garbage afterwards. Calls
  *            that share a workspace must be ordered on one stream.
  * Scale range: the tensor-core path (M > 8, or PATH_GEMM) holds d_w * (q - 8) exactly as

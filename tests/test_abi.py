@@ -50,7 +50,8 @@ def _align(v):
 
 @pytest.mark.parametrize("M,N,K,group", [(1, 4096, 4096, 0), (64, 1536, 384, 0), (1024, 4096, 4096, 0),
                                          (1024, 4096, 4096, 64), (1024, 4096, 4096, 128), (300, 333, 800, 0),
-                                         (300, 333, 800, 32), (20, 64, 256, 32)])
+                                         (300, 333, 800, 32), (20, 64, 256, 32), (4096, 4096, 14336, 0),
+                                         (256, 4096, 14336, 0), (3, 5, 8192, 0), (100, 333, 8192, 64)])
 def test_workspace_bytes(lib, M, N, K, group):
     B = K // 32
     gemv = _align(M * K) + _align(M * B * 4) + _align(M * B * 4)
@@ -62,12 +63,14 @@ def test_workspace_bytes(lib, M, N, K, group):
     tc = _align(rows * B * 64) + _align(rows * B * 4) + (_align(rows * (K // group) * 4) if group else 0)
     if group and tt == 128:  # affine on CTA pairs: 16 bytes of code sums per token and block
         tc += _align(rows * B * 16)
-    # split of K when the output tiles do not fill the SMs (148 without a GPU): partial
-    # outputs of M*N f32 per split, at least 16 quant blocks per split
+    # split of K: at least one split per 128 quant blocks (the accumulation chain bound),
+    # more when the output tiles do not fill the SMs (148 without a GPU): partial outputs of
+    # M*N f32 per split, at least 16 quant blocks per split
     tiles = -(-N // 128) * ntok
-    ks = 1
+    kmin = -(-B // 128)
+    ks = kmin
     if (M * N) % 4 == 0 and tiles < 148:
-        ks = max(1, min(148 // tiles, B // 16))
+        ks = max(kmin, min(148 // tiles, B // 16))
     if ks > 1:
         tc += _align(ks * M * N * 4)
     assert w4a8.w4a8_workspace_bytes(M, N, K, group) == max(gemv, tc)

@@ -1,8 +1,8 @@
 """Q4_K GEMV and its input-gradient backward on the GPU against the oracle, element by
-element. Tolerance from the f32 arithmetic: each output is one chain of fused
-multiply-adds per lane (forward: K/8 terms; backward: about N/32 rows), then a fixed
-tree of additions (at most 16 more roundings, plus the row ranges of the backward), and
-each weight is rounded once: |y - y_ref| <= (chain + 32) * 2^-24 * T with T = sum |terms|."""
+element, held to the same bound as every other contraction: |y - y_ref| <= 1e-5 * T with
+T = sum |terms| (terms exact in the oracle's f64). The kernels keep every f32 chain short
+at any size: the forward sums a super-block's 32 products, then 16 super-blocks, then the
+rest, and the backward caps a row range at 2048 rows and adds the ranges in groups of 16."""
 import numpy as np
 import pytest
 import torch
@@ -12,19 +12,20 @@ import oracle
 from block_quantized_w4a8_b200 import inputs
 
 pytestmark = pytest.mark.gpu
-U = 2.0 ** -24
+TOL = 1e-5
 
 
-def _check(got, ref, T, chain, what):
+def _check(got, ref, T, what):
     err = np.abs(got.astype(np.float64) - ref)
-    tol = (chain + 32) * U * T
+    tol = TOL * T
     bad = err > tol
     assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside; worst {np.max(err / np.maximum(T, 1e-300))}"
 
 
 # (M, N, K): one token, two, an odd count (a one-token tail launch), ragged N (row groups
-# of 4 and CTAs of 32 rows), a single super-block, full decode size
-SHAPES = [(1, 300, 256), (2, 77, 512), (3, 129, 1024), (5, 1000, 2048), (1, 4096, 4096)]
+# of 4 and CTAs of 32 rows), a single super-block, full decode size, long K (more than 16
+# super-blocks per warp: all three levels of the sum)
+SHAPES = [(1, 300, 256), (2, 77, 512), (3, 129, 1024), (5, 1000, 2048), (1, 4096, 4096), (1, 64, 65536)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -34,11 +35,13 @@ def test_gemv_q4_k_vs_oracle(M, N, K):
     yref, T = oracle.gemv_q4_k(x.numpy(), W.numpy(), N, nthreads=8)
     y = w4a8.gemv_q4_k(x.cuda(), W.cuda())
     torch.cuda.synchronize()
-    _check(y.cpu().numpy(), yref, T, K // 8, f"forward M={M} N={N} K={K}")
+    _check(y.cpu().numpy(), yref, T, f"forward M={M} N={N} K={K}")
 
 
-# backward: one row range (small N) and several (partial sums reduced in order)
-BSHAPES = [(1, 300, 256), (2, 77, 512), (3, 1000, 1024), (1, 4096, 4096), (4, 2048, 4096)]
+# backward: one row range (small N) and several (partial sums reduced in order), many
+# ranges (more than 16: grouped reduction), long K with N above one range's 2048 rows
+BSHAPES = [(1, 300, 256), (2, 77, 512), (3, 1000, 1024), (1, 4096, 4096), (4, 2048, 4096), (1, 8192, 256),
+           (1, 5000, 65536)]
 
 
 @pytest.mark.parametrize("M,N,K", BSHAPES)
@@ -48,7 +51,7 @@ def test_gemv_q4_k_backward_vs_oracle(M, N, K):
     dxref, T = oracle.gemv_q4_k_backward(dy.numpy(), W.numpy(), K, nthreads=8)
     dx = w4a8.gemv_q4_k_backward(dy.cuda(), W.cuda(), K)
     torch.cuda.synchronize()
-    _check(dx.cpu().numpy(), dxref, T, N // 32 + 1, f"backward M={M} N={N} K={K}")
+    _check(dx.cpu().numpy(), dxref, T, f"backward M={M} N={N} K={K}")
 
 
 def test_backward_is_deterministic():
