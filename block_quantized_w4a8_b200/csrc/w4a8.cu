@@ -13,6 +13,7 @@
 #include "device_common.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_i8.cuh"
 #include "q4k.cuh"
 #include "gemv.cuh"
 #include "gemv_resident.cuh"
@@ -72,6 +73,11 @@ inline int tc_token_tiles(int M) {
     const int n = int(cdiv(M, tt));
     return (tt == 128) ? (n + 1) / 2 * 2 : n;
 }
+
+// Q4_0 with at most 64 tokens per tile takes the int8 tensor-core kernel (gemm_i8.cuh)
+// when the scale rows can be fetched by TMA (K a multiple of 256). The decision depends on
+// M, K and the format only, so the prepared form (quantise, then contract) agrees with it.
+inline bool use_i8(int M, int K, int group) { return group == 0 && tc_token_tile(M) <= 64 && K % 256 == 0; }
 
 struct TcWs {  // tensor-core operand layout (see quant_act_tc_kernel)
     __half* tok;
@@ -140,6 +146,14 @@ w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, 
                          bool wide = false) {
     const int64_t nblocks = int64_t(w.tiles) * w.tt * (K / 32);
     const dim3 grid(unsigned(cdiv(nblocks * 8, 256)));
+    if (!wide && use_i8(M, K, group)) {  // int8 token operand for gemm_i8_kernel
+        int8_t* tok = reinterpret_cast<int8_t*>(w.tok);
+        if (dt == W4A8_BF16)
+            quant_act_i8_kernel<true><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, tok, w.dxs);
+        else
+            quant_act_i8_kernel<false><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, tok, w.dxs);
+        return launch_status();
+    }
     if (wide) {
         if (dt == W4A8_BF16)
             quant_act_tc_kernel<true, 2><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
@@ -468,9 +482,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 2-D tensor map over a row-major [rows][cols] array of `esize`-byte elements with row
-// pitch `pitch` bytes, box [box_rows][box_cols]; no swizzle, zero fill outside.
+// pitch `pitch` bytes, box [box_rows][box_cols]; zero fill outside; no swizzle unless given.
 bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols, uint64_t rows,
-               uint64_t pitch, uint32_t box_cols, uint32_t box_rows) {
+               uint64_t pitch, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};
@@ -478,9 +493,8 @@ bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     (void)esize;
-    return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int FMT, bool TOKL, int MN>
@@ -568,6 +582,42 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
     return run_splitk_reduce(part, sp.ks, M, N, y, epi, stream);
 }
 
+// int8 tensor-core kernel for Q4_0, 16..64 tokens per tile (use_i8).
+template <int MN>
+w4a8_status launch_gemm_i8(int M, int N, int K, const TcWs& w, const uint8_t* wq, const uint16_t* ws, void* y,
+                           const Epilogue& epi, bool pdl, size_t work_bytes, cudaStream_t stream) {
+    using Gm = i8::Geo<MN>;
+    static bool configured[64] = {false};
+    int dev = 0;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return cuda_status(ed);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        const cudaError_t ea = cudaFuncSetAttribute(i8::gemm_i8_kernel<MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    Gm::SMEM_BYTES);
+        if (ea != cudaSuccess) return cuda_status(ea);
+        configured[dev] = true;
+    }
+    // Codes as bytes [N][K/2] in boxes of 128 bytes (8 quant blocks) x 128 rows, 128-byte
+    // swizzle (K is a multiple of 256: every stage is one whole box).
+    CUtensorMap tq;
+    if (!encode_2d(&tq, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 128,
+                   Gm::NW, CU_TENSOR_MAP_SWIZZLE_128B))
+        return W4A8_ERR_CUDA;
+    // Scales as fp16 [N][K/32] in boxes of 8 (one stage) x 128 rows.
+    CUtensorMap ts;
+    if (!encode_2d(&ts, ws, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(K / 32), uint64_t(N), uint64_t(K / 32) * 2,
+                   Gm::S, Gm::NW))
+        return W4A8_ERR_CUDA;
+    const KSplit sp = tc_split(M, N, K, w.bytes, work_bytes);
+    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(w.tok) + w.bytes);
+    const dim3 grid(unsigned(cdiv(N, Gm::NW)), unsigned(w.tiles), unsigned(sp.ks));
+    cudaError_t e = launch_pdl_if(pdl, i8::gemm_i8_kernel<MN>, grid, dim3(Gm::NUM_THREADS), size_t(Gm::SMEM_BYTES),
+                                  stream, M, N, K, (const int8_t*)w.tok, (const float*)w.dxs, y, tq, ts,
+                                  sp.bsplit, part, epi);
+    if (e != cudaSuccess || sp.ks == 1) return cuda_status(e);
+    return run_splitk_reduce(part, sp.ks, M, N, y, epi, stream);
+}
+
 // Orientation by token tile: tiles of 16..64 tokens put the tokens on the MMA's N; tiles
 // of 128 tokens put them on the TMEM lanes with 128 weight rows per tile, on CTA pairs
 // when the scale rows can be fetched by TMA (their pitch a multiple of 16 bytes).
@@ -575,6 +625,13 @@ template <int FMT>
 w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uint8_t* wq, const uint16_t* ws,
                         const uint16_t* wb, void* y, const Epilogue& epi, bool pdl, size_t work_bytes,
                         cudaStream_t stream) {
+    if (FMT == 0 && use_i8(M, K, group)) {
+        switch (w.tt) {
+            case 16: return launch_gemm_i8<16>(M, N, K, w, wq, ws, y, epi, pdl, work_bytes, stream);
+            case 32: return launch_gemm_i8<32>(M, N, K, w, wq, ws, y, epi, pdl, work_bytes, stream);
+            default: return launch_gemm_i8<64>(M, N, K, w, wq, ws, y, epi, pdl, work_bytes, stream);
+        }
+    }
     switch (w.tt) {
         case 16: return launch_gemm_tc<FMT, false, 16>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
         case 32: return launch_gemm_tc<FMT, false, 32>(M, N, K, group, w, wq, ws, wb, y, epi, pdl, work_bytes, stream);
