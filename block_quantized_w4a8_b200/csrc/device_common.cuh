@@ -169,6 +169,16 @@ __device__ __forceinline__ bool bounded_wait_warp(uint32_t bar, uint32_t parity,
     return bounded_wait_warp_slow<CLUSTER>(bar, parity, abort);
 }
 
+// Warp-wide wait for two barriers: both probed at once on the fast path (one round trip
+// when both phases are already complete), else each waited for in turn.
+__device__ __forceinline__ bool bounded_wait2_warp(uint32_t bar1, uint32_t parity1, uint32_t bar2, uint32_t parity2,
+                                                   volatile uint32_t* abort) {
+    const bool a = mbar_try_wait_nohint(bar1, parity1);
+    const bool b = mbar_try_wait_nohint(bar2, parity2);
+    if (__all_sync(0xffffffffu, a && b)) return true;
+    return bounded_wait_warp(bar1, parity1, abort) && bounded_wait_warp(bar2, parity2, abort);
+}
+
 // Named hardware barrier over `nthreads` threads (whole warps); waiting warps issue
 // nothing until the last one arrives.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {

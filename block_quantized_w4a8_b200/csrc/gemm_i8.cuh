@@ -23,15 +23,18 @@
 // Pipelines: a ring of raw code boxes (one 2-D TMA box of 128 rows x 128 bytes -- 8 blocks
 // of codes -- per stage, 128-byte swizzled so that the producers' 16-byte reads down a
 // column are conflict-free) that the copy warp keeps full from the start, before the grid
-// waits on its predecessor; a ring of MMA operands (expanded weights, token codes) that
-// the MMA warp itself hands back, by a tensor-core commit, once the stage's MMAs are done;
+// waits on its predecessor; a ring of MMA operands -- the expanded weights in tensor memory
+// (the MMA's A from TMEM: row p of the tile is lane p, written by the thread that expanded
+// it, so the expansion costs no shared-memory bandwidth), the token codes in shared memory
+// -- that the MMA warp itself hands back, by a tensor-core commit, once the stage's MMAs
+// are done;
 // and a ring of the stage's weight scales (one TMA box of 128 rows x 8 fp16) and d_x rows
 // that the epilogue hands back: the epilogue reads every operand from shared memory,
 // never waiting on a global load behind the weight stream. So the producers run ahead of the
 // tensor core by the operand ring and the tensor core ahead of the epilogue by the TMEM
 // groups, and no slot waits for a role that does not read it.
 // Warp roles: epilogue warps (TMEM lane quarter x column chunk); four producer warps (one
-// weight row per thread: nibbles -> bytes in the MMA's K-major core-matrix layout); one
+// weight row per thread: nibbles -> bytes, stored to the row's TMEM lane); one
 // MMA warp (also allocates TMEM); one copy warp for the raw code boxes; one copy warp for
 // the token codes, scales and d_x (the only role that waits on the preceding grid). Every
 // wait is bounded; on a timeout all roles stop, copies and MMAs are drained and TMEM is
@@ -54,12 +57,14 @@ __host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
            | (1u << 7) | (1u << 10)           // A, B format s8
            | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
-__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+// D (TMEM) += A (TMEM: row i in lane i, K along the columns, 4 bytes per column) x B
+// (shared memory, K-major), one MMA of M = 128, N = MN, K = 32.
+__device__ __forceinline__ void tc_mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.eq.b32 p, 0, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc)
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc)
         : "memory");
 }
 
@@ -71,16 +76,14 @@ template <int MN>
 struct Geo {
     static constexpr int TT = MN;                 // tokens per tile
     static constexpr int NW = 128;                // weight rows per tile
-    static constexpr int W_BLK = NW * 32;         // expanded weights of one block
     static constexpr int T_BLK = TT * 32;
     static constexpr int DX_BLK = TT * 4;
     static constexpr int S = 8;                   // quant blocks per stage (one code box)
     static constexpr int RAW_BYTES = NW * 128;    // one code box, 1024-aligned slots
-    // operand slot: expanded weights (1024-aligned), token codes
-    static constexpr int OFF_W = 0;
-    static constexpr int OFF_T = OFF_W + S * W_BLK;
-    static constexpr int OP_BYTES = tc::align_up(OFF_T + S * T_BLK, 1024);
-    static constexpr int NO = 3;                  // operand slots
+    // operand slot: the stage's token codes in shared memory (1024-aligned) and its
+    // expanded weights in tensor memory (8 columns per block)
+    static constexpr int OP_BYTES = tc::align_up(S * T_BLK, 1024);
+    static constexpr int NO = 4;                  // operand slots
     // epilogue slot: the stage's weight scales (NW rows x S fp16), then d_x (S x TT f32)
     static constexpr int SC_BYTES = NW * S * 2;
     static constexpr int ES_BYTES = SC_BYTES + S * DX_BLK;
@@ -90,14 +93,22 @@ struct Geo {
     static constexpr int OFF_DX = OFF_OPS + NO * OP_BYTES;
     static constexpr int OFF_CTRL = tc::align_up(OFF_DX + ND * ES_BYTES, 1024);
     static constexpr int SMEM_BYTES = OFF_CTRL + 1024 + 1024;
-    static constexpr int NBUF = 512 / MN;                  // TMEM accumulator tiles (one per block)
+    // TMEM: accumulators in columns [0, 256), operand slots' weights in [256, 256 + NO * 64)
+    static constexpr int ACC_COLS = 256;
+    static constexpr int A_COL0 = ACC_COLS;
+    static constexpr int A_SLOT_COLS = S * 8;
+    static constexpr int NBUF = ACC_COLS / MN;             // TMEM accumulator tiles (one per block)
     static constexpr int GS = tc::cmin(S, NBUF / 2);       // blocks per TMEM group (at least two groups)
     static constexpr int NG = tc::cmin(8, NBUF / GS);      // TMEM groups, used in turn
     static constexpr int HALVES = S / GS;                  // TMEM groups per stage
-    static constexpr int TMEM_COLS = NG * GS * MN;
-    static constexpr int CW = MN / 2;                      // columns per epilogue warp (8 warps)
+    static constexpr int TMEM_COLS = 512;
+    // columns per epilogue warp: 8 warps at 16 tokens, 16 warps above (more warps per SM
+    // sub-partition to cover the tensor-memory load latency)
+    static constexpr int CW = MN == 64 ? 16 : 8;
     static constexpr int EPI_WARPS = 4 * MN / CW;
-    static constexpr int PROD_WARPS = NW / 32;
+    // two producer warps per TMEM lane quarter, each expanding half of the stage's blocks
+    static constexpr int PROD_WARPS = 2 * NW / 32;
+    static constexpr int PROD_BLKS = S / 2;
     static constexpr int PROD_WARP0 = EPI_WARPS;
     static constexpr int MMA_WARP = PROD_WARP0 + PROD_WARPS;
     static constexpr int COPY_WARP = MMA_WARP + 1;
@@ -105,11 +116,12 @@ struct Geo {
     static constexpr int NUM_THREADS = (OPC_WARP + 1) * 32;
     static constexpr uint32_t IDESC = idesc_i8_s32(128, MN);
     static_assert(MN == 16 || MN == 32 || MN == 64, "MMA N");
-    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation");
+    static_assert(NG * GS * MN <= ACC_COLS && A_COL0 + NO * A_SLOT_COLS <= TMEM_COLS, "TMEM allocation");
     static_assert(NR >= 2, "raw ring depth");
+    static_assert(PROD_BLKS == 4, "a producer warp stores 32 TMEM columns per stage");
     static_assert(NG >= 2 && S % GS == 0, "TMEM groups");
     static_assert(SMEM_BYTES <= tc::SMEM_LIMIT, "shared memory");
-    static_assert(OFF_T % 128 == 0 && OFF_DX % 16 == 0 && OP_BYTES % 1024 == 0, "operand alignment");
+    static_assert(OFF_DX % 16 == 0 && OP_BYTES % 1024 == 0, "operand alignment");
     static_assert(NO <= 4 && ND <= 8, "control block");
 };
 
@@ -188,6 +200,17 @@ __device__ __forceinline__ void tmem_preset(uint32_t taddr) {
 #undef W4A8_M8
 #undef W4A8_M4
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Stores 32 words into 32 TMEM columns of this warp's lane quarter.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
 
 // Q4_0 only. Launch: grid (ceil(N / 128), token tiles, splits of K), Geo<MN>::NUM_THREADS
 // threads, Geo<MN>::SMEM_BYTES of dynamic shared memory; K a multiple of 256 and splits of
@@ -203,8 +226,8 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
     using Gm = Geo<MN>;
     constexpr int S = Gm::S, NR = Gm::NR, NO = Gm::NO, ND = Gm::ND, NG = Gm::NG, GS = Gm::GS, HALVES = Gm::HALVES;
     constexpr int TT = Gm::TT, NW = Gm::NW, CW = Gm::CW;
-    constexpr int W_BLK = Gm::W_BLK, T_BLK = Gm::T_BLK, DX_BLK = Gm::DX_BLK;
-    constexpr int OFF_W = Gm::OFF_W, OFF_T = Gm::OFF_T, OFF_DX = Gm::OFF_DX;
+    constexpr int T_BLK = Gm::T_BLK, DX_BLK = Gm::DX_BLK;
+    constexpr int OFF_DX = Gm::OFF_DX;
     constexpr int RAW_BYTES = Gm::RAW_BYTES, OP_BYTES = Gm::OP_BYTES, OFF_OPS = Gm::OFF_OPS;
     constexpr int EPI_WARPS = Gm::EPI_WARPS, PROD_WARP0 = Gm::PROD_WARP0;
     constexpr int MMA_WARP = Gm::MMA_WARP, COPY_WARP = Gm::COPY_WARP, OPC_WARP = Gm::OPC_WARP;
@@ -265,35 +288,43 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
 
     if (warp >= PROD_WARP0 && warp < MMA_WARP) {
         // ------------------------------------------------------------ producer
-        const int p = threadIdx.x - PROD_WARP0 * 32;  // weight row within the tile
+        // Weight row p of the tile is TMEM lane p: producer warp i writes lanes of quarter
+        // i % 4 (the rows 32 (i % 4) .. + 31) for blocks 4 (i / 4) .. + 3 of each stage.
+        static_assert(PROD_WARP0 % 4 == 0, "producer warp i must own TMEM lane quarter i % 4");
+        const int pw = warp - PROD_WARP0;
+        const int p = (pw & 3) * 32 + lane;
+        const int kq = (pw >> 2) * Gm::PROD_BLKS;
+        const uint32_t a_lane = tmem_base + (uint32_t(warp & 3) << 21) + uint32_t(Gm::A_COL0 + kq * 8);
         for (int st = 0; st < nstages; ++st) {
             const int rs = st % NR, os = st % NO;
-            if (!bounded_wait_warp(bar(&ctrl->op_empty[os]), ((st / NO) & 1) ^ 1, abort)) break;
-            if (!bounded_wait_warp(bar(&ctrl->raw_full[rs]), (st / NR) & 1, abort)) break;
+            // the slot's previous MMAs are complete and the stage's code box has landed
+            if (!bounded_wait2_warp(bar(&ctrl->op_empty[os]), ((st / NO) & 1) ^ 1, bar(&ctrl->raw_full[rs]),
+                                    (st / NR) & 1, abort))
+                break;
+            tc_fence_after();
             const uint8_t* rp = raw_ptr(rs);
-            uint8_t* op = op_ptr(os);
-            // All eight 16-byte chunks of row p of the swizzled box first (independent loads
-            // in flight together), then the expansion and stores.
-            uint4 wv[S];
+            // This warp's four 16-byte chunks of row p of the swizzled box first (independent
+            // loads in flight together), then the expansion and one TMEM store.
+            uint4 wv[Gm::PROD_BLKS];
 #pragma unroll
-            for (int k = 0; k < S; ++k) wv[k] = *reinterpret_cast<const uint4*>(rp + p * 128 + ((k ^ (p & 7)) << 4));
+            for (int k = 0; k < Gm::PROD_BLKS; ++k)
+                wv[k] = *reinterpret_cast<const uint4*>(rp + p * 128 + (((kq + k) ^ (p & 7)) << 4));
+            uint32_t v[32];
 #pragma unroll
-            for (int k = 0; k < S; ++k) {
+            for (int k = 0; k < Gm::PROD_BLKS; ++k) {
                 const uint32_t w[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
-                uint32_t lo[4], hi[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    lo[c] = ((w[c] << 4) & 0xF0F0F0F0u) ^ 0x80808080u;  // 16 * (q - 8), elements 4c..4c+3
-                    hi[c] = (w[c] & 0xF0F0F0F0u) ^ 0x80808080u;         // elements 16+4c..16+4c+3
+                    v[8 * k + c] = ((w[c] << 4) & 0xF0F0F0F0u) ^ 0x80808080u;  // 16 * (q - 8), elements 4c..4c+3
+                    v[8 * k + 4 + c] = (w[c] & 0xF0F0F0F0u) ^ 0x80808080u;     // elements 16+4c..16+4c+3
                 }
-                uint8_t* dst = op + OFF_W + k * W_BLK + (p >> 3) * SBO + (p & 7) * 16;
-                *reinterpret_cast<uint4*>(dst) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                *reinterpret_cast<uint4*>(dst + LBO) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             }
-            // The box was read (the stores above consumed every load): hand it back. The
-            // expanded rows are made visible to the tensor core (each lane's proxy fence,
-            // then one arrival for the warp).
-            fence_proxy_async_smem();
+            // block kq + k: elements 0..31 in columns 8 (kq + k) .. + 7 of the slot
+            tmem_st32(a_lane + uint32_t(os * Gm::A_SLOT_COLS), v);
+            // The box was read (the store above consumed every load): hand it back. The
+            // expanded rows are complete in TMEM before the warp's one arrival.
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(&ctrl->raw_empty[rs]));
@@ -331,7 +362,7 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
             if (leader) {
                 const uint32_t fb = bar(&ctrl->op_full[os]);
                 mbar_arrive_expect_tx(fb, uint32_t(S * T_BLK));
-                bulk_g2s(smem_addr(op_ptr(os) + OFF_T),
+                bulk_g2s(smem_addr(op_ptr(os)),
                          reinterpret_cast<const uint8_t*>(tok) + (int64_t(t) * B + b0) * T_BLK, uint32_t(S * T_BLK), fb);
             }
             issued_op = st + 1;
@@ -374,10 +405,10 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < GS; ++kk) {
                         const int k = hf * GS + kk;
-                        const uint32_t w_addr = smem0 + uint32_t(OFF_OPS + os * OP_BYTES + OFF_W + k * W_BLK);
-                        const uint32_t t_addr = smem0 + uint32_t(OFF_OPS + os * OP_BYTES + OFF_T + k * T_BLK);
-                        tc_mma_i8(tmem_base + uint32_t((g * GS + kk) * MN), smem_desc_kmajor(w_addr, LBO, SBO),
-                                  smem_desc_kmajor(t_addr, LBO, SBO), Gm::IDESC);
+                        const uint32_t a_col = uint32_t(Gm::A_COL0 + os * Gm::A_SLOT_COLS + k * 8);
+                        const uint32_t t_addr = smem0 + uint32_t(OFF_OPS + os * OP_BYTES + k * T_BLK);
+                        tc_mma_i8_ta(tmem_base + uint32_t((g * GS + kk) * MN), tmem_base + a_col,
+                                     smem_desc_kmajor(t_addr, LBO, SBO), Gm::IDESC);
                     }
                     tc_commit(bar(&ctrl->tfull[g]));  // the group's accumulators are complete
                     if (hf == HALVES - 1) tc_commit(bar(&ctrl->op_empty[os]));  // the stage's operands are read
@@ -430,25 +461,30 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
                     // d_w / 16 (exact) of block k of the stage
                     const float ws = 0.0625f * __half2float(__ushort_as_half(
                                                    uint16_t((k & 1) ? (scw[k >> 1] >> 16) : (scw[k >> 1] & 0xFFFFu))));
-                    uint32_t pr[CW];
                     const uint32_t ta = lane_base + uint32_t((g * GS + kk) * MN + c0);
-                    tmem_cols(ta, pr);
+                    const float* dxk = reinterpret_cast<const float*>(dp + Gm::SC_BYTES + k * DX_BLK) + c0;
+                    const float ncw = -kMagic * ws;  // exact
+                    const unsigned long long ws2 = pack2(ws, ws), nc2 = pack2(ncw, ncw);
+                    // the tile's columns in chunks of at most 16 (register pressure)
+                    constexpr int CH = CW < 16 ? CW : 16;
+#pragma unroll
+                    for (int c = 0; c < CW; c += CH) {
+                        uint32_t pr[CH];
+                        tmem_cols(ta + uint32_t(c), pr);
+#pragma unroll
+                        for (int j = 0; j < CH; j += 4) {
+                            const float4 dv = *reinterpret_cast<const float4*>(dxk + c + j);  // broadcast
+                            // acc += round(D16 * ws) * d_x
+                            fma2_magic(acc2[(c + j) / 2], pr[j], pr[j + 1], dv.x, dv.y, ws2, nc2);
+                            fma2_magic(acc2[(c + j) / 2 + 1], pr[j + 2], pr[j + 3], dv.z, dv.w, ws2, nc2);
+                        }
+                    }
                     tmem_preset<CW>(ta);  // for the tile's next use
-                    if (kk == GS - 1) {  // the group's tiles are all in registers and preset: free it
+                    if (kk == GS - 1) {  // the group's tiles are all read and preset: free it
                         tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(&ctrl->tempty[g]));
-                    }
-                    const float* dxk = reinterpret_cast<const float*>(dp + Gm::SC_BYTES + k * DX_BLK) + c0;
-                    const float ncw = -kMagic * ws;  // exact
-                    const unsigned long long ws2 = pack2(ws, ws), nc2 = pack2(ncw, ncw);
-#pragma unroll
-                    for (int j = 0; j < CW; j += 4) {
-                        const float4 dv = *reinterpret_cast<const float4*>(dxk + j);  // broadcast
-                        // acc += round(D16 * ws) * d_x
-                        fma2_magic(acc2[j / 2], pr[j], pr[j + 1], dv.x, dv.y, ws2, nc2);
-                        fma2_magic(acc2[j / 2 + 1], pr[j + 2], pr[j + 3], dv.z, dv.w, ws2, nc2);
                     }
                     dep = fmaf(dxk[0], ws, dep);  // depends on this block's scale and d_x loads
                 }
