@@ -23,7 +23,8 @@ namespace {
 
 using namespace w4a8;
 
-// Largest M served by the dp4a GEMV when the path is AUTO.
+// Largest M served by the dp4a GEMV when the path is AUTO and there is no int8
+// tensor-core kernel for the shape (affine codes, K not a multiple of 256).
 constexpr int kGemvMaxM = 8;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -645,20 +646,21 @@ w4a8_status run_gemm_tc(int M, int N, int K, int group, const TcWs& w, const uin
     }
 }
 
-inline bool use_gemv(int M, w4a8_path path);
+inline bool use_gemv(int M, int N, int K, int group, w4a8_path path);
 
 // Smallest workspace a call of this shape accepts on `path`: the GEMV's activation, or the
 // tensor-core operand plus the partial outputs of the split of K that bounds the
 // accumulation chain (K > 4096); a larger one, up to w4a8_workspace_bytes, lets the
 // tensor-core path split K further to fill the SMs.
-size_t min_workspace_bytes(int M, int N, int K, int group, w4a8_path path) {
-    if (use_gemv(M, path)) return gemv_ws(nullptr, M, K).bytes;
+// `split`: a call of the prepare / contract pair (the path rule without N).
+size_t min_workspace_bytes(int M, int N, int K, int group, w4a8_path path, bool split = false) {
+    if (use_gemv(M, split ? -1 : N, K, group, path)) return gemv_ws(nullptr, M, K).bytes;
     return tc_ws(nullptr, M, K, group).bytes + partial_bytes(tc_split_min(K), M, N);
 }
 
 w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, const void* wq, const void* ws,
                             const void* wb, bool affine, int group, const void* y, const void* work,
-                            size_t work_bytes, w4a8_path path) {
+                            size_t work_bytes, w4a8_path path, bool split = false) {
     if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 32) != 0) return W4A8_ERR_INVALID_ARG;
     if (!x || !wq || !ws || !y || (affine && !wb)) return W4A8_ERR_INVALID_ARG;
     if (dt != W4A8_F32 && dt != W4A8_BF16) return W4A8_ERR_UNSUPPORTED;
@@ -671,7 +673,7 @@ w4a8_status check_gemm_args(int M, int N, int K, const void* x, w4a8_dtype dt, c
         return W4A8_ERR_MISALIGNED;
     if (!work) return W4A8_ERR_WORKSPACE;
     if (!aligned16(work)) return W4A8_ERR_MISALIGNED;
-    if (work_bytes < min_workspace_bytes(M, N, K, affine ? group : 0, path)) return W4A8_ERR_WORKSPACE;
+    if (work_bytes < min_workspace_bytes(M, N, K, affine ? group : 0, path, split)) return W4A8_ERR_WORKSPACE;
     return W4A8_OK;
 }
 
@@ -693,8 +695,17 @@ w4a8_status make_epilogue(const w4a8_epilogue* in, Epilogue* out) {
     return W4A8_OK;
 }
 
-inline bool use_gemv(int M, w4a8_path path) {
-    return (path == W4A8_PATH_GEMV) || (path == W4A8_PATH_AUTO && M <= kGemvMaxM);
+// Whether AUTO takes the GEMV. Q4_0 shapes with the int8 tensor-core kernel switch at the
+// per-call times measured on B200 (weights streamed from HBM): the tensor kernel's time is
+// nearly flat in M up to 16 tokens while the GEMV's grows with M, so it wins from M = 3 on
+// 4096 x 14336 and 14336 x 4096 (at M = 4: 15.7 vs 24.0 us) and from M = 5 on 4096 x 4096
+// and 2048 x 8192 (at M = 4 the GEMV's 8.7 us beats 10.0 us). N < 0: N is not known (the
+// prepare / contract pair), and the rule takes M and K only.
+inline bool use_gemv(int M, int N, int K, int group, w4a8_path path) {
+    if (path != W4A8_PATH_AUTO) return path == W4A8_PATH_GEMV;
+    if (!use_i8(M, K, group)) return M <= kGemvMaxM;
+    if (N < 0) return M <= 3;
+    return M <= 2 || (M <= 4 && int64_t(N) * K <= (int64_t(1) << 25));
 }
 
 // Quantise x into the workspace layout of the chosen path.
@@ -725,7 +736,7 @@ w4a8_status gemm_impl(int M, int N, int K, int group, const void* x, w4a8_dtype 
                       size_t work_bytes, w4a8_path path, cudaStream_t stream) {
     w4a8_status st = check_gemm_args(M, N, K, x, dt, wq, ws, wb, FMT == 1, group, y, work, work_bytes, path);
     if (st != W4A8_OK) return st;
-    const bool gemv = use_gemv(M, path);
+    const bool gemv = use_gemv(M, N, K, FMT == 1 ? group : 0, path);
     if (gemv && gemv_fused(M, K)) return run_gemv_fused<FMT>(M, N, K, group, x, dt, wq, ws, wb, y, epi, stream);
     st = prepare_impl(M, K, FMT == 1 ? group : 0, x, dt, work, gemv, stream);
     if (st != W4A8_OK) return st;
@@ -969,9 +980,9 @@ w4a8_status w4a8_prepare_act(int M, int K, int group, const void* x, w4a8_dtype 
     const bool affine = group != 0;
     // the weight pointers are not used here; pass x so their null / alignment checks pass
     w4a8_status st = check_gemm_args(M, 1, K, x, dtype, x, x, x, affine, group, static_cast<const float*>(x), ws,
-                                     ws_bytes, path);
+                                     ws_bytes, path, true);
     if (st != W4A8_OK) return st;
-    return prepare_impl(M, K, group, x, dtype, ws, use_gemv(M, path), stream);
+    return prepare_impl(M, K, group, x, dtype, ws, use_gemv(M, -1, K, group, path), stream);
 }
 
 w4a8_status w4a8_gemm_epi(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
@@ -995,10 +1006,11 @@ w4a8_status w4a8_gemm_affine_epi(int M, int N, int K, int group, const void* x, 
 
 w4a8_status w4a8_gemm_prepared(int M, int N, int K, const uint8_t* qs, const uint16_t* d_fp16, float* y,
                                const void* ws, size_t ws_bytes, w4a8_path path, cudaStream_t stream) {
-    w4a8_status st = check_gemm_args(M, N, K, qs, W4A8_F32, qs, d_fp16, nullptr, false, 0, y, ws, ws_bytes, path);
+    w4a8_status st =
+        check_gemm_args(M, N, K, qs, W4A8_F32, qs, d_fp16, nullptr, false, 0, y, ws, ws_bytes, path, true);
     if (st != W4A8_OK) return st;
-    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, kPlain, const_cast<void*>(ws), ws_bytes, use_gemv(M, path),
-                            false, stream);
+    return contract_impl<0>(M, N, K, 0, qs, d_fp16, nullptr, y, kPlain, const_cast<void*>(ws), ws_bytes,
+                            use_gemv(M, -1, K, 0, path), false, stream);
 }
 
 w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint32_t* q, const uint16_t* scale_bf16,
@@ -1006,10 +1018,10 @@ w4a8_status w4a8_gemm_affine_prepared(int M, int N, int K, int group, const uint
                                       w4a8_path path, cudaStream_t stream) {
     const uint8_t* wq = reinterpret_cast<const uint8_t*>(q);
     w4a8_status st =
-        check_gemm_args(M, N, K, wq, W4A8_F32, wq, scale_bf16, bias_bf16, true, group, y, ws, ws_bytes, path);
+        check_gemm_args(M, N, K, wq, W4A8_F32, wq, scale_bf16, bias_bf16, true, group, y, ws, ws_bytes, path, true);
     if (st != W4A8_OK) return st;
     return contract_impl<1>(M, N, K, group, wq, scale_bf16, bias_bf16, y, kPlain, const_cast<void*>(ws), ws_bytes,
-                            use_gemv(M, path), false, stream);
+                            use_gemv(M, -1, K, group, path), false, stream);
 }
 
 // Scratch of w4a8_gemm_noalloc. In host code this name is only a stand-in for the

@@ -115,11 +115,14 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group);
  *            K, 0) bytes (or at least the path's minimum, see there), owned by the
  *            caller; contents on entry are ignored and are garbage afterwards. Calls
  *            that share a workspace must be ordered on one stream.
- * Scale range: the tensor-core path (M > 8, or PATH_GEMM) holds d_w * (q - 8) exactly as
- * two fp16 values formed by one fused multiply-add each, which requires |d_w| < 2728
- * (weights of magnitude up to ~21800). A larger, infinite or NaN scale makes the kernel
- * set W4A8_ERR_RANGE in the device status word (w4a8_last_device_error) and the affected
- * outputs are not reliable. The GEMV path (M <= 8, or PATH_GEMV) has no such limit.
+ * Paths (AUTO): the dp4a GEMV for M <= 2, for M <= 4 when N * K <= 2^25, and for
+ * M <= 8 when K is not a multiple of 256; otherwise tensor cores: int8 MMAs on the
+ * original codes for M <= 64 (K a multiple of 256), fp16 MMAs on CTA pairs above.
+ * Scale range: the fp16 tensor-core kernels hold d_w * (q - 8) exactly as two fp16 values
+ * formed by one fused multiply-add each, which requires |d_w| < 2728 (weights of magnitude
+ * up to ~21800). A larger, infinite or NaN scale makes the kernel set W4A8_ERR_RANGE in
+ * the device status word (w4a8_last_device_error) and the affected outputs are not
+ * reliable. The GEMV and the int8 kernel have no such limit.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, WORKSPACE, CUDA.
  */
 w4a8_status w4a8_gemm(int M, int N, int K, const void* x, w4a8_dtype dtype,
@@ -204,8 +207,9 @@ w4a8_status w4a8_gemm_affine_epi(int M, int N, int K, int group, const void* x, 
  * once and the per-call re-quantisation the tract page identifies as per-op overhead
  * ("W4A8MatMul op" measurements) is paid once.
  *  w4a8_prepare_act   quantises x (M x K) into `ws` in the layout of the path that a
- *                     matmul of this M takes (`path` AUTO resolves by M exactly as
- *                     w4a8_gemm does; group = 0 for Q4_0 weights, else 32, 64 or 128).
+ *                     matmul of this M takes (`path` AUTO resolves without N: the GEMV
+ *                     for M <= 3 where w4a8_gemm would take the int8 tensor kernel,
+ *                     else for M <= 8; group = 0 for Q4_0 weights, else 32, 64 or 128).
  *  w4a8_gemm_prepared / w4a8_gemm_affine_prepared
  *                     run only the contraction, reading the quantised activation from
  *                     `ws`. They must be given the same M, K, group and path as the
