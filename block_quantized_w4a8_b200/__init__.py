@@ -18,7 +18,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libw4a8.so")
+# W4A8_LIB=checked selects the checked variant (device-side checks, W4A8_ERR_CHECK), built
+# beside it; the default is the production library.
+LIB_PATH = os.path.join(_HERE, "libw4a8_checked.so" if os.environ.get("W4A8_LIB") == "checked" else "libw4a8.so")
 
 W4A8_OK = 0
 STATUS_NAMES = {0: "W4A8_OK", 1: "W4A8_ERR_INVALID_ARG", 2: "W4A8_ERR_UNSUPPORTED", 3: "W4A8_ERR_WORKSPACE",
@@ -32,7 +34,7 @@ EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a
            "w4a8_pack_affine_nbit", "w4a8_gemm_affine_nbit", "w4a8_gemv_q4_k", "w4a8_gemv_q4_k_backward",
            "w4a8_q4_k_backward_workspace_bytes", "w4a8_prepare_act",
            "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_gemm_noalloc", "w4a8_last_device_error",
-           "w4a8_last_cuda_error_string", "w4a8_status_string"]
+           "w4a8_last_cuda_error_string", "w4a8_status_string", "w4a8_selftest_bounded_wait"]
 
 
 class W4A8Error(RuntimeError):
@@ -75,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
         "w4a8_gemm_noalloc": (I, [I, I, I, P, I, P, P, P, P]),
         "w4a8_last_device_error": (I, []),
+        "w4a8_selftest_bounded_wait": (I, [ctypes.c_ulonglong, P, P]),
         "w4a8_status_string": (ctypes.c_char_p, [I]),
         "w4a8_last_cuda_error_string": (ctypes.c_char_p, []),
     }
@@ -294,6 +297,16 @@ def w4a8_gemm_noalloc(x, qs, d, y, stream=None) -> None:
 
 def w4a8_last_device_error() -> int:
     return int(load_library().w4a8_last_device_error())
+
+
+def w4a8_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    """Runs the library's self-test of its bounded device waits (see the header) and
+    returns the outcome bits (7 = the wait ran out, and the second warp stopped through the
+    abort flag within 100 ms)."""
+    out = ctypes.c_uint(0)
+    _check("w4a8_selftest_bounded_wait",
+           load_library().w4a8_selftest_bounded_wait(int(limit_ns), ctypes.byref(out), _stream(stream)))
+    return int(out.value)
 
 
 def w4a8_last_cuda_error_string() -> str:

@@ -38,6 +38,12 @@ __device__ __forceinline__ bool checked(bool ok) {
     return true;
 }
 
+// Checked build: the element range [off, off + len) of an operand lies within its extent
+// (the copy or access is skipped and kDevErrChecked recorded otherwise).
+__device__ __forceinline__ bool in_range(long long off, long long len, long long extent) {
+    return checked(off >= 0 && len >= 0 && off + len <= extent);
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -143,15 +149,17 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, vola
 
 // Warp-wide wait: every lane probes the barrier and a vote makes the outcome uniform
 // (phase completion is monotonic, so a lane that saw it keeps seeing it), so the warp
-// never diverges. Same limits as bounded_wait. All 32 lanes must call it.
+// never diverges. Same limits as bounded_wait (`limit_ns` other than kWaitLimitNs only in
+// the self-test of the waits). All 32 lanes must call it.
 template <bool CLUSTER = false>
-__device__ __noinline__ bool bounded_wait_warp_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+__device__ __noinline__ bool bounded_wait_warp_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                                    unsigned long long limit_ns = kWaitLimitNs) {
     const unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (__all_sync(0xffffffffu, mbar_try_wait<CLUSTER>(bar, parity))) return true;
         if ((it & 15u) == 0u) {
             uint32_t stop = *abort;
-            if (!stop && global_timer_ns() - t0 > kWaitLimitNs) stop = 2u;
+            if (!stop && global_timer_ns() - t0 > limit_ns) stop = 2u;
             stop = __shfl_sync(0xffffffffu, stop, 0);
             if (stop) {
                 if (stop == 2u && (threadIdx.x & 31u) == 0u) {
@@ -164,9 +172,37 @@ __device__ __noinline__ bool bounded_wait_warp_slow(uint32_t bar, uint32_t parit
     }
 }
 template <bool CLUSTER = false>
-__device__ __forceinline__ bool bounded_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+__device__ __forceinline__ bool bounded_wait_warp(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
     if (__all_sync(0xffffffffu, mbar_try_wait_nohint<CLUSTER>(bar, parity))) return true;
-    return bounded_wait_warp_slow<CLUSTER>(bar, parity, abort);
+    return bounded_wait_warp_slow<CLUSTER>(bar, parity, abort, limit_ns);
+}
+
+// Self-test of the bounded waits (the failure path of every pipeline): warp 0 waits with
+// limit `limit_ns` on a barrier that nothing arrives at; warp 1 waits on another such
+// barrier with the production limit and must stop through the abort flag that warp 0
+// raises when its wait runs out. Nothing else is in flight. Bits of *outcome: 1 = warp 0
+// gave up, 2 = warp 1 gave up, 4 = warp 1 stopped within 100 ms of starting. One CTA of
+// 64 threads.
+__global__ void __launch_bounds__(64, 1) selftest_wait_kernel(unsigned long long limit_ns, unsigned int* outcome) {
+    __shared__ __align__(8) unsigned long long bars[2];
+    __shared__ uint32_t abort_flag;
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bars[0]), 1);
+        mbar_init(smem_addr(&bars[1]), 1);
+        abort_flag = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+    const unsigned long long t0 = global_timer_ns();
+    const bool ok = bounded_wait_warp(smem_addr(&bars[warp]), 0, &abort_flag, warp == 0 ? limit_ns : kWaitLimitNs);
+    const unsigned long long t1 = global_timer_ns();
+    if ((threadIdx.x & 31u) == 0u) {
+        unsigned int bits = ok ? 0u : (warp == 0 ? 1u : 2u);
+        if (warp == 1 && !ok && t1 - t0 < 100000000ull) bits |= 4u;
+        atomicOr(outcome, bits);
+    }
 }
 
 // Warp-wide wait for two barriers: both probed at once on the fast path (one round trip

@@ -359,7 +359,9 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
             const int os = st % NO, ds = st % ND;
             const int b0 = kb0 + st * S;
             if (!bounded_wait_warp(bar(&ctrl->op_empty[os]), ((st / NO) & 1) ^ 1, abort)) break;
-            if (leader) {
+            // (checked build: the stage's token codes and d_x lie within the operands of
+            // gridDim.y token tiles)
+            if (leader && in_range((int64_t(t) * B + b0) * T_BLK, S * T_BLK, int64_t(gridDim.y) * B * T_BLK)) {
                 const uint32_t fb = bar(&ctrl->op_full[os]);
                 mbar_arrive_expect_tx(fb, uint32_t(S * T_BLK));
                 bulk_g2s(smem_addr(op_ptr(os)),
@@ -367,7 +369,7 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
             }
             issued_op = st + 1;
             if (!bounded_wait_warp(bar(&ctrl->dx_empty[ds]), ((st / ND) & 1) ^ 1, abort)) break;
-            if (leader) {
+            if (leader && in_range((int64_t(t) * B + b0) * TT, S * TT, int64_t(gridDim.y) * B * TT)) {
                 const uint32_t db = bar(&ctrl->dx_full[ds]);
                 mbar_arrive_expect_tx(db, uint32_t(Gm::ES_BYTES));
                 tma_load_2d<2>(smem_addr(es_ptr(ds)), &tm_s, b0, n0, db);

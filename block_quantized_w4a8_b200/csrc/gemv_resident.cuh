@@ -303,7 +303,8 @@ __global__ void __launch_bounds__(WARPS * 32, 2)
         mbar_init_fence();
         const uint64_t pol = l2_evict_first_policy();
         mbar_arrive_expect_tx(bar, uint32_t(resident_weight_bytes(RC, K, E, FMT == 1)));
-        bulk_g2s_hint(wbase, wq + n0 * codes_row, uint32_t(RC * codes_row), bar, pol);
+        // (checked build: this CTA's rows lie within the N rows of the weights)
+        if (in_range(n0, RC, N)) bulk_g2s_hint(wbase, wq + n0 * codes_row, uint32_t(RC * codes_row), bar, pol);
         bulk_g2s_hint(sbase, reinterpret_cast<const uint8_t*>(wscale) + n0 * E * 2, uint32_t(RC * E * 2), bar, pol);
         if (FMT == 1)
             bulk_g2s_hint(bbase, reinterpret_cast<const uint8_t*>(wbias) + n0 * E * 2, uint32_t(RC * E * 2), bar, pol);

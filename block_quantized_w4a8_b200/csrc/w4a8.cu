@@ -1103,6 +1103,26 @@ w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dty
                         W4A8_PATH_AUTO, stream);
 }
 
+// Outcome word of w4a8_selftest_bounded_wait.
+static __device__ unsigned int g_selftest_outcome;
+
+w4a8_status w4a8_selftest_bounded_wait(unsigned long long limit_ns, unsigned int* outcome, cudaStream_t stream) {
+    if (!outcome || limit_ns < 1000ull || limit_ns > 1000000000ull) return W4A8_ERR_INVALID_ARG;
+    const unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_selftest_outcome, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    unsigned int* dev_outcome = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&dev_outcome), g_selftest_outcome);
+    if (e != cudaSuccess) return cuda_status(e);
+    w4a8::selftest_wait_kernel<<<1, 64, 0, stream>>>(limit_ns, dev_outcome);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e);
+    e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = cudaMemcpyFromSymbol(outcome, g_selftest_outcome, sizeof(*outcome));
+    return cuda_status(e);
+}
+
 w4a8_status w4a8_last_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return W4A8_ERR_CUDA;
     unsigned int v = 0;

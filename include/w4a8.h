@@ -324,6 +324,20 @@ w4a8_status w4a8_gemm_noalloc(int M, int N, int K, const void* x, w4a8_dtype dty
  */
 w4a8_status w4a8_last_device_error(void);
 
+/*
+ * Self-test of the failure path (not an operation of the method): runs one test kernel
+ * on `stream` in which a warp waits, through the library's own bounded-wait code, on an
+ * mbarrier that nothing arrives at, with a limit of `limit_ns` (1 us .. 1 s), while a
+ * second warp waits on another such barrier with the production limit and must stop
+ * through the abort flag that the first raises. No copy or MMA is in flight. Synchronises
+ * `stream`, then writes to the host word *outcome: bit 0 = the first wait ran out, bit 1 =
+ * the second wait stopped, bit 2 = it stopped within 100 ms (7 = all as designed). The
+ * kernel records W4A8_ERR_DEVICE_TIMEOUT in the device status word, as a real timeout
+ * does; the context stays usable.
+ * Errors: INVALID_ARG (outcome NULL, limit out of range), CUDA.
+ */
+w4a8_status w4a8_selftest_bounded_wait(unsigned long long limit_ns, unsigned int* outcome, cudaStream_t stream);
+
 /* Description of the CUDA error behind the last W4A8_ERR_CUDA returned to this thread
  * ("no error" if there was none). Static string, never NULL. */
 const char* w4a8_last_cuda_error_string(void);

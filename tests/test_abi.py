@@ -183,5 +183,15 @@ def test_checked_build_exports_the_same_boundary():
     assert chk.w4a8_status_string(8) == b"W4A8_ERR_CHECK"
 
 
+def test_selftest_hook_argument_errors(lib):
+    """The failure-path self-test rejects its arguments before touching the device."""
+    P = ctypes.c_void_p
+    out = ctypes.c_uint(0)
+    f = lib.w4a8_selftest_bounded_wait
+    assert f(ctypes.c_ulonglong(100000), None, P(0)) == 1          # outcome NULL
+    assert f(ctypes.c_ulonglong(0), ctypes.byref(out), P(0)) == 1  # limit below 1 us
+    assert f(ctypes.c_ulonglong(2 * 10 ** 9), ctypes.byref(out), P(0)) == 1  # above 1 s
+
+
 def test_status_string_of_check(lib):
     assert w4a8.w4a8_status_string(8) == "W4A8_ERR_CHECK"

@@ -256,6 +256,24 @@ def test_full_size_sampled(wl):
     check_tol(y[ms, ns], yref, T, wl.name)
 
 
+# Every K x N of the MLP sweep at M = 1, 8, 64 and 1024 (GEMV, int8 tensor kernel at 8
+# and 64 tokens, CTA pairs at 1024), through AUTO, on sampled outputs.
+SWEEP_FULL = [inputs.Workload(f"sweep_m{M}_k{K}_n{N}", M=M, K=K, N=N)
+              for K, N in inputs.SWEEP_SHAPES for M in (1, 8, 64, 1024)]
+
+
+@pytest.mark.parametrize("wl", SWEEP_FULL, ids=lambda w: w.name)
+def test_sweep_full_size_sampled(wl):
+    x, w = inputs.make(wl)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    y = as_np(w4a8.gemm(dev(x), qs, d))
+    rqx, rdx, _ = oracle.quant_act_q8_0(x.float().numpy())
+    rqs, rd = oracle.pack_q4_0(w.numpy())
+    ms, ns = inputs.sample_indices(wl.M, wl.N, 1000, seed=wl.M + wl.K)
+    yref, T = oracle.gemm_q4_0_sampled(rqx, rdx, rqs, rd, ms, ns)
+    check_tol(y[ms, ns], yref, T, wl.name)
+
+
 # ------------------------------------------------------------------ affine
 AFFINE_SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (20, 128, 640), (32, 256, 1024), (64, 1536, 384),
                  (200, 333, 1280), (130, 128, 4096), (300, 333, 1024), (200, 512, 4096)]
