@@ -27,6 +27,9 @@ using namespace w4a8;
 // tensor-core kernel for the shape (affine codes, K not a multiple of 256).
 constexpr int kGemvMaxM = 8;
 
+// Shared memory of one SM on sm_100 (228 KB; one CTA may use up to 227 KB).
+constexpr int kSmemPerSm = 233472;
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -803,19 +806,67 @@ w4a8_status pack_affine_impl(const void* w, w4a8_dtype dtype, int N, int K, int 
 // Row ranges of the backward: enough CTAs (super-block columns x ranges) for four per
 // SM, at least 32 rows per range, at most 2048 (a lane's f32 chain of products is then at
 // most 64 long).
-inline int q4k_row_ranges(int N, int K) {
+// Row ranges of the streamed Q4_K backward: with the K/256 super-block columns, about one
+// CTA per SM (at least 16 rows per range), more ranges when a range would exceed
+// kBwdMaxRows rows (the bound on a lane's chain of sums).
+inline int q4k_bwd_ranges(int N, int K) {
     const int nb = K / 256;
-    int64_t R = cdiv(4 * int64_t(sm_count()), nb);
-    const int64_t rmax = cdiv(N, 32);
+    int64_t R = cdiv(sm_count(), nb);
+    const int64_t rmax = cdiv(N, 16);
     if (R > rmax) R = rmax;
-    if (R < cdiv(N, 2048)) R = cdiv(N, 2048);
-    if (R < 1) R = 1;
-    const int rows = int(cdiv(N, R));
-    return int(cdiv(N, rows));
+    const int64_t rmin = cdiv(N, q4k::kBwdMaxRows);
+    if (R < rmin) R = rmin;
+    return int(R < 1 ? 1 : R);
 }
 inline size_t q4k_bwd_bytes(int M, int N, int K) {
-    const int R = q4k_row_ranges(N, K);
+    const int R = q4k_bwd_ranges(N, K);
     return R > 1 ? size_t(R) * (M < 2 ? M : 2) * K * 4 : 0;
+}
+template <int MT>
+w4a8_status launch_q4k_bwd(int N, int K, const float* dy, const uint8_t* w, float* out, int R, cudaStream_t stream) {
+    constexpr size_t smem = q4k::bwd_smem_bytes(MT);
+    static bool configured[64] = {false};
+    int dev = 0;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return cuda_status(ed);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        const cudaError_t ea = cudaFuncSetAttribute(q4k::bwd_stream_kernel<MT>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (ea != cudaSuccess) return cuda_status(ea);
+        configured[dev] = true;
+    }
+    // the weights as 8-byte elements [N][K/256 * 18], one box = one super-block column of 64 rows
+    CUtensorMap tm;
+    const uint64_t cols = uint64_t(K / 256) * (q4k::kBlockBytes / 8);
+    if (!encode_2d(&tm, w, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, cols, uint64_t(N), cols * 8, q4k::kBlockBytes / 8,
+                   q4k::kBwdSlotRows))
+        return W4A8_ERR_CUDA;
+    return cuda_status(launch_pdl(q4k::bwd_stream_kernel<MT>, dim3(unsigned((K / 256) * R)),
+                                  dim3(q4k::kStreamThreads), smem, stream, MT, N, K, dy, tm, out, R));
+}
+
+template <int MT, int MINB>
+w4a8_status launch_q4k_stream_b(int N, int K, const float* x, const uint8_t* w, float* y, const q4k::StreamPlan& sp,
+                                cudaStream_t stream) {
+    static bool configured[64] = {false};
+    int dev = 0;
+    const cudaError_t ed = cudaGetDevice(&dev);
+    if (ed != cudaSuccess) return cuda_status(ed);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        const cudaError_t ea = cudaFuncSetAttribute(q4k::fwd_stream_kernel<MT, MINB>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(tc::SMEM_LIMIT));
+        if (ea != cudaSuccess) return cuda_status(ea);
+        configured[dev] = true;
+    }
+    const int G = N < sm_count() ? N : sm_count();
+    return cuda_status(launch_pdl(q4k::fwd_stream_kernel<MT, MINB>, dim3(unsigned(G)), dim3(q4k::kStreamThreads),
+                                  sp.smem, stream, MT, N, K, x, w, y, sp.kc, sp.nst));
+}
+template <int MT>
+w4a8_status launch_q4k_stream(int N, int K, const float* x, const uint8_t* w, float* y, const q4k::StreamPlan& sp,
+                              cudaStream_t stream) {
+    return sp.two_per_sm ? launch_q4k_stream_b<MT, 2>(N, K, x, w, y, sp, stream)
+                         : launch_q4k_stream_b<MT, 1>(N, K, x, w, y, sp, stream);
 }
 w4a8_status check_q4k(int M, int N, int K, const void* a, const void* w, const void* out) {
     if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 256) != 0 || !a || !w || !out) return W4A8_ERR_INVALID_ARG;
@@ -834,6 +885,17 @@ w4a8_status w4a8_gemv_q4_k(int M, int N, int K, const float* x, const uint8_t* w
     const dim3 grid(unsigned(cdiv(N, 16)));  // 16 rows per CTA
     for (int m0 = 0; m0 < M; m0 += 2) {
         const int mt = (M - m0 < 2) ? (M - m0) : 2;
+        // The streamed kernel where x of the launch's tokens fits in shared memory beside
+        // the weight ring; the 16-rows-per-CTA kernel otherwise.
+        const q4k::StreamPlan sp = q4k::stream_plan(mt, K, size_t(tc::SMEM_LIMIT), size_t(kSmemPerSm));
+        if (sp.ok) {
+            const w4a8_status ls = mt == 1 ? launch_q4k_stream<1>(N, K, x + int64_t(m0) * K, w_q4k,
+                                                                  y + int64_t(m0) * N, sp, stream)
+                                           : launch_q4k_stream<2>(N, K, x + int64_t(m0) * K, w_q4k,
+                                                                  y + int64_t(m0) * N, sp, stream);
+            if (ls != W4A8_OK) return ls;
+            continue;
+        }
         if (mt == 1)
             q4k::gemv_kernel<1><<<grid, q4k::kThreads, 0, stream>>>(1, N, K, x + int64_t(m0) * K, w_q4k,
                                                                    y + int64_t(m0) * N);
@@ -856,25 +918,20 @@ w4a8_status w4a8_gemv_q4_k_backward(int M, int N, int K, const float* dy, const 
                                     void* ws, size_t ws_bytes, cudaStream_t stream) {
     w4a8_status st = check_q4k(M, N, K, dy, w_q4k, dx);
     if (st != W4A8_OK) return st;
-    const int R = q4k_row_ranges(N, K);
+    const int R = q4k_bwd_ranges(N, K);
     const size_t need = q4k_bwd_bytes(M, N, K);
     if (need > 0) {
         if (!ws || ws_bytes < need) return W4A8_ERR_WORKSPACE;
         if (!aligned16(ws)) return W4A8_ERR_MISALIGNED;
     }
-    const int rows = int(cdiv(N, R));
     float* part = static_cast<float*>(ws);
-    const dim3 grid(unsigned(K / 256), unsigned(R));
     for (int m0 = 0; m0 < M; m0 += 2) {
         const int mt = (M - m0 < 2) ? (M - m0) : 2;
         const float* dyc = dy + int64_t(m0) * N;
         float* dxc = dx + int64_t(m0) * K;
         float* out = R > 1 ? part : dxc;
-        if (mt == 1)
-            q4k::bwd_kernel<1><<<grid, q4k::kThreads, 0, stream>>>(1, N, K, rows, dyc, w_q4k, out);
-        else
-            q4k::bwd_kernel<2><<<grid, q4k::kThreads, 0, stream>>>(2, N, K, rows, dyc, w_q4k, out);
-        st = launch_status();
+        st = mt == 1 ? launch_q4k_bwd<1>(N, K, dyc, w_q4k, out, R, stream)
+                     : launch_q4k_bwd<2>(N, K, dyc, w_q4k, out, R, stream);
         if (st != W4A8_OK) return st;
         if (R > 1) {
             const int64_t count = int64_t(mt) * K;
