@@ -705,8 +705,8 @@ def run_wide(args, torch, w4a8, oracle, inputs, steps, dev, int8_peak):
 
 def run_q4k(args, torch, w4a8, oracle, inputs, steps, dev, peaks):
     """Q4_K GEMV (y = x W^T) and its input gradient (dX = dY W) with FP32 activations at
-    decode size (M=1, K=N=4096), each checked against the oracle on sampled outputs before
-    it is timed; weight GB/s against the measured HBM copy bandwidth."""
+    decode size (M=1, K=N=4096), each checked against the oracle on all outputs before it
+    is timed; weight GB/s against the measured HBM copy bandwidth."""
     import numpy as np
     out = []
     M, N, K = 1, 4096, 4096
@@ -725,9 +725,9 @@ def run_q4k(args, torch, w4a8, oracle, inputs, steps, dev, peaks):
     torch.cuda.synchronize()
     yref, Ty = oracle.gemv_q4_k(x.numpy(), W.numpy(), N, nthreads=8)
     dxref, Tx = oracle.gemv_q4_k_backward(dy.numpy(), W.numpy(), K, nthreads=8)
-    tol = 2.0 ** -24 * (K // 8 + 32)
-    ok_f = bool(np.all(np.abs(y.cpu().numpy().astype(np.float64) - yref) <= tol * Ty))
-    ok_b = bool(np.all(np.abs(dx.cpu().numpy().astype(np.float64) - dxref) <= 2.0 ** -24 * (N // 32 + 33) * Tx))
+    # the same tolerance as every other output: 1e-5 of the sum of |terms|
+    ok_f = bool(np.all(np.abs(y.cpu().numpy().astype(np.float64) - yref) <= 1e-5 * Ty))
+    ok_b = bool(np.all(np.abs(dx.cpu().numpy().astype(np.float64) - dxref) <= 1e-5 * Tx))
     for name, ok, fn in [("q4_k_gemv_m1_4096x4096", ok_f, lambda i: w4a8.w4a8_gemv_q4_k(xd, sets[i % R], y)),
                          ("q4_k_backward_m1_4096x4096", ok_b,
                           lambda i: w4a8.w4a8_gemv_q4_k_backward(dyd, sets[i % R], dx, ws))]:
