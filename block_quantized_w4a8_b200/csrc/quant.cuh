@@ -174,6 +174,60 @@ __global__ void __launch_bounds__(256) quant_act_tc_kernel(const void* __restric
     }
 }
 
+// The same quantisation into the Q4_0 operand (FMT 0) with four lanes per block: lane c
+// loads the eight elements of its 16-byte segment (4c..4c+3 and 16+4c..16+4c+3, two
+// 16-byte loads for f32 x) and writes that segment, so no codes pass between lanes.
+// Same layout, rounding and padding as quant_act_tc_kernel<BF16, 0>.
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_act_tc4_kernel(const void* __restrict__ x, int M, int K, int tt,
+                                                            int64_t nblocks, __half* __restrict__ tok,
+                                                            float* __restrict__ dxs) {
+    pdl_launch_dependents();
+    const int B = K >> 5;
+    const int64_t blk = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 2;
+    const int c = threadIdx.x & 3;
+    const bool valid = blk < nblocks;
+    const int64_t m = valid ? blk / B : 0;
+    const int b = valid ? int(blk - m * B) : 0;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (valid && m < M) {
+        float a[4], h[4];
+        load4<BF16>(x, m * K + int64_t(b) * 32 + c * 4, a);
+        load4<BF16>(x, m * K + int64_t(b) * 32 + 16 + c * 4, h);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[i] = a[i];
+            v[4 + i] = h[i];
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const float d = __fdiv_rn(amax, 127.0f);
+    const float id = (d != 0.0f) ? __frcp_rn(d) : 0.0f;
+    int q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = max(-127, min(127, static_cast<int>(roundf(__fmul_rn(v[i], id)))));
+    if (valid) {
+        const int64_t t = m / tt;
+        const int r = int(m - t * tt);
+        const int64_t chunk = t * B + b;
+        // slot order of segment c: 4c, 4c+2, 4c+1, 4c+3, 16+4c, 16+4c+2, 16+4c+1, 16+4c+3
+        const int e[8] = {q[0], q[2], q[1], q[3], q[4], q[6], q[5], q[7]};
+        uint32_t hw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            hw[i] = uint32_t(__half_as_ushort(__int2half_rn(e[2 * i]))) |
+                    (uint32_t(__half_as_ushort(__int2half_rn(e[2 * i + 1]))) << 16);
+        char* dst = reinterpret_cast<char*>(tok) + chunk * tcgeo::tok_block_bytes(tt) + (r >> 3) * 512 + c * 128 +
+                    (r & 7) * 16;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        if (c == 0) dxs[chunk * tt + r] = d;
+    }
+}
+
 // ------------------------------------------------------------------ Q4_0 pack
 // 8 lanes per block; blocks numbered row-major, so block i is W[32i .. 32i+31] and its
 // 16 code bytes are qs[16i .. 16i+15].

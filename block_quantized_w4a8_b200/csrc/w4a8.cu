@@ -166,10 +166,11 @@ w4a8_status run_quant_tc(const void* x, w4a8_dtype dt, int M, int K, int group, 
             quant_act_tc_kernel<false, 2><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
                                                                   w.sums);
     } else if (group == 0) {
+        const dim3 grid4(unsigned(cdiv(nblocks * 4, 256)));  // four lanes per block
         if (dt == W4A8_BF16)
-            quant_act_tc_kernel<true, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0, nullptr);
+            quant_act_tc4_kernel<true><<<grid4, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs);
         else
-            quant_act_tc_kernel<false, 0><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, 0, nullptr);
+            quant_act_tc4_kernel<false><<<grid4, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs);
     } else {
         if (dt == W4A8_BF16)
             quant_act_tc_kernel<true, 1><<<grid, 256, 0, stream>>>(x, M, K, w.tt, nblocks, w.tok, w.dxs, w.z, group,
