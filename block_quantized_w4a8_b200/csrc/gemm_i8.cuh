@@ -12,10 +12,11 @@
 // bytes, no arithmetic. Byte j of a block's 16 code bytes holds element j (low nibble)
 // and element j + 16 (high nibble), so the expanded row is elements 0..31 in order.
 // Token operand: the Q8_0 codes in element order (quant_act_i8_kernel). The MMA gives
-// D16 = 16 * sum (q - 8) q_x exactly (|D16| <= 520192 < 2^22). The MMA accumulates onto
-// tensor-memory words preset to the bits of the float 1.5 * 2^23 (0x4B400000): the floats
-// in [2^23, 2^24) are the integers, so each word then is the float 1.5 * 2^23 + D16 exactly,
-// with no conversion instruction. The epilogue forms round(D16 * d_w / 16) with one FMA
+// D16 = 16 * sum (q - 8) q_x exactly (|D16| <= 520192 < 2^22). For 16 and 32 tokens the MMA
+// accumulates onto tensor-memory words preset to the bits of the float 1.5 * 2^23
+// (0x4B400000): the floats in [2^23, 2^24) are the integers, so each word then is the float
+// 1.5 * 2^23 + D16 exactly, with no conversion instruction; for 64 tokens the MMA writes
+// D16 and the epilogue adds the same bits with an integer add after the load. The epilogue forms round(D16 * d_w / 16) with one FMA
 // (F * w - 1.5 * 2^23 * w; the addend is exact, w having at most 12 significant bits) and
 // adds its product with d_x with a second: two roundings per block, and unlike the fp16
 // path no range limit on the weight scales.
@@ -57,14 +58,15 @@ __host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
            | (1u << 7) | (1u << 10)           // A, B format s8
            | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
-// D (TMEM) += A (TMEM: row i in lane i, K along the columns, 4 bytes per column) x B
-// (shared memory, K-major), one MMA of M = 128, N = MN, K = 32.
-__device__ __forceinline__ void tc_mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc) {
+// D (TMEM) = A (TMEM: row i in lane i, K along the columns, 4 bytes per column) x B
+// (shared memory, K-major) + D if `accumulate`, one MMA of M = 128, N = MN, K = 32.
+__device__ __forceinline__ void tc_mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "setp.eq.b32 p, 0, 0;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc)
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -115,6 +117,11 @@ struct Geo {
     static constexpr int OPC_WARP = COPY_WARP + 1;
     static constexpr int NUM_THREADS = (OPC_WARP + 1) * 32;
     static constexpr uint32_t IDESC = idesc_i8_s32(128, MN);
+    // How the epilogue turns a tile's int32 into the float 1.5 * 2^23 + D16: by presetting
+    // the tile to the bits of 1.5 * 2^23 for the MMA to accumulate onto (16 and 32 tokens),
+    // or by an integer add after the load (64 tokens, where the preset stores would write
+    // 256 KB of tensor memory per stage; measured 38.9 -> 34.2 us at 4096 x 14336).
+    static constexpr bool PRESET = MN <= 32;
     static_assert(MN == 16 || MN == 32 || MN == 64, "MMA N");
     static_assert(NG * GS * MN <= ACC_COLS && A_COL0 + NO * A_SLOT_COLS <= TMEM_COLS, "TMEM allocation");
     static_assert(NR >= 2, "raw ring depth");
@@ -396,8 +403,9 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
 #pragma unroll
             for (int hf = 0; hf < HALVES; ++hf, ++gi) {
                 const int g = gi % NG;
-                // (phase 0 of tempty: the epilogue's first preset of the columns)
-                if (!bounded_wait_warp(bar(&ctrl->tempty[g]), (gi / NG) & 1, abort)) {
+                // (with presets, phase 0 of tempty is the epilogue's first preset of the
+                // columns; without, the groups start free)
+                if (!bounded_wait_warp(bar(&ctrl->tempty[g]), ((gi / NG) & 1) ^ (Gm::PRESET ? 0 : 1), abort)) {
                     ok = false;
                     break;
                 }
@@ -410,7 +418,7 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
                         const uint32_t a_col = uint32_t(Gm::A_COL0 + os * Gm::A_SLOT_COLS + k * 8);
                         const uint32_t t_addr = smem0 + uint32_t(OFF_OPS + os * OP_BYTES + k * T_BLK);
                         tc_mma_i8_ta(tmem_base + uint32_t((g * GS + kk) * MN), tmem_base + a_col,
-                                     smem_desc_kmajor(t_addr, LBO, SBO), Gm::IDESC);
+                                     smem_desc_kmajor(t_addr, LBO, SBO), Gm::IDESC, Gm::PRESET ? 1u : 0u);
                     }
                     tc_commit(bar(&ctrl->tfull[g]));  // the group's accumulators are complete
                     if (hf == HALVES - 1) tc_commit(bar(&ctrl->op_empty[os]));  // the stage's operands are read
@@ -432,13 +440,15 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
 #pragma unroll
         for (int j = 0; j < CW / 2; ++j) acc2[j] = 0ull;
         const uint32_t lane_base = tmem_base + (uint32_t(q * 32) << 16);
-        // Preset every accumulator column of this warp, then release the TMEM groups.
-        for (int c = 0; c < NG * GS; ++c) tmem_preset<CW>(lane_base + uint32_t(c * MN + c0));
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-            for (int g = 0; g < NG; ++g) mbar_arrive(bar(&ctrl->tempty[g]));
+        if (Gm::PRESET) {
+            // Preset every accumulator column of this warp, then release the TMEM groups.
+            for (int c = 0; c < NG * GS; ++c) tmem_preset<CW>(lane_base + uint32_t(c * MN + c0));
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                for (int g = 0; g < NG; ++g) mbar_arrive(bar(&ctrl->tempty[g]));
+        }
         const int n = n0 + r;
         int gi = 0;
         bool ok = true;
@@ -476,14 +486,16 @@ __global__ void __launch_bounds__(Geo<MN>::NUM_THREADS, 1)
 #pragma unroll
                         for (int j = 0; j < CH; j += 4) {
                             const float4 dv = *reinterpret_cast<const float4*>(dxk + c + j);  // broadcast
-                            // acc += round(D16 * ws) * d_x
-                            fma2_magic(acc2[(c + j) / 2], pr[j], pr[j + 1], dv.x, dv.y, ws2, nc2);
-                            fma2_magic(acc2[(c + j) / 2 + 1], pr[j + 2], pr[j + 3], dv.z, dv.w, ws2, nc2);
+                            // acc += round(D16 * ws) * d_x (the words as floats 1.5 * 2^23 + D16)
+                            constexpr uint32_t add = Gm::PRESET ? 0u : kMagicBits;
+                            fma2_magic(acc2[(c + j) / 2], pr[j] + add, pr[j + 1] + add, dv.x, dv.y, ws2, nc2);
+                            fma2_magic(acc2[(c + j) / 2 + 1], pr[j + 2] + add, pr[j + 3] + add, dv.z, dv.w, ws2,
+                                       nc2);
                         }
                     }
-                    tmem_preset<CW>(ta);  // for the tile's next use
-                    if (kk == GS - 1) {  // the group's tiles are all read and preset: free it
-                        tmem_wait_st();
+                    if (Gm::PRESET) tmem_preset<CW>(ta);  // for the tile's next use
+                    if (kk == GS - 1) {  // the group's tiles are all read (and preset): free it
+                        if (Gm::PRESET) tmem_wait_st();
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(&ctrl->tempty[g]));
