@@ -257,21 +257,6 @@ def timed_replays(step, steps, torch, replays, dist=None):
     return out
 
 
-def auto_path(M, N, K, group=0):
-    """The kernel family w4a8_gemm's AUTO path takes for a shape (the library's dispatch
-    rule, restated here to label the results): the dp4a GEMV for M <= 2, for M <= 4 when
-    N*K <= 2^25 and for M <= 8 where the int8 kernel does not apply; the int8 tensor-core
-    kernel for M <= 64 (Q4_0, K a multiple of 256); fp16 MMAs (CTA pairs) above."""
-    i8 = group == 0 and M <= 64 and K % 256 == 0
-    if i8:
-        if M <= 2 or (M <= 4 and N * K <= 2 ** 25):
-            return "gemv"
-        return "gemm_i8"
-    if M <= 8:
-        return "gemv"
-    return "gemm_pair" if M > 64 else "gemm_tc"
-
-
 def copies_for(bytes_per_copy: int) -> int:
     return max(2, math.ceil(2 * L2_BYTES / max(1, bytes_per_copy)))
 
@@ -559,7 +544,7 @@ def run_extra(args, torch, w4a8, oracle, inputs, peaks, traffic, dev):
             def kstep(i):
                 qq, dd = sets[i % R]
                 w4a8.w4a8_gemm_prepared(M, K, qq, dd, y, ws)
-        path = auto_path(M, N, K, wl.group if affine else 0)
+        path = w4a8.w4a8_gemm_path(M, N, K, wl.group if affine else 0)
         hbm_bound = path in ("gemv", "gemm_i8")
         entry = {"workload": wl.name, "M": M, "N": N, "K": K, "path": path, "parity": "pass" if ok else "FAIL"}
         if ok:
@@ -634,7 +619,7 @@ def run_epilogue(args, torch, w4a8, oracle, inputs, steps, dev):
         got = y.float().cpu().numpy()[ms, ns].astype(np.float64)
         ok = bool(np.all(np.abs(got - ref) <= 1e-5 * T + np.abs(ref) * 2.0 ** -7))
         entry = {"workload": wl.name + "_bias_bf16out", "M": M, "N": N, "K": K,
-                 "path": auto_path(M, N, K), "epilogue": "f32 bias per column, bf16 output",
+                 "path": w4a8.w4a8_gemm_path(M, N, K), "epilogue": "f32 bias per column, bf16 output",
                  "parity": "pass" if ok else "FAIL"}
         if ok:
             def step(i):

@@ -34,7 +34,9 @@ EXPORTS = ["w4a8_pack_q4_0", "w4a8_quant_act_q8_0", "w4a8_workspace_bytes", "w4a
            "w4a8_pack_affine_nbit", "w4a8_gemm_affine_nbit", "w4a8_gemv_q4_k", "w4a8_gemv_q4_k_backward",
            "w4a8_q4_k_backward_workspace_bytes", "w4a8_prepare_act",
            "w4a8_gemm_prepared", "w4a8_gemm_affine_prepared", "w4a8_gemm_noalloc", "w4a8_last_device_error",
-           "w4a8_last_cuda_error_string", "w4a8_status_string", "w4a8_selftest_bounded_wait"]
+           "w4a8_last_cuda_error_string", "w4a8_status_string", "w4a8_selftest_bounded_wait",
+           "w4a8_gemm_path"]
+KERNEL_NAMES = {1: "gemv", 2: "gemm_i8", 3: "gemm_tc", 4: "gemm_pair"}
 
 
 class W4A8Error(RuntimeError):
@@ -78,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "w4a8_gemm_noalloc": (I, [I, I, I, P, I, P, P, P, P]),
         "w4a8_last_device_error": (I, []),
         "w4a8_selftest_bounded_wait": (I, [ctypes.c_ulonglong, P, P]),
+        "w4a8_gemm_path": (I, [I, I, I, I, I]),
         "w4a8_status_string": (ctypes.c_char_p, [I]),
         "w4a8_last_cuda_error_string": (ctypes.c_char_p, []),
     }
@@ -307,6 +310,15 @@ def w4a8_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
     _check("w4a8_selftest_bounded_wait",
            load_library().w4a8_selftest_bounded_wait(int(limit_ns), ctypes.byref(out), _stream(stream)))
     return int(out.value)
+
+
+def w4a8_gemm_path(M: int, N: int, K: int, group: int = 0, path: int = 0) -> str:
+    """The kernel family the matmul of this shape runs ("gemv", "gemm_i8", "gemm_tc",
+    "gemm_pair"); raises ValueError for a shape the call would reject."""
+    k = int(load_library().w4a8_gemm_path(M, N, K, group, path))
+    if k not in KERNEL_NAMES:
+        raise ValueError(f"no kernel for M={M} N={N} K={K} group={group} path={path}")
+    return KERNEL_NAMES[k]
 
 
 def w4a8_last_cuda_error_string() -> str:

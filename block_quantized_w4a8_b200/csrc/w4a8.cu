@@ -977,6 +977,17 @@ size_t w4a8_workspace_bytes(int M, int N, int K, int group) {
     return a > b ? a : b;
 }
 
+int w4a8_gemm_path(int M, int N, int K, int group, w4a8_path path) {
+    if (!dims_ok(M, N) || !dims_ok(K, 1) || (K % 32) != 0) return 0;
+    if (group != 0 && ((group != 32 && group != 64 && group != 128) || (K % group) != 0)) return 0;
+    if (path != W4A8_PATH_AUTO && path != W4A8_PATH_GEMV && path != W4A8_PATH_GEMM) return 0;
+    if (use_gemv(M, N, K, group, path)) return W4A8_KERNEL_GEMV;
+    if (group == 0 && use_i8(M, K, group)) return W4A8_KERNEL_TC_INT8;
+    if (tc_token_tile(M) <= 64) return W4A8_KERNEL_TC_FP16;
+    const int E = group == 0 ? K / 32 : K / group;
+    return (E * 2) % 16 == 0 ? W4A8_KERNEL_TC_PAIR : W4A8_KERNEL_TC_FP16;
+}
+
 w4a8_status w4a8_gemm_ex(int M, int N, int K, const void* x, w4a8_dtype dtype, const uint8_t* qs,
                          const uint16_t* d_fp16, float* y, void* ws, size_t ws_bytes, w4a8_path path,
                          cudaStream_t stream) {

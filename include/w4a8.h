@@ -104,6 +104,24 @@ w4a8_status w4a8_quant_act_q8_0(const void* x, w4a8_dtype dtype, int M, int K,
 size_t w4a8_workspace_bytes(int M, int N, int K, int group);
 
 /*
+ * Which kernel family w4a8_gemm (group = 0) or w4a8_gemm_affine (group = 32, 64 or 128)
+ * runs for a shape on `path` (host logic only: no device work). The choice is the
+ * M-based dispatch between the memory-bound small-M path and the tensor-core path (tract
+ * PR #2432, follow-up on the decode regime; MLX PR #4802, introduction: its int8 kernel
+ * only from M = 32), with the crossover measured on B200. Returns W4A8_KERNEL_GEMV (dp4a GEMV), W4A8_KERNEL_TC_INT8
+ * (tcgen05 kind::i8, tokens as the MMA's N), W4A8_KERNEL_TC_FP16 (tcgen05 kind::f16, one
+ * CTA), W4A8_KERNEL_TC_PAIR (kind::f16 on CTA pairs), or 0 for sizes, groups or paths the
+ * call would reject.
+ */
+enum {
+    W4A8_KERNEL_GEMV = 1,
+    W4A8_KERNEL_TC_INT8 = 2,
+    W4A8_KERNEL_TC_FP16 = 3,
+    W4A8_KERNEL_TC_PAIR = 4
+};
+int w4a8_gemm_path(int M, int N, int K, int group, w4a8_path path);
+
+/*
  * y = x . W^T with W in Q4_0 (from w4a8_pack_q4_0) and x quantised to Q8_0 inside the
  * call: y[m][n] = sum_b f32(d_w[n][b]) * d_x[m][b] * D[m][n][b], with
  * D = sum_{j<32} (q_w - 8) * q_x computed exactly. The sum over blocks is taken in f32;

@@ -183,6 +183,34 @@ def test_checked_build_exports_the_same_boundary():
     assert chk.w4a8_status_string(8) == b"W4A8_ERR_CHECK"
 
 
+@pytest.mark.parametrize("M,N,K,group,path,want", [
+    (1, 4096, 4096, 0, 0, "gemv"),            # decode
+    (2, 4096, 14336, 0, 0, "gemv"),
+    (3, 4096, 14336, 0, 0, "gemm_i8"),        # large weights: the int8 kernel from M = 3
+    (3, 4096, 4096, 0, 0, "gemv"),            # small weights: the GEMV up to M = 4
+    (4, 2048, 8192, 0, 0, "gemv"),
+    (5, 4096, 4096, 0, 0, "gemm_i8"),
+    (64, 4096, 4096, 0, 0, "gemm_i8"),
+    (65, 4096, 4096, 0, 0, "gemm_pair"),      # 128-token tiles on CTA pairs
+    (16, 1536, 384, 0, 0, "gemm_tc"),         # K not a multiple of 256: no int8 kernel
+    (8, 1536, 384, 0, 0, "gemv"),
+    (200, 333, 800, 0, 0, "gemm_tc"),         # K/32 = 25 scales per row: no TMA pitch for pairs
+    (1, 4096, 4096, 0, 2, "gemm_i8"),         # forced tensor path
+    (300, 4096, 4096, 0, 1, "gemv"),          # forced GEMV
+    (8, 4096, 4096, 64, 0, "gemv"),           # affine: the GEMV up to M = 8
+    (9, 4096, 4096, 64, 0, "gemm_tc"),
+    (1024, 4096, 4096, 128, 0, "gemm_pair"),
+])
+def test_gemm_path_rule(lib, M, N, K, group, path, want):
+    """The dispatch (host logic) at the measured crossovers and the format limits."""
+    assert w4a8.w4a8_gemm_path(M, N, K, group, path) == want
+
+
+def test_gemm_path_rejects(lib):
+    for args in [(0, 8, 32, 0, 0), (8, 8, 48, 0, 0), (8, 8, 128, 16, 0), (8, 8, 96, 64, 0), (8, 8, 32, 0, 7)]:
+        assert lib.w4a8_gemm_path(*args) == 0
+
+
 def test_selftest_hook_argument_errors(lib):
     """The failure-path self-test rejects its arguments before touching the device."""
     P = ctypes.c_void_p
