@@ -221,30 +221,6 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Named barrier that also ANDs a predicate over the participating threads.
-__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r)
-        : "r"(uint32_t(v)), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
-// Group-wide wait: one thread of the group polls the mbarrier, the others block on a
-// named barrier, so only one warp of the group spends issue slots while waiting. All
-// threads of the group must call it together; the barrier's AND hands every one of them
-// the leader's result, so the group never splits.
-__device__ __forceinline__ bool bounded_wait_group(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                                   bool leader, uint32_t barrier_id, uint32_t nthreads) {
-    const bool ok = leader ? bounded_wait(bar, parity, abort) : true;
-    return named_barrier_and(barrier_id, nthreads, ok);
-}
-
 // Warp-wide wait used only to drain asynchronous copies before a CTA exits: waits up to
 // `limit_ns` and reports nothing (the caller has already recorded why it stopped).
 __device__ __noinline__ void drain_wait_warp(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
@@ -424,11 +400,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-// Arrive on a barrier of another CTA of the cluster (address from mapa_shared), releasing
-// this thread's earlier memory operations at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
 // Remote arrive with the default (CTA-scope) release: enough to signal that tensor-memory
 // reads ordered before it by tcgen05.fence::before_thread_sync are done. The cluster-
 // scope release costs several hundred cycles more per arrival.
@@ -510,17 +481,6 @@ __device__ __forceinline__ void tmem_wait_ld64(uint32_t (&r)[64]) {
                  : "memory");
 }
 
-// 16 lanes x (8 columns x 4) of 32-bit words (tcgen05.ld.16x256b.x4): thread t gets, for
-// column group j = 0..3, r[4j+0..1] = row (lane base + t/4), columns 8j + 2(t%4) + {0,1}
-// and r[4j+2..3] = row (lane base + t/4 + 8), the same columns.
-__device__ __forceinline__ void tmem_ld_16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
@@ -539,61 +499,7 @@ __device__ __forceinline__ void tmem_ld_32x32_x16(uint32_t taddr, uint32_t (&r)[
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
-// Waits for this thread's outstanding tensor-memory loads; both register sets are
-// threaded through the asm so that no use of them moves above the wait.
-__device__ __forceinline__ void tmem_wait_ld16x2(uint32_t (&a)[16], uint32_t (&b)[16]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
-                   "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]),
-                   "+r"(a[15]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]),
-                   "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]),
-                   "+r"(b[14]), "+r"(b[15])
-                 :
-                 : "memory");
-}
-
-// Packed f32 pair arithmetic (sm_100): acc += d * (x * w), lane-wise on two floats, each
-// operation rounded to nearest (no contraction across the multiply and the FMA).
-__device__ __forceinline__ void fma2_scaled(unsigned long long& acc, uint32_t d0, uint32_t d1, float x0, float x1,
-                                            unsigned long long w2) {
-    asm("{\n\t.reg .b64 dd, xx, ss;\n\t"
-        "mov.b64 dd, {%1, %2};\n\t"
-        "mov.b64 xx, {%3, %4};\n\t"
-        "mul.rn.f32x2 ss, xx, %5;\n\t"
-        "fma.rn.f32x2 %0, dd, ss, %0;\n\t}\n"
-        : "+l"(acc)
-        : "r"(d0), "r"(d1), "f"(x0), "f"(x1), "l"(w2));
-}
-// acc += (d0, d1) * s2, lane-wise, one rounding per lane.
-__device__ __forceinline__ void fma2(unsigned long long& acc, uint32_t d0, uint32_t d1, unsigned long long s2) {
-    asm("{\n\t.reg .b64 dd;\n\t"
-        "mov.b64 dd, {%1, %2};\n\t"
-        "fma.rn.f32x2 %0, dd, %3, %0;\n\t}\n"
-        : "+l"(acc)
-        : "r"(d0), "r"(d1), "l"(s2));
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-    unsigned long long r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-// acc += (p0, p1) * (s0, s1), lane-wise, one rounding per lane.
-__device__ __forceinline__ void fma2_pp(unsigned long long& acc, uint32_t p0, uint32_t p1, uint32_t s0, uint32_t s1) {
-    asm("{\n\t.reg .b64 pp, ss;\n\t"
-        "mov.b64 pp, {%1, %2};\n\t"
-        "mov.b64 ss, {%3, %4};\n\t"
-        "fma.rn.f32x2 %0, pp, ss, %0;\n\t}\n"
-        : "+l"(acc)
-        : "r"(p0), "r"(p1), "r"(s0), "r"(s1));
-}
-// acc += b * (z0, z1)
-__device__ __forceinline__ void fma2_bias(unsigned long long& acc, float z0, float z1, unsigned long long b2) {
-    asm("{\n\t.reg .b64 zz;\n\t"
-        "mov.b64 zz, {%1, %2};\n\t"
-        "fma.rn.f32x2 %0, zz, %3, %0;\n\t}\n"
-        : "+l"(acc)
-        : "f"(z0), "f"(z1), "l"(b2));
-}
+// Two floats as one 64-bit register pair (the operand of packed f32x2 instructions) and back.
 __device__ __forceinline__ unsigned long long pack2(float a, float b) {
     unsigned long long r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
@@ -602,12 +508,6 @@ __device__ __forceinline__ unsigned long long pack2(float a, float b) {
 __device__ __forceinline__ void unpack2(unsigned long long v, float& a, float& b) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
 }
-
-// Per-warpgroup register budget changes (all warps of a warpgroup execute them).
-template <int N>
-__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
-template <int N>
-__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ float warp_max8(float v) {  // max over aligned groups of 8 lanes
