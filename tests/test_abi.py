@@ -171,6 +171,19 @@ def test_q4_k_argument_errors(lib):
     assert lib.w4a8_q4_k_backward_workspace_bytes(1, 8, 256) == 16      # one row range: no partials
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (2, 4096, 4096), (1, 14336, 4096), (1, 4096, 14336),
+                                   (5, 100000, 256), (1, 64, 512), (3, 20, 1024)])
+def test_q4_k_backward_workspace(lib, M, N, K):
+    """Row ranges of the Q4_K backward (148 SMs without a GPU): about one CTA per SM over
+    the K/256 super-block columns, at least 16 rows per range, at most 512 rows per range
+    (the bound on a lane's chain of sums); partial sums of min(M, 2) tokens per range."""
+    nb = K // 256
+    R = min(-(-148 // nb), -(-N // 16))
+    R = max(R, -(-N // 512), 1)
+    want = R * min(M, 2) * K * 4 if R > 1 else 16
+    assert lib.w4a8_q4_k_backward_workspace_bytes(M, N, K) == want
+
+
 def test_checked_build_exports_the_same_boundary():
     """The checked variant (-DW4A8_CHECKED: device-side checks of each copy's alignment,
     reported as W4A8_ERR_CHECK) builds and exports every declared entry point."""
