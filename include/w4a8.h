@@ -289,8 +289,10 @@ w4a8_status w4a8_gemm_affine_nbit(int M, int N, int K, int group, int bits, cons
  *                           current device's SM count (query it with that device current);
  *                           it is 16 when the shape needs a single row range, and then
  *                           `ws` may also be NULL. Returns 0 for invalid sizes.
- * Sums are taken in f32 with fused multiply-adds; each output is within a few units of
- * 2^-24 * (terms per chain) of the exact value relative to sum |terms|.
+ * Each weight is dequantised as the page's d1 * q - m1 rounded once (d1 = d * sc, m1 = dmin
+ * * m, both exact in f32); sums are taken in f32 in short chains (forward: 32 products,
+ * then a row's super-blocks, then a warp; backward: at most 512 rows per range, ranges
+ * added in groups of 16), so each output is within 1e-5 * sum |terms| of the exact value.
  * All pointers device memory, 16-byte aligned, caller-owned; async on `stream`.
  * Errors: INVALID_ARG (sizes, K % 256, null), MISALIGNED, WORKSPACE, CUDA.
  */
