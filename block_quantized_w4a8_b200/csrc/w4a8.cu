@@ -700,16 +700,20 @@ w4a8_status make_epilogue(const w4a8_epilogue* in, Epilogue* out) {
 }
 
 // Whether AUTO takes the GEMV. Q4_0 shapes with the int8 tensor-core kernel switch at the
-// per-call times measured on B200 (weights streamed from HBM): the tensor kernel's time is
-// nearly flat in M up to 16 tokens while the GEMV's grows with M, so it wins from M = 3 on
-// 4096 x 14336 and 14336 x 4096 (at M = 4: 15.7 vs 24.0 us) and from M = 5 on 4096 x 4096
-// and 2048 x 8192 (at M = 4 the GEMV's 8.7 us beats 10.0 us). N < 0: N is not known (the
-// prepare / contract pair), and the rule takes M and K only.
+// per-call times measured on B200 (weights streamed from HBM, M = 2..8): the tensor
+// kernel's time is nearly flat in M up to 16 tokens while the GEMV's grows with M, so it
+// wins from M = 3 on K x N = 4096 x 14336 (M = 2: 15.1 vs 15.8 us, M = 3: 20.6 vs 15.7), from
+// M = 2 on 14336 x 4096 (17.7 vs 16.4: the long rows cost the GEMV more), and from M = 5 on
+// 4096 x 4096 and 8192 x 2048 (M = 4: 8.2 vs 10.0 and 9.1 vs 10.9; M = 5: 14.0 vs 10.1).
+// N < 0: N is not known (the prepare / contract pair), and the rule takes M and K only.
 inline bool use_gemv(int M, int N, int K, int group, w4a8_path path) {
     if (path != W4A8_PATH_AUTO) return path == W4A8_PATH_GEMV;
     if (!use_i8(M, K, group)) return M <= kGemvMaxM;
     if (N < 0) return M <= 3;
-    return M <= 2 || (M <= 4 && int64_t(N) * K <= (int64_t(1) << 25));
+    const bool small = int64_t(N) * K <= (int64_t(1) << 25);
+    if (M == 1) return true;
+    if (M == 2) return K <= 8192 || small;
+    return M <= 4 && small;
 }
 
 // Quantise x into the workspace layout of the chosen path.

@@ -133,8 +133,9 @@ int w4a8_gemm_path(int M, int N, int K, int group, w4a8_path path);
  *            K, 0) bytes (or at least the path's minimum, see there), owned by the
  *            caller; contents on entry are ignored and are garbage afterwards. Calls
  *            that share a workspace must be ordered on one stream.
- * Paths (AUTO): the dp4a GEMV for M <= 2, for M <= 4 when N * K <= 2^25, and for
- * M <= 8 when K is not a multiple of 256; otherwise tensor cores: int8 MMAs on the
+ * Paths (AUTO): the dp4a GEMV for M = 1, for M = 2 when K <= 8192, for M <= 4 when
+ * N * K <= 2^25, and for M <= 8 when K is not a multiple of 256; otherwise tensor
+ * cores: int8 MMAs on the
  * original codes for M <= 64 (K a multiple of 256), fp16 MMAs on CTA pairs above.
  * Scale range: the fp16 tensor-core kernels hold d_w * (q - 8) exactly as two fp16 values
  * formed by one fused multiply-add each, which requires |d_w| < 2728 (weights of magnitude

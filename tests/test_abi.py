@@ -198,7 +198,8 @@ def test_checked_build_exports_the_same_boundary():
 
 @pytest.mark.parametrize("M,N,K,group,path,want", [
     (1, 4096, 4096, 0, 0, "gemv"),            # decode
-    (2, 4096, 14336, 0, 0, "gemv"),
+    (2, 14336, 4096, 0, 0, "gemv"),           # K x N = 4096 x 14336: the GEMV at M = 2
+    (2, 4096, 14336, 0, 0, "gemm_i8"),        # K x N = 14336 x 4096: the long rows favour the int8 kernel
     (3, 4096, 14336, 0, 0, "gemm_i8"),        # large weights: the int8 kernel from M = 3
     (3, 4096, 4096, 0, 0, "gemv"),            # small weights: the GEMV up to M = 4
     (4, 2048, 8192, 0, 0, "gemv"),
