@@ -274,6 +274,28 @@ def test_sweep_full_size_sampled(wl):
     check_tol(y[ms, ns], yref, T, wl.name)
 
 
+CROSSOVER = [inputs.Workload(f"crossover_m{M}_k{K}_n{N}", M=M, K=K, N=N, seed=M + N)
+             for K, N in inputs.SWEEP_SHAPES + [(4096, 4096)] for M in (2, 4, 5)]
+
+
+@pytest.mark.parametrize("wl", CROSSOVER, ids=lambda w: w.name)
+def test_dispatch_crossover_sampled(wl):
+    """At the GEMV / int8-kernel crossover (M = 2..5) the AUTO call agrees with the
+    oracle, and with the path the dispatch rule names forced explicitly: the two paths
+    give the same result up to the tolerance, whichever the rule picks."""
+    x, w = inputs.make(wl)
+    qs, d = w4a8.pack_q4_0(dev(w))
+    rqx, rdx, _ = oracle.quant_act_q8_0(x.float().numpy())
+    rqs, rd = oracle.pack_q4_0(w.numpy())
+    ms, ns = inputs.sample_indices(wl.M, wl.N, 1000, seed=wl.M * 7 + wl.K)
+    yref, T = oracle.gemm_q4_0_sampled(rqx, rdx, rqs, rd, ms, ns)
+    chosen = w4a8.w4a8_gemm_path(wl.M, wl.N, wl.K)
+    for path in ("auto", "gemv", "gemm"):
+        y = as_np(w4a8.gemm(dev(x), qs, d, path=PATHS[path]))
+        check_tol(y[ms, ns], yref, T, f"{wl.name} {path} (auto: {chosen})")
+        assert w4a8.w4a8_last_device_error() == 0
+
+
 # ------------------------------------------------------------------ affine
 AFFINE_SHAPES = [(1, 64, 128), (3, 300, 640), (8, 256, 1024), (20, 128, 640), (32, 256, 1024), (64, 1536, 384),
                  (200, 333, 1280), (130, 128, 4096), (300, 333, 1024), (200, 512, 4096)]
