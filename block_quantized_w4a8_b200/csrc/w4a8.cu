@@ -4,7 +4,9 @@
 
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -35,6 +37,65 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline bool dims_ok(int a, int b) { return a > 0 && b > 0 && a <= W4A8_MAX_DIM && b <= W4A8_MAX_DIM; }
+
+// Unique ID of the calling thread's current CUDA context (false when there is none, or
+// when the driver does not offer the query).
+bool current_context_id(unsigned long long* id) {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` in the calling thread's current
+// context, once per kernel and context. The attribute belongs to the context's copy of the
+// kernel: a context created after cudaDeviceReset starts without it, so each record keeps
+// the ID of the context it was set in, and the attribute is set again whenever the current
+// context has no record (or cannot be identified). The records are read and written under
+// a lock, so first calls from several host threads do not race.
+cudaError_t smem_limit_once(const void* func, int bytes) {
+    struct Rec {
+        const void* func;
+        unsigned long long ctx;
+        int bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Rec> recs;
+    unsigned long long id = 0;
+    const bool known = current_context_id(&id);
+    std::lock_guard<std::mutex> lock(mu);
+    if (known)
+        for (const Rec& r : recs)
+            if (r.func == func && r.ctx == id && r.bytes >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess || !known) return e;
+    for (Rec& r : recs)
+        if (r.func == func && r.ctx == id) {
+            r.bytes = bytes;
+            return e;
+        }
+    recs.push_back({func, id, bytes});
+    return e;
+}
+
+template <typename Kernel>
+cudaError_t smem_limit_once(Kernel* kernel, int bytes) {
+    return smem_limit_once(reinterpret_cast<const void*>(kernel), bytes);
+}
 
 // Last CUDA error a call of this thread turned into W4A8_ERR_CUDA.
 thread_local cudaError_t t_last_cuda_error = cudaSuccess;
@@ -188,34 +249,27 @@ constexpr size_t kGemv2MaxSmem = 160 * 1024;
 constexpr int64_t kFuseMaxElems = 16384;
 
 int sm_count() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];  // zero until filled; every filler stores the same value
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int v = 0;
+    int v = cached[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-        cached[dev] = v;
+        cached[dev].store(v, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return v;
 }
 
 inline int gemv_mt(int mc) { return mc == 1 ? 1 : mc == 2 ? 2 : mc <= 4 ? 4 : 8; }
 
-// Launch one persistent-GEMV instantiation (sets its shared-memory limit once per device).
+// Launch one persistent-GEMV instantiation (sets its shared-memory limit once per context).
 template <int MT, int FMT, int XMODE>
 cudaError_t launch_gemv2(int M, int N, int K, int group, const void* x, const int8_t* qx, const float* dx,
                          const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb, void* y,
                          const Epilogue& epi, cudaStream_t stream) {
-    static bool configured[64] = {false};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
     const size_t smem = gemv2_smem_bytes(MT, K);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv2_kernel<MT, FMT, XMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(kGemv2MaxSmem));
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(gemv2_kernel<MT, FMT, XMODE>, int(kGemv2MaxSmem));
+    if (ea != cudaSuccess) return ea;
     const int64_t ctas = cdiv(N, kGemv2Warps);
     const dim3 grid(unsigned(ctas < sm_count() ? ctas : sm_count()));
     return launch_pdl(gemv2_kernel<MT, FMT, XMODE>, grid, dim3(kGemv2Threads), smem, stream, M, N, K, group, x, qx,
@@ -289,15 +343,8 @@ template <int MT, int FMT, bool QX, int XS>
 cudaError_t launch_gv(const GvPlan& p, int M, int N, int K, int group, const void* x, int xbf16, const int8_t* qx,
                       const float* dx, const int32_t* sx, const uint8_t* wq, const uint16_t* ws, const uint16_t* wb,
                       void* y, const Epilogue& epi, cudaStream_t stream) {
-    static bool configured[64] = {false};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gv::gemv_resident_kernel<MT, FMT, QX, XS>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGvSmemMax));
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(gv::gemv_resident_kernel<MT, FMT, QX, XS>, int(kGvSmemMax));
+    if (ea != cudaSuccess) return ea;
     return launch_pdl(gv::gemv_resident_kernel<MT, FMT, QX, XS>, dim3(unsigned(p.grid)),
                       dim3(gv::warps_for(MT) * 32), p.smem, stream, M, N, K, group, x, xbf16, qx, dx, sx, wq, ws, wb,
                       y, epi, p.lnsw);
@@ -473,16 +520,14 @@ w4a8_status run_splitk_reduce(const float* part, int ks, int M, int N, void* y, 
 // cuTensorMapEncodeTiled, resolved once through the runtime (no link against the driver
 // library).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {  // initialised once, thread-safe
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        return PFN_cuTensorMapEncodeTiled_v12000(nullptr);
+    }();
     return fn;
 }
 
@@ -507,16 +552,8 @@ w4a8_status launch_gemm_tc(int M, int N, int K, int group, const TcWs& w, const 
                            const uint16_t* wb, void* y, const Epilogue& epi, bool pdl, size_t work_bytes,
                            cudaStream_t stream) {
     using Gm = tc::Geo<FMT, TOKL, MN>;
-    static bool configured[64] = {false};
-    int dev = 0;
-    const cudaError_t ed = cudaGetDevice(&dev);
-    if (ed != cudaSuccess) return cuda_status(ed);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_tc_kernel<FMT, TOKL, MN>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM_BYTES);
-        if (ea != cudaSuccess) return cuda_status(ea);
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(tc::gemm_tc_kernel<FMT, TOKL, MN>, Gm::SMEM_BYTES);
+    if (ea != cudaSuccess) return cuda_status(ea);
     // Tensor maps of the packed weights: codes as bytes [N][K/2] in boxes of 16 bytes (one
     // quant block) x NW rows; scales (affine: scales and biases) as 16-bit [N][E] in boxes
     // of 8 x NW, fetched by TMA only when the row pitch 2E is a multiple of 16 bytes.
@@ -554,16 +591,8 @@ w4a8_status launch_gemm_pair(int M, int N, int K, int group, const TcWs& w, cons
                              const uint16_t* wb, void* y, const Epilogue& epi, bool pdl, size_t work_bytes,
                              cudaStream_t stream) {
     using Gm = tc::PairGeo<FMT>;
-    static bool configured[64] = {false};
-    int dev = 0;
-    const cudaError_t ed = cudaGetDevice(&dev);
-    if (ed != cudaSuccess) return cuda_status(ed);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(tc::gemm_pair_kernel<FMT>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::SMEM_BYTES);
-        if (ea != cudaSuccess) return cuda_status(ea);
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(tc::gemm_pair_kernel<FMT>, Gm::SMEM_BYTES);
+    if (ea != cudaSuccess) return cuda_status(ea);
     CUtensorMap tq, tsc, tbi;
     memset(&tbi, 0, sizeof(tbi));
     const int E = (FMT == 0) ? K / 32 : K / group;  // scales per row (a multiple of 8 here)
@@ -592,16 +621,8 @@ template <int MN>
 w4a8_status launch_gemm_i8(int M, int N, int K, const TcWs& w, const uint8_t* wq, const uint16_t* ws, void* y,
                            const Epilogue& epi, bool pdl, size_t work_bytes, cudaStream_t stream) {
     using Gm = i8::Geo<MN>;
-    static bool configured[64] = {false};
-    int dev = 0;
-    const cudaError_t ed = cudaGetDevice(&dev);
-    if (ed != cudaSuccess) return cuda_status(ed);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(i8::gemm_i8_kernel<MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    Gm::SMEM_BYTES);
-        if (ea != cudaSuccess) return cuda_status(ea);
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(i8::gemm_i8_kernel<MN>, Gm::SMEM_BYTES);
+    if (ea != cudaSuccess) return cuda_status(ea);
     // Codes as bytes [N][K/2] in boxes of 128 bytes (8 quant blocks) x 128 rows, 128-byte
     // swizzle (K is a multiple of 256: every stage is one whole box).
     CUtensorMap tq;
@@ -830,16 +851,8 @@ inline size_t q4k_bwd_bytes(int M, int N, int K) {
 template <int MT>
 w4a8_status launch_q4k_bwd(int N, int K, const float* dy, const uint8_t* w, float* out, int R, cudaStream_t stream) {
     constexpr size_t smem = q4k::bwd_smem_bytes(MT);
-    static bool configured[64] = {false};
-    int dev = 0;
-    const cudaError_t ed = cudaGetDevice(&dev);
-    if (ed != cudaSuccess) return cuda_status(ed);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(q4k::bwd_stream_kernel<MT>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (ea != cudaSuccess) return cuda_status(ea);
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(q4k::bwd_stream_kernel<MT>, int(smem));
+    if (ea != cudaSuccess) return cuda_status(ea);
     // the weights as 8-byte elements [N][K/256 * 18], one box = one super-block column of 64 rows
     CUtensorMap tm;
     const uint64_t cols = uint64_t(K / 256) * (q4k::kBlockBytes / 8);
@@ -853,16 +866,8 @@ w4a8_status launch_q4k_bwd(int N, int K, const float* dy, const uint8_t* w, floa
 template <int MT, int MINB>
 w4a8_status launch_q4k_stream_b(int N, int K, const float* x, const uint8_t* w, float* y, const q4k::StreamPlan& sp,
                                 cudaStream_t stream) {
-    static bool configured[64] = {false};
-    int dev = 0;
-    const cudaError_t ed = cudaGetDevice(&dev);
-    if (ed != cudaSuccess) return cuda_status(ed);
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        const cudaError_t ea = cudaFuncSetAttribute(q4k::fwd_stream_kernel<MT, MINB>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(tc::SMEM_LIMIT));
-        if (ea != cudaSuccess) return cuda_status(ea);
-        configured[dev] = true;
-    }
+    const cudaError_t ea = smem_limit_once(q4k::fwd_stream_kernel<MT, MINB>, int(tc::SMEM_LIMIT));
+    if (ea != cudaSuccess) return cuda_status(ea);
     const int G = N < sm_count() ? N : sm_count();
     return cuda_status(launch_pdl(q4k::fwd_stream_kernel<MT, MINB>, dim3(unsigned(G)), dim3(q4k::kStreamThreads),
                                   sp.smem, stream, MT, N, K, x, w, y, sp.kc, sp.nst));
@@ -1104,29 +1109,6 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_
 }  // extern "C"
 
 namespace {
-
-// Unique ID of the calling thread's current CUDA context (false when there is none, or
-// when the driver does not offer the query).
-bool current_context_id(unsigned long long* id) {
-    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
-    static PFN_cuCtxGetId_v12000 get_id = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-        p = nullptr;
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-    });
-    if (!get_current || !get_id) return false;
-    CUcontext ctx = nullptr;
-    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
-    return get_id(ctx, id) == CUDA_SUCCESS;
-}
 
 // Device address of g_noalloc_scratch in the current context of device `dev`. The address
 // belongs to a context, not to a device: after cudaDeviceReset the next context loads the
