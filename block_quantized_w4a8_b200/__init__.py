@@ -46,6 +46,42 @@ class W4A8Error(RuntimeError):
         self.status = status
 
 
+class Epilogue(ctypes.Structure):
+    """w4a8_epilogue: bias (N values or NULL), its element type, the element type of y."""
+    _fields_ = [("bias", ctypes.c_void_p), ("bias_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+_P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_EPI = ctypes.POINTER(Epilogue)
+# (result type, argument types) of every entry point, in the order include/w4a8.h declares
+# the arguments.
+SIGNATURES = {
+    "w4a8_pack_q4_0": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "w4a8_quant_act_q8_0": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
+    "w4a8_workspace_bytes": (_Z, [_I, _I, _I, _I]),
+    "w4a8_gemm": (_I, [_I, _I, _I, _P, _I, _P, _P, _P, _P, _Z, _P]),
+    "w4a8_gemm_ex": (_I, [_I, _I, _I, _P, _I, _P, _P, _P, _P, _Z, _I, _P]),
+    "w4a8_pack_affine": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "w4a8_gemm_affine": (_I, [_I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "w4a8_gemm_affine_ex": (_I, [_I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _Z, _I, _P]),
+    "w4a8_gemm_epi": (_I, [_I, _I, _I, _P, _I, _P, _P, _EPI, _P, _P, _Z, _I, _P]),
+    "w4a8_gemm_affine_epi": (_I, [_I, _I, _I, _I, _P, _I, _P, _P, _P, _EPI, _P, _P, _Z, _I, _P]),
+    "w4a8_pack_affine_nbit": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "w4a8_gemm_affine_nbit": (_I, [_I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _EPI, _P, _P, _Z, _I, _P]),
+    "w4a8_gemv_q4_k": (_I, [_I, _I, _I, _P, _P, _P, _P]),
+    "w4a8_gemv_q4_k_backward": (_I, [_I, _I, _I, _P, _P, _P, _P, _Z, _P]),
+    "w4a8_q4_k_backward_workspace_bytes": (_Z, [_I, _I, _I]),
+    "w4a8_prepare_act": (_I, [_I, _I, _I, _P, _I, _P, _Z, _I, _P]),
+    "w4a8_gemm_prepared": (_I, [_I, _I, _I, _P, _P, _P, _P, _Z, _I, _P]),
+    "w4a8_gemm_affine_prepared": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _I, _P]),
+    "w4a8_gemm_noalloc": (_I, [_I, _I, _I, _P, _I, _P, _P, _P, _P]),
+    "w4a8_last_device_error": (_I, []),
+    "w4a8_selftest_bounded_wait": (_I, [ctypes.c_ulonglong, _P, _P]),
+    "w4a8_gemm_path": (_I, [_I, _I, _I, _I, _I]),
+    "w4a8_status_string": (ctypes.c_char_p, [_I]),
+    "w4a8_last_cuda_error_string": (ctypes.c_char_p, []),
+}
+
 _lib = None
 
 
@@ -57,34 +93,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise RuntimeError(f"libw4a8 is not built ({path} missing); run __graft_entry__.build()")
     lib = ctypes.CDLL(path)
-    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
-    sigs = {
-        "w4a8_pack_q4_0": (I, [P, I, I, I, P, P, P]),
-        "w4a8_quant_act_q8_0": (I, [P, I, I, I, P, P, P, P]),
-        "w4a8_workspace_bytes": (Z, [I, I, I, I]),
-        "w4a8_gemm": (I, [I, I, I, P, I, P, P, P, P, Z, P]),
-        "w4a8_gemm_ex": (I, [I, I, I, P, I, P, P, P, P, Z, I, P]),
-        "w4a8_pack_affine": (I, [P, I, I, I, I, P, P, P, P]),
-        "w4a8_gemm_affine": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, P]),
-        "w4a8_gemm_affine_ex": (I, [I, I, I, I, P, I, P, P, P, P, P, Z, I, P]),
-        "w4a8_gemm_epi": (I, [I, I, I, P, I, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
-        "w4a8_gemm_affine_epi": (I, [I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
-        "w4a8_pack_affine_nbit": (I, [P, I, I, I, I, I, P, P, P, P]),
-        "w4a8_gemm_affine_nbit": (I, [I, I, I, I, I, P, I, P, P, P, ctypes.POINTER(Epilogue), P, P, Z, I, P]),
-        "w4a8_gemv_q4_k": (I, [I, I, I, P, P, P, P]),
-        "w4a8_gemv_q4_k_backward": (I, [I, I, I, P, P, P, P, Z, P]),
-        "w4a8_q4_k_backward_workspace_bytes": (Z, [I, I, I]),
-        "w4a8_prepare_act": (I, [I, I, I, P, I, P, Z, I, P]),
-        "w4a8_gemm_prepared": (I, [I, I, I, P, P, P, P, Z, I, P]),
-        "w4a8_gemm_affine_prepared": (I, [I, I, I, I, P, P, P, P, P, Z, I, P]),
-        "w4a8_gemm_noalloc": (I, [I, I, I, P, I, P, P, P, P]),
-        "w4a8_last_device_error": (I, []),
-        "w4a8_selftest_bounded_wait": (I, [ctypes.c_ulonglong, P, P]),
-        "w4a8_gemm_path": (I, [I, I, I, I, I]),
-        "w4a8_status_string": (ctypes.c_char_p, [I]),
-        "w4a8_last_cuda_error_string": (ctypes.c_char_p, []),
-    }
-    for name, (res, args) in sigs.items():
+    for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
@@ -92,27 +101,63 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-class Epilogue(ctypes.Structure):
-    """w4a8_epilogue: bias (N values or NULL), its element type, the element type of y."""
-    _fields_ = [("bias", ctypes.c_void_p), ("bias_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
-
-
-def _epilogue(bias: torch.Tensor | None, out_dtype: torch.dtype) -> Epilogue:
-    e = Epilogue()
-    e.bias = _ptr(bias).value if bias is not None else None
-    e.bias_dtype = _dtype(bias) if bias is not None else W4A8_F32
-    e.out_dtype = W4A8_BF16 if out_dtype == torch.bfloat16 else (W4A8_F32 if out_dtype == torch.float32 else 99)
-    return e
-
-
-def _ptr(t: torch.Tensor | None):
-    if t is None:
-        return None
+# ------------------------------------------------------------------ argument checks
+# The C ABI takes bare pointers, so the kernels would read or write past a tensor that is
+# smaller than the layout its call implies, or reach into another GPU's memory. Every
+# pointer argument is therefore checked here against the bytes its layout needs and the
+# device of the call's first tensor, which must be the thread's current CUDA device (the
+# library launches there). A need of 0 defers to the library (a shape or mode it rejects).
+def _device(t: torch.Tensor) -> int:
+    """Device index of the call: that of `t`, which must be the current CUDA device."""
     if not t.is_cuda:
         raise ValueError("libw4a8 takes device tensors")
+    dev = t.get_device()
+    cur = torch.cuda.current_device()
+    if dev != cur:
+        raise ValueError(f"libw4a8: tensors on cuda:{dev} while cuda:{cur} is the current device")
+    return dev
+
+
+def _ptr(t: torch.Tensor | None, dev: int, need: int = 0, name: str = "tensor"):
+    if t is None:
+        return None
+    if t.get_device() != dev:
+        raise ValueError(f"libw4a8: {name} is not on the call's device")
     if not t.is_contiguous():
-        raise ValueError("libw4a8 takes contiguous tensors")
+        raise ValueError(f"libw4a8 takes contiguous tensors ({name})")
+    if t.nbytes < need:
+        raise ValueError(f"libw4a8: {name} holds {t.nbytes} bytes; this call uses {need}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _valid_group(group: int) -> bool:
+    return group in (32, 64, 128)
+
+
+def _q4_0_bytes(N: int, K: int):
+    """Q4_0 weights: packed codes N x K/2 bytes, fp16 scales N x K/32."""
+    return N * (K // 2), N * (K // 32) * 2
+
+
+def _affine_bytes(N: int, K: int, group: int, bits: int = 4):
+    """Affine weights: codes N x K*bits/8 bytes, bf16 scale and bias N x K/group each."""
+    codes = N * (K * bits // 8) if bits in (4, 6, 8) else 0
+    return codes, (N * (K // group) * 2 if _valid_group(group) else 0)
+
+
+def _q4_k_bytes(N: int, K: int) -> int:
+    """Q4_K weights: N rows of K/256 super-blocks of 144 bytes."""
+    return N * (K // 256) * 144
+
+
+def _epilogue(bias: torch.Tensor | None, y: torch.Tensor, N: int, dev: int) -> Epilogue:
+    e = Epilogue()
+    p = _ptr(bias, dev, N * bias.element_size(), "bias") if bias is not None else None
+    e.bias = p.value if p is not None else None
+    e.bias_dtype = _dtype(bias) if bias is not None else W4A8_F32
+    out_dtype = y.dtype
+    e.out_dtype = W4A8_BF16 if out_dtype == torch.bfloat16 else (W4A8_F32 if out_dtype == torch.float32 else 99)
+    return e
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -137,14 +182,20 @@ def _check(fn: str, status: int) -> None:
 # ------------------------------------------------------------------ C ABI, one to one
 def w4a8_pack_q4_0(w: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, stream=None) -> None:
     N, K = w.shape
-    _check("w4a8_pack_q4_0", load_library().w4a8_pack_q4_0(_ptr(w), _dtype(w), N, K, _ptr(qs), _ptr(d), _stream(stream)))
+    dev = _device(w)
+    nq, nd = _q4_0_bytes(N, K)
+    _check("w4a8_pack_q4_0", load_library().w4a8_pack_q4_0(_ptr(w, dev), _dtype(w), N, K, _ptr(qs, dev, nq, "qs"),
+                                                           _ptr(d, dev, nd, "d"), _stream(stream)))
 
 
 def w4a8_quant_act_q8_0(x: torch.Tensor, qx: torch.Tensor, dx: torch.Tensor, sx: torch.Tensor | None = None,
                         stream=None) -> None:
     M, K = x.shape
+    dev = _device(x)
+    nb = M * (K // 32) * 4
     _check("w4a8_quant_act_q8_0",
-           load_library().w4a8_quant_act_q8_0(_ptr(x), _dtype(x), M, K, _ptr(qx), _ptr(dx), _ptr(sx), _stream(stream)))
+           load_library().w4a8_quant_act_q8_0(_ptr(x, dev), _dtype(x), M, K, _ptr(qx, dev, M * K, "qx"),
+                                              _ptr(dx, dev, nb, "dx"), _ptr(sx, dev, nb, "sx"), _stream(stream)))
 
 
 def w4a8_workspace_bytes(M: int, N: int, K: int, group: int = 0) -> int:
@@ -154,26 +205,34 @@ def w4a8_workspace_bytes(M: int, N: int, K: int, group: int = 0) -> int:
 def w4a8_gemm_ex(x, qs, d, y, ws, path: int = PATH_AUTO, stream=None) -> None:
     M, K = x.shape
     N = qs.shape[0]
-    _check("w4a8_gemm_ex", load_library().w4a8_gemm_ex(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d), _ptr(y),
-                                                       _ptr(ws), ws.numel() * ws.element_size(), path,
-                                                       _stream(stream)))
+    dev = _device(x)
+    nq, nd = _q4_0_bytes(N, K)
+    _check("w4a8_gemm_ex", load_library().w4a8_gemm_ex(M, N, K, _ptr(x, dev), _dtype(x), _ptr(qs, dev, nq, "qs"),
+                                                       _ptr(d, dev, nd, "d"), _ptr(y, dev, M * N * 4, "y"),
+                                                       _ptr(ws, dev), ws.nbytes, path, _stream(stream)))
 
 
 def w4a8_gemm(x, qs, d, y, ws, stream=None) -> None:
     M, K = x.shape
     N = qs.shape[0]
-    _check("w4a8_gemm", load_library().w4a8_gemm(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d), _ptr(y), _ptr(ws),
-                                                 ws.numel() * ws.element_size(), _stream(stream)))
+    dev = _device(x)
+    nq, nd = _q4_0_bytes(N, K)
+    _check("w4a8_gemm", load_library().w4a8_gemm(M, N, K, _ptr(x, dev), _dtype(x), _ptr(qs, dev, nq, "qs"),
+                                                 _ptr(d, dev, nd, "d"), _ptr(y, dev, M * N * 4, "y"), _ptr(ws, dev),
+                                                 ws.nbytes, _stream(stream)))
 
 
 def w4a8_gemm_epi(x, qs, d, y, ws, bias=None, path: int = PATH_AUTO, stream=None) -> None:
     """y (f32 or bf16, M x N) = x . W^T + bias (bias: N values, f32 or bf16, or None)."""
     M, K = x.shape
     N = qs.shape[0]
-    epi = _epilogue(bias, y.dtype)
-    _check("w4a8_gemm_epi", load_library().w4a8_gemm_epi(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d),
-                                                         ctypes.byref(epi), _ptr(y), _ptr(ws),
-                                                         ws.numel() * ws.element_size(), path, _stream(stream)))
+    dev = _device(x)
+    nq, nd = _q4_0_bytes(N, K)
+    epi = _epilogue(bias, y, N, dev)
+    _check("w4a8_gemm_epi", load_library().w4a8_gemm_epi(M, N, K, _ptr(x, dev), _dtype(x), _ptr(qs, dev, nq, "qs"),
+                                                         _ptr(d, dev, nd, "d"), ctypes.byref(epi),
+                                                         _ptr(y, dev, M * N * y.element_size(), "y"), _ptr(ws, dev),
+                                                         ws.nbytes, path, _stream(stream)))
 
 
 def w4a8_gemm_affine_epi(x, q, scale, bias_w, y, ws, group: int, bias=None, path: int = PATH_AUTO,
@@ -181,17 +240,24 @@ def w4a8_gemm_affine_epi(x, q, scale, bias_w, y, ws, group: int, bias=None, path
     """Affine weights (scale, bias_w from w4a8_pack_affine) with the output epilogue."""
     M, K = x.shape
     N = q.shape[0]
-    epi = _epilogue(bias, y.dtype)
+    dev = _device(x)
+    nq, ns = _affine_bytes(N, K, group)
+    epi = _epilogue(bias, y, N, dev)
     _check("w4a8_gemm_affine_epi",
-           load_library().w4a8_gemm_affine_epi(M, N, K, group, _ptr(x), _dtype(x), _ptr(q), _ptr(scale), _ptr(bias_w),
-                                               ctypes.byref(epi), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
-                                               path, _stream(stream)))
+           load_library().w4a8_gemm_affine_epi(M, N, K, group, _ptr(x, dev), _dtype(x), _ptr(q, dev, nq, "q"),
+                                               _ptr(scale, dev, ns, "scale"), _ptr(bias_w, dev, ns, "bias_w"),
+                                               ctypes.byref(epi), _ptr(y, dev, M * N * y.element_size(), "y"),
+                                               _ptr(ws, dev), ws.nbytes, path, _stream(stream)))
 
 
 def w4a8_pack_affine_nbit(w, group: int, bits: int, q, scale, bias, stream=None) -> None:
     N, K = w.shape
-    _check("w4a8_pack_affine_nbit", load_library().w4a8_pack_affine_nbit(_ptr(w), _dtype(w), N, K, group, bits,
-                                                                         _ptr(q), _ptr(scale), _ptr(bias),
+    dev = _device(w)
+    nq, ns = _affine_bytes(N, K, group, bits)
+    _check("w4a8_pack_affine_nbit", load_library().w4a8_pack_affine_nbit(_ptr(w, dev), _dtype(w), N, K, group, bits,
+                                                                         _ptr(q, dev, nq, "q"),
+                                                                         _ptr(scale, dev, ns, "scale"),
+                                                                         _ptr(bias, dev, ns, "bias"),
                                                                          _stream(stream)))
 
 
@@ -201,28 +267,36 @@ def w4a8_gemm_affine_nbit(x, q, scale, bias_w, y, ws, group: int, bits: int, bia
     output epilogue (y f32 or bf16; `bias` per column or None)."""
     M, K = x.shape
     N = q.shape[0]
-    epi = _epilogue(bias, y.dtype)
+    dev = _device(x)
+    nq, ns = _affine_bytes(N, K, group, bits)
+    epi = _epilogue(bias, y, N, dev)
     _check("w4a8_gemm_affine_nbit",
-           load_library().w4a8_gemm_affine_nbit(M, N, K, group, bits, _ptr(x), _dtype(x), _ptr(q), _ptr(scale),
-                                                _ptr(bias_w), ctypes.byref(epi), _ptr(y), _ptr(ws),
-                                                ws.numel() * ws.element_size(), path, _stream(stream)))
+           load_library().w4a8_gemm_affine_nbit(M, N, K, group, bits, _ptr(x, dev), _dtype(x), _ptr(q, dev, nq, "q"),
+                                                _ptr(scale, dev, ns, "scale"), _ptr(bias_w, dev, ns, "bias_w"),
+                                                ctypes.byref(epi), _ptr(y, dev, M * N * y.element_size(), "y"),
+                                                _ptr(ws, dev), ws.nbytes, path, _stream(stream)))
 
 
 def w4a8_gemv_q4_k(x, w_q4k, y, stream=None) -> None:
     """y (M, N) f32 = x (M, K) f32 . W^T, W in Q4_K (uint8 (N, K/256*144))."""
     M, K = x.shape
     N = w_q4k.shape[0]
-    _check("w4a8_gemv_q4_k", load_library().w4a8_gemv_q4_k(M, N, K, _ptr(x), _ptr(w_q4k), _ptr(y), _stream(stream)))
+    dev = _device(x)
+    _check("w4a8_gemv_q4_k", load_library().w4a8_gemv_q4_k(M, N, K, _ptr(x, dev), _ptr(w_q4k, dev, _q4_k_bytes(N, K),
+                                                                                          "w_q4k"),
+                                                           _ptr(y, dev, M * N * 4, "y"), _stream(stream)))
 
 
 def w4a8_gemv_q4_k_backward(dy, w_q4k, dx, ws, stream=None) -> None:
     """dx (M, K) f32 = dy (M, N) f32 . W (the input gradient), W in Q4_K."""
     M, N = dy.shape
     K = dx.shape[1]
-    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    dev = _device(dy)
+    nbytes = ws.nbytes if ws is not None else 0
     _check("w4a8_gemv_q4_k_backward",
-           load_library().w4a8_gemv_q4_k_backward(M, N, K, _ptr(dy), _ptr(w_q4k), _ptr(dx),
-                                                  _ptr(ws) if ws is not None else None, nbytes, _stream(stream)))
+           load_library().w4a8_gemv_q4_k_backward(M, N, K, _ptr(dy, dev), _ptr(w_q4k, dev, _q4_k_bytes(N, K), "w_q4k"),
+                                                  _ptr(dx, dev, M * K * 4, "dx"), _ptr(ws, dev), nbytes,
+                                                  _stream(stream)))
 
 
 def w4a8_q4_k_backward_workspace_bytes(M: int, N: int, K: int) -> int:
@@ -246,46 +320,61 @@ def gemv_q4_k_backward(dy, w_q4k, K: int, ws=None, stream=None):
 
 def w4a8_pack_affine(w, group: int, q, scale, bias, stream=None) -> None:
     N, K = w.shape
-    _check("w4a8_pack_affine", load_library().w4a8_pack_affine(_ptr(w), _dtype(w), N, K, group, _ptr(q), _ptr(scale),
-                                                               _ptr(bias), _stream(stream)))
+    dev = _device(w)
+    nq, ns = _affine_bytes(N, K, group)
+    _check("w4a8_pack_affine", load_library().w4a8_pack_affine(_ptr(w, dev), _dtype(w), N, K, group,
+                                                               _ptr(q, dev, nq, "q"), _ptr(scale, dev, ns, "scale"),
+                                                               _ptr(bias, dev, ns, "bias"), _stream(stream)))
 
 
 def w4a8_gemm_affine_ex(x, q, scale, bias, y, ws, group: int, path: int = PATH_AUTO, stream=None) -> None:
     M, K = x.shape
     N = q.shape[0]
+    dev = _device(x)
+    nq, ns = _affine_bytes(N, K, group)
     _check("w4a8_gemm_affine_ex",
-           load_library().w4a8_gemm_affine_ex(M, N, K, group, _ptr(x), _dtype(x), _ptr(q), _ptr(scale), _ptr(bias),
-                                              _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), path,
+           load_library().w4a8_gemm_affine_ex(M, N, K, group, _ptr(x, dev), _dtype(x), _ptr(q, dev, nq, "q"),
+                                              _ptr(scale, dev, ns, "scale"), _ptr(bias, dev, ns, "bias"),
+                                              _ptr(y, dev, M * N * 4, "y"), _ptr(ws, dev), ws.nbytes, path,
                                               _stream(stream)))
 
 
 def w4a8_gemm_affine(x, q, scale, bias, y, ws, group: int, stream=None) -> None:
     M, K = x.shape
     N = q.shape[0]
+    dev = _device(x)
+    nq, ns = _affine_bytes(N, K, group)
     _check("w4a8_gemm_affine",
-           load_library().w4a8_gemm_affine(M, N, K, group, _ptr(x), _dtype(x), _ptr(q), _ptr(scale), _ptr(bias),
-                                           _ptr(y), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+           load_library().w4a8_gemm_affine(M, N, K, group, _ptr(x, dev), _dtype(x), _ptr(q, dev, nq, "q"),
+                                           _ptr(scale, dev, ns, "scale"), _ptr(bias, dev, ns, "bias"),
+                                           _ptr(y, dev, M * N * 4, "y"), _ptr(ws, dev), ws.nbytes, _stream(stream)))
 
 
 def w4a8_prepare_act(x, ws, group: int = 0, path: int = PATH_AUTO, stream=None) -> None:
     M, K = x.shape
-    _check("w4a8_prepare_act", load_library().w4a8_prepare_act(M, K, group, _ptr(x), _dtype(x), _ptr(ws),
-                                                               ws.numel() * ws.element_size(), path, _stream(stream)))
+    dev = _device(x)
+    _check("w4a8_prepare_act", load_library().w4a8_prepare_act(M, K, group, _ptr(x, dev), _dtype(x), _ptr(ws, dev),
+                                                               ws.nbytes, path, _stream(stream)))
 
 
 def w4a8_gemm_prepared(M: int, K: int, qs, d, y, ws, path: int = PATH_AUTO, stream=None) -> None:
     N = qs.shape[0]
-    _check("w4a8_gemm_prepared", load_library().w4a8_gemm_prepared(M, N, K, _ptr(qs), _ptr(d), _ptr(y), _ptr(ws),
-                                                                   ws.numel() * ws.element_size(), path,
-                                                                   _stream(stream)))
+    dev = _device(qs)
+    nq, nd = _q4_0_bytes(N, K)
+    _check("w4a8_gemm_prepared", load_library().w4a8_gemm_prepared(M, N, K, _ptr(qs, dev, nq, "qs"),
+                                                                   _ptr(d, dev, nd, "d"), _ptr(y, dev, M * N * 4, "y"),
+                                                                   _ptr(ws, dev), ws.nbytes, path, _stream(stream)))
 
 
 def w4a8_gemm_affine_prepared(M: int, K: int, group: int, q, scale, bias, y, ws, path: int = PATH_AUTO,
                               stream=None) -> None:
     N = q.shape[0]
+    dev = _device(q)
+    nq, ns = _affine_bytes(N, K, group)
     _check("w4a8_gemm_affine_prepared",
-           load_library().w4a8_gemm_affine_prepared(M, N, K, group, _ptr(q), _ptr(scale), _ptr(bias), _ptr(y),
-                                                    _ptr(ws), ws.numel() * ws.element_size(), path,
+           load_library().w4a8_gemm_affine_prepared(M, N, K, group, _ptr(q, dev, nq, "q"),
+                                                    _ptr(scale, dev, ns, "scale"), _ptr(bias, dev, ns, "bias"),
+                                                    _ptr(y, dev, M * N * 4, "y"), _ptr(ws, dev), ws.nbytes, path,
                                                     _stream(stream)))
 
 
@@ -294,8 +383,11 @@ def w4a8_gemm_noalloc(x, qs, d, y, stream=None) -> None:
     (for callers that may not allocate device memory). Calls must not overlap on the GPU."""
     M, K = x.shape
     N = qs.shape[0]
-    _check("w4a8_gemm_noalloc", load_library().w4a8_gemm_noalloc(M, N, K, _ptr(x), _dtype(x), _ptr(qs), _ptr(d),
-                                                                 _ptr(y), _stream(stream)))
+    dev = _device(x)
+    nq, nd = _q4_0_bytes(N, K)
+    _check("w4a8_gemm_noalloc", load_library().w4a8_gemm_noalloc(M, N, K, _ptr(x, dev), _dtype(x),
+                                                                 _ptr(qs, dev, nq, "qs"), _ptr(d, dev, nd, "d"),
+                                                                 _ptr(y, dev, M * N * 4, "y"), _stream(stream)))
 
 
 def w4a8_last_device_error() -> int:
