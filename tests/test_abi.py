@@ -6,6 +6,8 @@ import os
 import re
 
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import block_quantized_w4a8_b200 as w4a8
 
@@ -218,6 +220,52 @@ def test_checked_build_exports_the_same_boundary():
 def test_gemm_path_rule(lib, M, N, K, group, path, want):
     """The dispatch (host logic) at the measured crossovers and the format limits."""
     assert w4a8.w4a8_gemm_path(M, N, K, group, path) == want
+
+
+shapes = st.tuples(st.integers(1, 5000), st.integers(1, 20000), st.integers(1, 600).map(lambda b: 32 * b),
+                   st.sampled_from([0, 32, 64, 128]))
+
+
+@settings(max_examples=400, deadline=None)
+@given(shape=shapes)
+def test_gemm_path_properties(lib, shape):
+    """Over random valid shapes: AUTO takes one of the four kernel families; the int8
+    kernel only for Q4_0 with K a multiple of 256 and M <= 64, the CTA pairs only above 64
+    tokens; a forced GEMV is always the GEMV and a forced tensor path never is; AUTO
+    follows the measured crossover; and the workspace size is defined."""
+    M, N, K, group = shape
+    if group and K % group:
+        assert lib.w4a8_gemm_path(M, N, K, group, 0) == 0
+        assert lib.w4a8_workspace_bytes(M, N, K, group) == 0
+        return
+    auto = lib.w4a8_gemm_path(M, N, K, group, 0)
+    assert auto in (1, 2, 3, 4)
+    assert lib.w4a8_gemm_path(M, N, K, group, 1) == 1
+    assert lib.w4a8_gemm_path(M, N, K, group, 2) in (2, 3, 4)
+    i8 = group == 0 and K % 256 == 0 and M <= 64
+    if auto == 2 or lib.w4a8_gemm_path(M, N, K, group, 2) == 2:
+        assert i8
+    if auto == 4:
+        assert M > 64
+    small = N * K <= 1 << 25
+    want_gemv = (M == 1 or (M == 2 and (K <= 8192 or small)) or (M <= 4 and small)) if i8 else M <= 8
+    assert (auto == 1) == want_gemv, (M, N, K, group, auto)
+    assert lib.w4a8_workspace_bytes(M, N, K, group) > 0
+
+
+@settings(max_examples=200, deadline=None)
+@given(shape=shapes)
+def test_gemm_path_never_returns_to_the_gemv_as_m_grows(lib, shape):
+    """Once AUTO takes a tensor-core kernel at some M, it does so at every larger M."""
+    _, N, K, group = shape
+    if group and K % group:
+        return
+    seen_tensor = False
+    for M in list(range(1, 70)) + [128, 256, 1024]:
+        auto = lib.w4a8_gemm_path(M, N, K, group, 0)
+        if seen_tensor:
+            assert auto != 1, (M, N, K, group)
+        seen_tensor = seen_tensor or auto != 1
 
 
 def test_gemm_path_rejects(lib):
