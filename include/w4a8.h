@@ -23,6 +23,10 @@
  *  - The kernels never trap, assert or wait without bound. Every internal wait has a
  *    time limit; when one runs out the kernel records W4A8_ERR_DEVICE_TIMEOUT in a
  *    device status word (read it with w4a8_last_device_error) and exits cleanly.
+ *  - Calls run on the calling thread's current device and may come from several host
+ *    threads. The host state the library keeps (each kernel's raised shared-memory limit,
+ *    the no-alloc scratch address) is recorded per CUDA context under a lock, so calls
+ *    keep working in a context created after cudaDeviceReset.
  */
 #ifndef W4A8_H_
 #define W4A8_H_
